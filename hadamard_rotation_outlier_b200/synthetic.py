@@ -1,0 +1,231 @@
+"""Seeded synthetic inputs for the rotate + quantize path.
+
+This module only draws random numbers and converts them to bfloat16 bit
+patterns.  It holds none of the method's arithmetic (no Hadamard transform,
+no scale, no rounding to codes), so both the CUDA path and the CPU oracle can
+take their inputs from it.
+
+Workloads follow the five synthetic configurations this library is measured
+on: activations with about 0.1% of channels ~100x larger (the outlier
+statistic quoted on [Hartmann rotation] §1), Q/K heads and KV-cache rows with
+a few outlier dimensions per head, and heavy-tailed Student-t(3) rows of a
+width that is not a power of two.  Rows are generated in fixed chunks, each
+from its own seed, so any row range can be regenerated without producing the
+whole tensor.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+CHUNK_ROWS = 256
+DEFAULT_SEED = 42
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (round to nearest, ties to even).
+
+    Returns the raw uint16 bit patterns.  Inputs must be finite.
+    """
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    return ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+
+
+@dataclasses.dataclass(frozen=True)
+class Tensor:
+    """One input tensor of a workload: its name, row count and outliers.
+
+    ``outlier_dims`` is the number of outlier columns per head (0 for none);
+    rows ``[h * rows_per_head, (h + 1) * rows_per_head)`` belong to head h.
+    ``outlier_key`` names the seed stream of the outlier columns, so that two
+    tensors (Q and K of one head) can share them.
+    """
+    name: str
+    rows: int
+    heads: int = 1
+    outlier_dims: int = 0
+    outlier_scale: float = 1.0
+    outlier_key: int = 0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    description: str
+    dim: int
+    block: int          # -1: one Hadamard block over the whole row
+    group: int          # -1: one scale per row
+    bits: int
+    with_signs: bool
+    dist: str           # "normal" or "student_t3"
+    tensors: tuple
+    dequant: bool = False
+
+    @property
+    def rows(self) -> int:
+        return sum(t.rows for t in self.tensors)
+
+    @property
+    def elements(self) -> int:
+        return self.rows * self.dim
+
+    def scales_per_row(self) -> int:
+        return self.dim // (self.dim if self.group == -1 else self.group)
+
+    def quant_bytes(self) -> int:
+        """bf16 in + codes out + fp32 scales out, each byte moved once."""
+        n = self.elements
+        codes = n if self.bits == 8 else n // 2
+        return 2 * n + codes + 4 * self.rows * self.scales_per_row()
+
+    def dequant_bytes(self, out_bytes_per_elem: int = 2) -> int:
+        """codes + fp32 scales in + reconstructed values out."""
+        n = self.elements
+        codes = n if self.bits == 8 else n // 2
+        return codes + 4 * self.rows * self.scales_per_row() + out_bytes_per_elem * n
+
+    def with_rows(self, rows_per_tensor: int) -> "Workload":
+        """The same recipe with fewer rows per tensor (for oracle-sized tests).
+
+        Head structure is kept: rows are spread over the same number of heads.
+        """
+        ts = []
+        for t in self.tensors:
+            r = max(t.heads, (rows_per_tensor // t.heads) * t.heads)
+            ts.append(dataclasses.replace(t, rows=r))
+        return dataclasses.replace(self, tensors=tuple(ts))
+
+
+WORKLOADS = {
+    "c1_tok256_h4096_b128_int4": Workload(
+        name="c1_tok256_h4096_b128_int4",
+        description="256 tokens x hidden 4096, N(0,1) with 4 seeded channels x100; "
+                    "block Hadamard 128 (32 blocks), no signs; per-token INT4",
+        dim=4096, block=128, group=-1, bits=4, with_signs=False, dist="normal",
+        tensors=(Tensor("x", 256, 1, 4, 100.0, 1),)),
+    "c2_qk_h32_s8192_d128_int8": Workload(
+        name="c2_qk_h32_s8192_d128_int8",
+        description="Q and K [1,32,8192,128], N(0,1) with 2 outlier dims per head x50 "
+                    "(shared by Q and K); full 128-point Hadamard; per token-head INT8",
+        dim=128, block=-1, group=-1, bits=8, with_signs=False, dist="normal",
+        tensors=(Tensor("q", 32 * 8192, 32, 2, 50.0, 2),
+                 Tensor("k", 32 * 8192, 32, 2, 50.0, 2))),
+    "c3_tok16384_h4096_full_signs_int4": Workload(
+        name="c3_tok16384_h4096_full_signs_int4",
+        description="16384 tokens x hidden 4096, N(0,1) with 4 channels (0.1%) x100; "
+                    "seeded signs then full 4096-point Hadamard; per-token INT4",
+        dim=4096, block=-1, group=-1, bits=4, with_signs=True, dist="normal",
+        tensors=(Tensor("x", 16384, 1, 4, 100.0, 3),)),
+    "c4_kv_h8_t131072_d128_int4_g128": Workload(
+        name="c4_kv_h8_t131072_d128_int4_g128",
+        description="K and V [8,131072,128], N(0,1), K with 4 outlier dims per head x30; "
+                    "128-point Hadamard; INT4 group 128; then dequant + inverse",
+        dim=128, block=128, group=128, bits=4, with_signs=False, dist="normal",
+        tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
+                 Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
+        dequant=True),
+    "c5_tok32768_w11008_b128_signs_int4_g128": Workload(
+        name="c5_tok32768_w11008_b128_signs_int4_g128",
+        description="32768 tokens x 11008 (86 blocks of 128), Student-t(3); seeded signs, "
+                    "block Hadamard 128; INT4 group 128",
+        dim=11008, block=128, group=128, bits=4, with_signs=True, dist="student_t3",
+        tensors=(Tensor("x", 32768, 1, 0, 1.0, 6),)),
+}
+
+WORKLOAD_ORDER = list(WORKLOADS)
+
+
+def outlier_columns(t: Tensor, dim: int, seed: int = DEFAULT_SEED) -> np.ndarray:
+    """Seeded outlier column indices, shape [heads, outlier_dims] (sorted)."""
+    if t.outlier_dims == 0:
+        return np.zeros((t.heads, 0), dtype=np.int64)
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x0D11, t.outlier_key]))
+    cols = [np.sort(rng.choice(dim, size=t.outlier_dims, replace=False)) for _ in range(t.heads)]
+    return np.stack(cols).astype(np.int64)
+
+
+def signs(wl: Workload, seed: int = DEFAULT_SEED):
+    """The seeded +-1 sign vector of a workload (int8 [dim]) or None."""
+    if not wl.with_signs:
+        return None
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x5160, wl.dim]))
+    return (rng.integers(0, 2, size=wl.dim) * 2 - 1).astype(np.int8)
+
+
+def _chunk_values(dist: str, dim: int, n_rows: int, ss: np.random.SeedSequence) -> np.ndarray:
+    rng = np.random.default_rng(ss)
+    if dist == "normal":
+        return rng.standard_normal((n_rows, dim), dtype=np.float32)
+    if dist == "student_t3":
+        return rng.standard_t(3, size=(n_rows, dim)).astype(np.float32)
+    raise ValueError(dist)
+
+
+def _chunk(wl: Workload, ti: int, c: int, seed: int, cols: np.ndarray) -> np.ndarray:
+    t = wl.tensors[ti]
+    r0 = c * CHUNK_ROWS
+    r1 = min(t.rows, r0 + CHUNK_ROWS)
+    ss = np.random.SeedSequence([seed, 0xDA7A, ti, c])
+    v = _chunk_values(wl.dist, wl.dim, r1 - r0, ss)
+    if t.outlier_dims:
+        rows_per_head = t.rows // t.heads
+        heads = np.arange(r0, r1) // rows_per_head
+        for h in np.unique(heads):
+            sel = heads == h
+            v[np.ix_(sel, cols[h])] *= np.float32(t.outlier_scale)
+    return f32_to_bf16_bits(v)
+
+
+def tensor_rows(wl: Workload, ti: int, r0: int, r1: int, seed: int = DEFAULT_SEED,
+                threads: int | None = None) -> np.ndarray:
+    """Rows [r0, r1) of tensor ``ti`` as bfloat16 bits (uint16 [r1-r0, dim])."""
+    t = wl.tensors[ti]
+    if not (0 <= r0 <= r1 <= t.rows):
+        raise ValueError("row range out of bounds")
+    out = np.empty((r1 - r0, wl.dim), dtype=np.uint16)
+    if r1 == r0:
+        return out
+    cols = outlier_columns(t, wl.dim, seed)
+    c0, c1 = r0 // CHUNK_ROWS, (r1 - 1) // CHUNK_ROWS + 1
+
+    def work(c):
+        a = _chunk(wl, ti, c, seed, cols)
+        lo = max(r0, c * CHUNK_ROWS)
+        hi = min(r1, c * CHUNK_ROWS + a.shape[0])
+        out[lo - r0:hi - r0] = a[lo - c * CHUNK_ROWS:hi - c * CHUNK_ROWS]
+
+    n = c1 - c0
+    nthreads = threads or min(n, os.cpu_count() or 1, 32)
+    if nthreads <= 1:
+        for c in range(c0, c1):
+            work(c)
+    else:
+        with ThreadPoolExecutor(nthreads) as ex:
+            list(ex.map(work, range(c0, c1)))
+    return out
+
+
+def tensor(wl: Workload, ti: int, seed: int = DEFAULT_SEED) -> np.ndarray:
+    """A whole input tensor as bfloat16 bits (uint16 [rows, dim])."""
+    return tensor_rows(wl, ti, 0, wl.tensors[ti].rows, seed)
+
+
+def random_bf16(rows: int, dim: int, seed: int, dist: str = "normal",
+                outlier_cols=(), outlier_scale: float = 100.0) -> np.ndarray:
+    """Free-form seeded bf16 input for shape sweeps (uint16 [rows, dim])."""
+    ss = np.random.SeedSequence([seed, 0xF4EE, rows, dim])
+    v = _chunk_values(dist, dim, rows, ss)
+    if len(outlier_cols):
+        v[:, np.asarray(outlier_cols)] *= np.float32(outlier_scale)
+    return f32_to_bf16_bits(v)
+
+
+def random_signs(dim: int, seed: int) -> np.ndarray:
+    """Seeded +-1 int8 sign vector of length ``dim``."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x5161, dim]))
+    return (rng.integers(0, 2, size=dim) * 2 - 1).astype(np.int8)

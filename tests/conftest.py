@@ -1,0 +1,37 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def read_golden(name):
+    """Parse a ``name = v1, v2, ...`` fixture file into {name: [floats]}."""
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = line.split("=", 1)
+            out[key.strip()] = [float(v) for v in val.split(",")]
+    return out
+
+
+@pytest.fixture(scope="session")
+def golden_pages():
+    return read_golden("pages_printed_values.txt")
+
+
+@pytest.fixture(scope="session")
+def golden_hand():
+    return read_golden("hand_worked_examples.txt")

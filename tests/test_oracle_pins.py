@@ -1,0 +1,361 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks one oracle function against something the pages or the
+mathematics fix: values the pages print, hand-worked cases, closed forms,
+library routines (scipy's Sylvester construction) and brute force.  Every test
+here runs on the CPU.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle as O
+from hadamard_rotation_outlier_b200 import synthetic as S
+
+POW2 = [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024]
+
+
+def _popcount_matrix(n):
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    bits = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    return np.where(bits % 2 == 0, 1, -1).astype(np.int64)
+
+
+# ---------------------------------------------------------------- H itself
+
+@pytest.mark.parametrize("n", POW2)
+def test_sylvester_equals_scipy_hadamard(n):
+    # scipy.linalg.hadamard builds the same Sylvester matrix with +-1 entries.
+    ref = scipy.linalg.hadamard(n).astype(np.float64) / math.sqrt(n)
+    np.testing.assert_allclose(O.sylvester(n), ref, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 32, 128])
+def test_sylvester_closed_form_popcount(n):
+    # Textbook closed form: H[i, j] = (-1)^popcount(i & j) / sqrt(n).
+    np.testing.assert_allclose(O.sylvester(n) * math.sqrt(n), _popcount_matrix(n),
+                               rtol=0, atol=1e-12)
+
+
+def test_h2_printed_and_h4_kronecker(golden_pages):
+    h2 = np.array(golden_pages["h2_unnormalised"]).reshape(2, 2)
+    np.testing.assert_allclose(O.sylvester(2) * math.sqrt(2), h2, atol=1e-15)
+    # [Outlier nemesis] §2.1: H4 = H2 (x) H2
+    np.testing.assert_allclose(O.sylvester(4), np.kron(O.sylvester(2), O.sylvester(2)),
+                               atol=1e-15)
+
+
+@pytest.mark.parametrize("n", [2, 4, 16, 64, 256])
+def test_kronecker_recursion(n):
+    np.testing.assert_allclose(O.sylvester(2 * n), np.kron(O.sylvester(2), O.sylvester(n)),
+                               atol=1e-14)
+
+
+@pytest.mark.parametrize("n", POW2 + [4096])
+def test_orthogonal_symmetric_involution(n):
+    H = O.sylvester(n)
+    eye = np.eye(n)
+    np.testing.assert_allclose(H @ H.T, eye, atol=1e-12)
+    np.testing.assert_array_equal(H, H.T)
+    np.testing.assert_allclose(H @ H, eye, atol=1e-12)
+    np.testing.assert_allclose(np.abs(H), 1.0 / math.sqrt(n), rtol=1e-13)
+
+
+def test_sylvester_rejects_non_power_of_two():
+    for n in (0, 3, 6, 12, 11008):
+        with pytest.raises(ValueError):
+            O.sylvester(n)
+
+
+# ------------------------------------------------------------------ FWHT
+
+@pytest.mark.parametrize("n", POW2)
+def test_fwht_brute_force_integers(n):
+    # Brute force: y_j = sum_i x_i (-1)^popcount(i&j), exact in int64.
+    rng = np.random.default_rng(n)
+    x = rng.integers(-1000, 1000, size=(5, n))
+    brute = x @ _popcount_matrix(n)
+    got = O.fwht(x.astype(np.float64)) * math.sqrt(n)
+    if round(math.sqrt(n)) ** 2 == n:
+        # n = 4^k: sqrt(n) is a power of two, so every step is exact.
+        np.testing.assert_array_equal(got, brute.astype(np.float64))
+    else:
+        np.testing.assert_allclose(got, brute, rtol=1e-13, atol=1e-9)
+
+
+@pytest.mark.parametrize("n", [8, 128, 1024])
+def test_fwht_matches_dense_product(n):
+    x = np.random.default_rng(7).standard_normal((9, n))
+    np.testing.assert_allclose(O.fwht(x), x @ O.sylvester(n), rtol=0, atol=1e-12)
+
+
+def test_fwht_matches_dense_sampled_rows_4096():
+    x = np.random.default_rng(8).standard_normal((3, 4096))
+    np.testing.assert_allclose(O.fwht(x), x @ O.sylvester(4096), rtol=0, atol=1e-11)
+
+
+# -------------------------------------------------------------- rotation
+
+@pytest.mark.parametrize("method", ["dense", "fwht"])
+def test_rotation_preserves_norm(method):
+    x = np.random.default_rng(1).standard_normal((16, 512))
+    for block in (-1, 128, 8):
+        y = O.rotate(x, block=block, method=method)
+        np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1),
+                                   rtol=1e-13)
+
+
+@pytest.mark.parametrize("method", ["dense", "fwht"])
+def test_qk_scores_invariant(method):
+    # [Hartmann rotation] §1: Q_rot K_rot^T == Q K^T because H is orthogonal.
+    rng = np.random.default_rng(2)
+    Q = rng.standard_normal((32, 128))
+    K = rng.standard_normal((48, 128))
+    Q[:, 7] *= 50.0
+    K[:, 7] *= 50.0
+    Qr = O.rotate(Q, method=method)
+    Kr = O.rotate(K, method=method)
+    np.testing.assert_allclose(Qr @ Kr.T, Q @ K.T, rtol=0, atol=1e-10 * np.abs(Q @ K.T).max())
+
+
+def test_single_outlier_spreads_to_30_over_64(golden_pages):
+    # [Outlier nemesis] §2.2: one 30 among 4096 -> ~0.47 everywhere; exactly 30/64.
+    n = int(golden_pages["spread_example_dim"][0])
+    x = np.zeros((1, n))
+    x[0, 42] = golden_pages["spread_example_outlier"][0]
+    for method in ("dense", "fwht"):
+        y = O.rotate(x, method=method)
+        np.testing.assert_allclose(np.abs(y), 30.0 / 64.0, rtol=1e-12)
+        assert abs(30.0 / 64.0 - golden_pages["spread_example_magnitude_approx"][0]) < 0.005
+
+
+@pytest.mark.parametrize("dim,B,p", [(512, 128, 300), (96, 32, 5), (4096, 128, 4095)])
+def test_block_diagonal_one_hot_closed_form(dim, B, p):
+    x = np.zeros((1, dim))
+    x[0, p] = 1.0
+    y = O.rotate(x, block=B)[0]
+    b0 = (p // B) * B
+    expect = np.zeros(dim)
+    j = np.arange(B)
+    bits = np.array([bin(int((p % B) & int(v))).count("1") for v in j])
+    expect[b0:b0 + B] = np.where(bits % 2 == 0, 1.0, -1.0) / math.sqrt(B)
+    np.testing.assert_allclose(y, expect, atol=1e-14)
+
+
+def test_signs_apply_before_h_closed_form():
+    # Randomised Hadamard = diag(s) then H: e_p -> s_p * H[p, :] (not s * H[p, :]).
+    n = 64
+    s = S.random_signs(n, 3)
+    for p in (0, 5, 63):
+        x = np.zeros((1, n))
+        x[0, p] = 1.0
+        y = O.rotate(x, signs=s)[0]
+        np.testing.assert_allclose(y, s[p] * O.sylvester(n)[p], atol=1e-15)
+    assert np.any(s < 0) and np.any(s > 0)
+
+
+def test_hand_worked_rotations(golden_hand):
+    g = golden_hand
+    x = np.array([g["ex1_x"]])
+    np.testing.assert_allclose(O.rotate(x)[0], g["ex1_y"], atol=1e-14)
+    np.testing.assert_allclose(O.rotate(x, signs=np.array(g["ex2_signs"]))[0], g["ex2_y"],
+                               atol=1e-14)
+    x3 = np.array([g["ex3_x"]])
+    np.testing.assert_allclose(O.rotate(x3, block=4)[0], g["ex3_block4_y"], atol=1e-14)
+    np.testing.assert_allclose(O.rotate(x3)[0] * math.sqrt(8), g["ex3_full_y_times_sqrt8"],
+                               atol=1e-13)
+
+
+@pytest.mark.parametrize("method", ["dense", "fwht"])
+def test_inverse_undoes_forward(method):
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((6, 384))
+    s = S.random_signs(384, 9)
+    for block in (128, 64, 1):
+        y = O.rotate(x, block=block, signs=s, method=method)
+        np.testing.assert_allclose(O.inverse_rotate(y, block=block, signs=s, method=method), x,
+                                   atol=1e-12)
+
+
+# ------------------------------------------------------------- quantiser
+
+def test_int8_scale_example_from_page(golden_pages):
+    # [Hartmann rotation] §1: 200 among ~1 -> scale 200/127 ~ 1.57; small values -> +-1.
+    y = np.array([[200.0, 1.0, -1.0, 0.9, -1.1, 1.05, -0.95, 1.0]])
+    q, s64, s32, _ = O.quantize(y, 8, -1)
+    assert s64[0, 0] == pytest.approx(golden_pages["int8_scale_example_absmax"][0] / 127.0,
+                                      rel=1e-15)
+    assert round(float(s64[0, 0]), 2) == golden_pages["int8_scale_example_scale_approx"][0]
+    assert q[0, 0] == 127
+    assert set(np.unique(q[0, 1:])) == set(int(v) for v in
+                                           golden_pages["int8_scale_example_small_codes"])
+
+
+def test_hand_worked_quantisation(golden_hand):
+    g = golden_hand
+    y = np.array([g["ex1_y"]])
+    q, s64, s32, _ = O.quantize(y, 4, -1)
+    np.testing.assert_array_equal(q[0], g["ex1_int4_q"])
+    num, den = g["ex1_int4_scale_num_den"]
+    assert s64[0, 0] == pytest.approx(num / den, rel=1e-15)
+    assert s32[0, 0] == np.float32(num / den)
+    q8, _, _, _ = O.quantize(y, 8, -1)
+    np.testing.assert_array_equal(q8[0], g["ex1_int8_q"])
+    np.testing.assert_array_equal(O.pack_int4(q)[0], g["ex1_int4_bytes"])
+    q4, _, _, _ = O.quantize(np.array([g["ex4_y"]]), 4, -1)
+    np.testing.assert_array_equal(q4[0], g["ex4_q"])
+
+
+def test_hand_worked_end_to_end(golden_hand):
+    """rotate_quantize on bf16 inputs against the hand-derived codes and bytes."""
+    g = golden_hand
+
+    def bits(vals):
+        return S.f32_to_bf16_bits(np.array([vals], dtype=np.float32))
+
+    r = O.rotate_quantize(bits(g["ex1_x"]), block=-1, bits=4)
+    np.testing.assert_array_equal(r["codes"][0], g["ex1_int4_bytes"])
+    r = O.rotate_quantize(bits(g["ex1_x"]), block=-1, signs=np.array(g["ex2_signs"], np.int8),
+                          bits=4)
+    np.testing.assert_array_equal(r["q"][0], g["ex2_int4_q"])
+    np.testing.assert_array_equal(r["codes"][0], g["ex2_int4_bytes"])
+    r = O.rotate_quantize(bits(g["ex1_x"]), block=-1, bits=8)
+    np.testing.assert_array_equal(r["codes"][0], np.array(g["ex1_int8_q"], np.int8))
+    r = O.rotate_quantize(bits(g["ex3_x"]), block=4, bits=4, group=4)
+    np.testing.assert_array_equal(r["q"][0], g["ex3_block4_group4_q"])
+    np.testing.assert_array_equal(r["codes"][0], g["ex3_block4_group4_bytes"])
+    np.testing.assert_allclose(r["scales"][0], [5 / 7, 4 / 7], rtol=1e-7)
+    r = O.rotate_quantize(bits(g["ex3_x"]), block=4, bits=4, group=-1)
+    np.testing.assert_array_equal(r["q"][0], g["ex3_block4_rowgroup_q"])
+    r = O.rotate_quantize(bits(g["ex3_x"]), block=-1, bits=8, group=-1)
+    np.testing.assert_array_equal(r["q"][0], g["ex3_full_int8_q"])
+    r = O.rotate_quantize(bits(g["ex4_y"]), block=1, bits=4)
+    np.testing.assert_array_equal(r["q"][0], g["ex4_q"])
+
+
+def test_hand_worked_dequant(golden_hand):
+    g = golden_hand
+    codes = np.array([g["ex1_int4_bytes"]], dtype=np.uint8)
+    scales = np.array([[np.float32(5 / 7)]])
+    xh = O.dequant_rotate_inv(codes, scales, 4, block=-1, bits=4)
+    np.testing.assert_allclose(xh[0] * 14, g["ex1_int4_recon_times_14"], rtol=1e-7)
+    codes = np.array([g["ex2_int4_bytes"]], dtype=np.uint8)
+    xh = O.dequant_rotate_inv(codes, scales, 4, block=-1, bits=4,
+                              signs=np.array(g["ex2_signs"], np.int8))
+    # x*s had y = [-1,5,0,-2]; q = [-1,7,0,-3] -> yhat = [-5/7,5,0,-15/7]
+    yh = np.array([-5 / 7, 5, 0, -15 / 7])
+    expect = (yh @ (O.sylvester(4))) * np.array(g["ex2_signs"])
+    np.testing.assert_allclose(xh[0], expect, rtol=1e-7)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("group", [-1, 16, 64])
+def test_quantiser_bounds(bits, group):
+    rng = np.random.default_rng(bits * 100 + group)
+    y = rng.standard_normal((20, 128)) * rng.uniform(0.01, 100, size=(20, 1))
+    q, s64, s32, v = O.quantize(y, bits, group)
+    qmax = 2 ** (bits - 1) - 1
+    G = 128 if group == -1 else group
+    assert q.min() >= -qmax and q.max() <= qmax
+    sg = np.repeat(s64, G, axis=1)
+    # every value is within half a step of its reconstruction (no clipping ever happens)
+    assert np.all(np.abs(y - q * sg) <= sg / 2 * (1 + 1e-12))
+    # the largest |y| of each group maps to +-qmax
+    yg = y.reshape(20, -1, G)
+    qg = q.reshape(20, -1, G)
+    idx = np.argmax(np.abs(yg), axis=-1)
+    np.testing.assert_array_equal(np.abs(np.take_along_axis(qg, idx[..., None], -1)), qmax)
+    # scales are per group, in column order
+    np.testing.assert_allclose(s64, np.abs(yg).max(-1) / qmax, rtol=1e-15)
+
+
+def test_group_order_and_zero_group():
+    y = np.zeros((1, 24))
+    y[0, 8:16] = np.linspace(-3, 2, 8)
+    y[0, 16:24] = 70.0
+    q, s64, s32, v = O.quantize(y, 8, 8)
+    np.testing.assert_allclose(s64[0], [0.0, 3 / 127, 70 / 127])
+    np.testing.assert_array_equal(q[0, :8], 0)
+    np.testing.assert_array_equal(q[0, 16:], 127)
+    assert q[0, 8] == -127 and np.all(v[0, :8] == 0)
+
+
+def test_int4_pack_roundtrip_all_codes():
+    q = np.array([np.arange(-7, 8), np.arange(7, -8, -1)]).T.reshape(1, -1)
+    packed = O.pack_int4(q)
+    assert packed.shape == (1, q.shape[1] // 2)
+    np.testing.assert_array_equal(O.unpack_int4(packed), q)
+    np.testing.assert_array_equal(O.pack_int4(np.array([[-1, 7, -7, 0]])), [[0x7F, 0x09]])
+
+
+def test_reconstruction_error_bound():
+    rng = np.random.default_rng(11)
+    n = 256
+    x_bits = S.random_bf16(8, n, 5, outlier_cols=[3, 200])
+    for bits in (4, 8):
+        r = O.rotate_quantize(x_bits, block=128, bits=bits, group=64)
+        xh = O.dequant_rotate_inv(r["codes"], r["scales"], n, block=128, bits=bits, group=64)
+        x = O.bf16_bits_to_f64(x_bits)
+        smax = r["scales"].astype(np.float64).max(axis=1)
+        err = np.linalg.norm(x - xh, axis=1)
+        assert np.all(err <= math.sqrt(n) * smax / 2 * 1.0001)
+    del rng
+
+
+def test_rotated_error_far_below_unrotated(golden_pages):
+    """[Outlier nemesis] §2.2 example, orthonormal H (the page's numbers are garbled)."""
+    g = golden_pages
+    rng = np.random.default_rng(int(g["error_example_seed"][0]))
+    w = rng.standard_normal((1, 4096)).astype(np.float32)
+    w[0, int(g["error_example_outlier_index"][0])] = g["error_example_outlier_value"][0]
+    e0 = O.quant_error(w, 4)
+    e1 = O.quant_error(O.rotate(w.astype(np.float64)), 4)
+    assert e1 < e0 / 4
+    e0_8 = O.quant_error(w, 8)
+    e1_8 = O.quant_error(O.rotate(w.astype(np.float64)), 8)
+    assert e1_8 < e0_8 / 4
+
+
+def test_quant_error_definition_small():
+    # hand: x = [2, -1, 0.5], INT4: scale = 2/7; x/scale = [7, -3.5, 1.75]
+    # q = [7, -4, 2] (tie -3.5 -> -4, even); deq = [2, -8/7, 4/7]
+    # |err| = [0, 1/7, 1/14] -> mean = (3/14)/3 = 1/14
+    assert O.quant_error(np.array([2.0, -1.0, 0.5]), 4) == pytest.approx(1 / 14, rel=1e-12)
+
+
+def test_bf16_decode(golden_hand):
+    bits = np.array(golden_hand["bf16_bits"], dtype=np.uint16)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(bits), golden_hand["bf16_values"])
+
+
+def test_half_boundary_distance():
+    v = np.array([0.5, 2.5001, -3.4999, 7.0, -0.0])
+    np.testing.assert_allclose(O.half_boundary_distance(v), [0, 1e-4, 1e-4, 0.5, 0.5], atol=1e-9)
+
+
+def test_planted_mistakes_are_caught(golden_hand):
+    """A wrong sign, index or operand in a copy of the oracle fails the pins above."""
+    g = golden_hand
+    x = np.array([g["ex3_x"]])
+
+    def rotate_sign_after(x, signs):  # signs after H instead of before
+        return O.rotate(x) * signs
+
+    s = np.array([1, -1, 1, -1, 1, -1, 1, -1])
+    assert not np.allclose(rotate_sign_after(x, s), O.rotate(x, signs=s))
+
+    def rotate_wrong_block_axis(x, B):  # blocks taken as strided columns
+        n = x.shape[-1]
+        xb = x.reshape(-1, B, n // B).transpose(0, 2, 1)
+        return (xb @ O.sylvester(B)).transpose(0, 2, 1).reshape(x.shape)
+
+    assert not np.allclose(rotate_wrong_block_axis(x, 4)[0], g["ex3_block4_y"])
+
+    def unnormalised(x):
+        return x @ (O.sylvester(4) * 2)
+
+    assert not np.allclose(unnormalised(np.array([g["ex1_x"]]))[0], g["ex1_y"])
