@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark of the fused Hadamard rotate + quantise step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the hot path over the workload's whole batch: one
+rotate+quantise launch over every input row (plus, for the KV-cache workload,
+one dequantise+inverse launch to bf16).  Inputs are resident in HBM before the
+timed region.  Between timed steps a 256 MiB buffer is written to flush the
+126 MB L2; that write sits outside the CUDA events that time each step.  The
+default workload is the Q/K rotation (2 x [1, 32, 8192, 128] bf16, full
+128-point Hadamard, per token-head INT8).
+
+Multi-GPU (torchrun, one process per GPU): rows are independent, so every rank
+runs its own copy of the workload with no data-path collective ("weak"
+scaling); the process group only provides the barrier and the max over ranks
+of the timed duration.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead (rank 0 only, bounded samples of the same workload).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "c2_qk_h32_s8192_d128_int8"
+METRIC = "fused Hadamard+quantize GB/s (bf16 in→int4/int8 out), % of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
+                "generic": "rq_generic_kernel", "none": None}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=10)
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hadamard_rotation_outlier_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the quantise kernel from a committed ncu summary.
+
+    ``profiles/dram_traffic.txt`` holds lines ``workload source_hash bytes``;
+    the figure is used only while the kernel sources still hash the same.
+    """
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    h = kernel_source_hash()
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) == 3 and not ln.startswith("#") and parts[0] == workload and parts[1] == h:
+            return int(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Reads SM clock and clock-event reasons through NVML while the GPU works."""
+
+    def __init__(self, device_index: int):
+        self.ok = False
+        self.sm = []
+        self.reasons = set()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML missing: report clocks as unavailable
+            self.ok = False
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.sm.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+            r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in _REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def poll_until(self, event, min_samples: int = 3):
+        """Sample while ``event`` (a CUDA event recorded after the work) is pending."""
+        n = 0
+        while not event.query() or n < min_samples:
+            self.sample()
+            n += 1
+            if event.query() and n >= min_samples:
+                break
+            time.sleep(0.0005)
+
+    def summary(self):
+        if not self.ok or not self.sm:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml_unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.sm)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.sm)}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample_rate(wl, target_s: float, seed: int = 42):
+    """Time the oracle on a bounded row sample of ``wl``; returns (GB/s, info)."""
+    import oracle as O
+    from hadamard_rotation_outlier_b200 import synthetic as S
+
+    signs = S.signs(wl, seed)
+    t0 = wl.tensors[0]
+
+    def run(nrows):
+        x = S.tensor_rows(wl, 0, 0, nrows, seed)
+        t = time.perf_counter()
+        r = O.rotate_quantize(x, block=wl.block, signs=signs, bits=wl.bits, group=wl.group)
+        if wl.dequant:
+            O.dequant_rotate_inv(r["codes"], r["scales"], wl.dim, block=wl.block, signs=signs,
+                                 bits=wl.bits, group=wl.group)
+        return time.perf_counter() - t
+
+    n = min(t0.rows, max(1, (1 << 20) // wl.dim))
+    dt = run(n)
+    while dt < 0.2 * target_s and n < t0.rows:
+        n = min(t0.rows, int(n * min(8.0, max(2.0, 0.5 * target_s / max(dt, 1e-3)))))
+        dt = run(n)
+    frac = n / wl.rows
+    nbytes = wl.quant_bytes() * frac + (wl.dequant_bytes(2) * frac if wl.dequant else 0)
+    info = {"rows": n, "seconds": round(dt, 3), "bytes": int(nbytes)}
+    return nbytes / dt / 1e9, info
+
+
+# -------------------------------------------------------------- GPU arm
+
+def _dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+    from hadamard_rotation_outlier_b200 import binding as B
+    from hadamard_rotation_outlier_b200 import synthetic as S
+    from hadamard_rotation_outlier_b200.build import build
+    from hadamard_rotation_outlier_b200.steps import WorkloadStep
+
+    if args.workload not in S.WORKLOADS:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {list(S.WORKLOADS)}")
+    world, rank, local = _dist_setup(args)
+    if rank == 0:
+        build()
+    _barrier(world)
+    B.load_library()
+    wl = S.WORKLOADS[args.workload]
+    warmup = max(3, args.warmup)
+    steps = max(1, args.steps)
+    dev = torch.device("cuda", local if world > 1 else 0)
+
+    st = WorkloadStep(wl, dev, pinned_host=True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(warmup):
+        flush.zero_()
+        st.step(stream)
+    torch.cuda.synchronize(dev)
+
+    # ---- device-resident timed region ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    qends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if wl.dequant else None
+    done = torch.cuda.Event()
+    clocks = ClockSampler(dev.index)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = B.hadq_launch_count()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        st.quantize(stream)
+        if wl.dequant:
+            qends[i].record(stream)
+            st.dequantize(stream)
+        ends[i].record(stream)
+    done.record(stream)
+    clocks.poll_until(done)
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    launches = B.hadq_launch_count() - n0
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = _max_over_ranks(world, sum(step_ms))
+    quant_ms = ([s.elapsed_time(e) for s, e in zip(starts, qends)] if wl.dequant else step_ms)
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = run_e2e(st, stream, args.e2e_steps, world)
+
+    if rank != 0:
+        return None
+    bytes_step = st.bytes_per_step
+    value = world * bytes_step * steps / (total_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    q_bytes = wl.quant_bytes()
+    q_ms = sum(quant_ms) / len(quant_ms)
+    achieved = q_bytes / (q_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(wl.name)
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(total_ms / steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": wl.name, "description": wl.description, "rows": wl.rows, "dim": wl.dim,
+            "block": wl.block, "group": wl.group, "bits": wl.bits, "signs": wl.with_signs,
+            "dequant_in_step": wl.dequant, "bytes_per_step": bytes_step,
+            "rows_per_s": round(world * wl.rows * steps / (total_ms * 1e-3), 1),
+            "l2": "flushed between steps (256 MiB write outside the timed events)",
+            "parallelism": f"dp{world} (independent rows, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits,
+                                                              wl.group, wl.with_signs, True)],
+            "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": q_bytes, "avg_launch_ms": round(q_ms, 5),
+        },
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if wl.dequant:
+        dq_ms = [e.elapsed_time(f) for e, f in zip(qends, ends)]
+        out["roofline"]["dequant_achieved"] = round(wl.dequant_bytes(2) / (sum(dq_ms) / steps * 1e-3) / 1e9, 1)
+    if not args.no_cpu_baseline:
+        rate, info = oracle_sample_rate(wl, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": round(rate, 4), "unit": "GB/s", "cores": cpu_threads(),
+                               "kind": "oracle",
+                               "sample": f"{info['rows']} rows of {wl.name} through the float64 "
+                                         f"oracle in {info['seconds']} s"}
+    return out
+
+
+def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
+    """Same metric through the public API with host buffers.
+
+    Every step copies the bf16 input from pinned host memory, runs the step's
+    launches and copies every output (codes, scales and, for the KV-cache
+    workload, the bf16 reconstruction) back to pinned host memory.  The batch
+    is cut into row chunks alternating over two streams so that host-to-device
+    copies, kernels and device-to-host copies overlap.
+    """
+    import torch
+    wl = st.wl
+    dev = st.x.device
+    h_codes = torch.empty(st.codes.shape, dtype=st.codes.dtype, pin_memory=True)
+    h_scales = torch.empty(st.scales.shape, dtype=torch.float32, pin_memory=True)
+    h_out = torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) if wl.dequant else None
+    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    rows = st.rows
+    per = -(-rows // nchunks)
+    from hadamard_rotation_outlier_b200 import binding as B
+
+    def one_step():
+        ev0 = torch.cuda.Event()
+        ev0.record(stream)
+        tails = []
+        for c in range(nchunks):
+            r0, r1 = c * per, min(rows, (c + 1) * per)
+            if r0 >= r1:
+                break
+            s = streams[c % 2]
+            s.wait_event(ev0)
+            with torch.cuda.stream(s):
+                st.x[r0:r1].copy_(st.x_host[r0:r1], non_blocking=True)
+                B.hadq_rotate_quantize(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
+                                       group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],
+                                       stream=s)
+                if wl.dequant:
+                    B.hadq_dequant_rotate_inv(st.codes[r0:r1], st.scales[r0:r1], wl.dim, block=wl.block,
+                                              signs=st.signs, bits=wl.bits, group=wl.group,
+                                              out=st.out[r0:r1], stream=s)
+                    h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
+                h_codes[r0:r1].copy_(st.codes[r0:r1], non_blocking=True)
+                h_scales[r0:r1].copy_(st.scales[r0:r1], non_blocking=True)
+            e = torch.cuda.Event()
+            e.record(s)
+            tails.append(e)
+        for e in tails:
+            stream.wait_event(e)
+
+    for _ in range(2):
+        one_step()
+    torch.cuda.synchronize(dev)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(steps):
+        one_step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    ms = _max_over_ranks(world, start.elapsed_time(end))
+    h2d = st.x.numel() * 2
+    d2h = h_codes.numel() * h_codes.element_size() + h_scales.numel() * 4
+    if h_out is not None:
+        d2h += h_out.numel() * 2
+    return {"value": round(world * st.bytes_per_step * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 4), "chunks": nchunks}
+
+
+# ------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """The CPU oracle as it stands, timed on this host's cores (rank 0 only)."""
+    from hadamard_rotation_outlier_b200 import synthetic as S
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    wl = S.WORKLOADS[args.workload]
+    steps = max(1, args.steps if args.steps <= 5 else 3)
+    target = max(1.0, args.cpu_seconds / 2)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle_sample_rate(wl, 0.5)
+    rates, infos = [], []
+    for _ in range(steps):
+        r, info = oracle_sample_rate(wl, target)
+        rates.append(r)
+        infos.append(info)
+    total_bytes = sum(i["bytes"] for i in infos)
+    total_s = sum(i["seconds"] for i in infos)
+    value = total_bytes / total_s / 1e9
+    sample = (f"{steps} steps, each {infos[0]['rows']} rows of {wl.name} through the float64 "
+              f"oracle (numpy, dense Sylvester product)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": round(total_s / steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "rows": wl.rows, "dim": wl.dim, "block": wl.block,
+                   "group": wl.group, "bits": wl.bits, "signs": wl.with_signs},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if args.impl == "ours" and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+"""Thin ctypes binding of libhadq.so (include/hadq.h), same names as the C ABI.
+
+This module only marshals arguments: it checks tensor dtypes, devices and
+contiguity, resolves the row count, allocates outputs with torch when the
+caller passes none, and calls the C entry point on the current CUDA stream.
+Every step of the computation runs in the library's CUDA kernels.  There is
+no fallback: if the library is missing or cannot be loaded, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhadq.so")
+
+HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
+HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
+PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic"}
+MAX_DIM = 32768
+
+EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_plan", "hadq_status_str",
+            "hadq_last_error", "hadq_launch_count", "hadq_version")
+
+
+class HadqError(RuntimeError):
+    """A non-OK status returned by the library."""
+
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libhadq.so (once) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libhadq.so not found at {path}; build it with "
+                           "`python -m hadamard_rotation_outlier_b200.build`")
+    lib = ctypes.CDLL(path)
+    c_i64, c_i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
+    lib.hadq_rotate_quantize.argtypes = [vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, vp, vp, vp]
+    lib.hadq_rotate_quantize.restype = ctypes.c_int
+    lib.hadq_dequant_rotate_inv.argtypes = [vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
+                                            ctypes.c_int, vp]
+    lib.hadq_dequant_rotate_inv.restype = ctypes.c_int
+    lib.hadq_plan.argtypes = [c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                              ctypes.POINTER(ctypes.c_int)]
+    lib.hadq_plan.restype = ctypes.c_int
+    lib.hadq_status_str.argtypes = [ctypes.c_int]
+    lib.hadq_status_str.restype = ctypes.c_char_p
+    lib.hadq_last_error.argtypes = []
+    lib.hadq_last_error.restype = ctypes.c_char_p
+    lib.hadq_launch_count.argtypes = []
+    lib.hadq_launch_count.restype = c_i64
+    lib.hadq_version.argtypes = []
+    lib.hadq_version.restype = c_i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != HADQ_OK:
+        lib = load_library()
+        msg = lib.hadq_status_str(status).decode()
+        detail = lib.hadq_last_error().decode()
+        raise HadqError(status, f"{msg}: {detail}" if detail else msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t, name, dtype, device, numel=None):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+
+
+def _resolve(dim, block, group):
+    G = dim if group == -1 else group
+    return G
+
+
+def hadq_status_str(status: int) -> str:
+    return load_library().hadq_status_str(status).decode()
+
+
+def hadq_last_error() -> str:
+    return load_library().hadq_last_error().decode()
+
+
+def hadq_launch_count() -> int:
+    return int(load_library().hadq_launch_count())
+
+
+def hadq_version() -> int:
+    return int(load_library().hadq_version())
+
+
+def hadq_plan(direction: int, rows: int, dim: int, block: int = -1, bits: int = 4, group: int = -1,
+              has_signs: bool = False, aligned16: bool = True) -> str:
+    """Host-only: validate sizes and name the kernel family a call would use."""
+    path = ctypes.c_int(0)
+    _check(load_library().hadq_plan(direction, rows, dim, block, bits, group, int(has_signs),
+                                    int(aligned16), ctypes.byref(path)))
+    return PATH_NAMES[path.value]
+
+
+def hadq_rotate_quantize(x: torch.Tensor, block: int = -1, signs: torch.Tensor | None = None,
+                         bits: int = 4, group: int = -1, codes: torch.Tensor | None = None,
+                         scales: torch.Tensor | None = None, rotated_out: torch.Tensor | None = None,
+                         stream=None):
+    """Rotate then quantise the last dimension of a bf16 CUDA tensor.
+
+    Returns ``(codes, scales)``: int8 ``[..., dim]`` (bits 8) or uint8
+    ``[..., dim/2]`` (bits 4), and float32 ``[..., dim/G]``.  ``rotated_out``
+    (float32, same shape as ``x``) receives the rotated values if given.
+    """
+    lib = load_library()
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"x must be bfloat16, got {x.dtype}")
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    dim = x.shape[-1]
+    rows = x.numel() // dim if dim else 0
+    lead = tuple(x.shape[:-1])
+    dev = x.device
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(0, rows, dim, block, bits, group, 0, 1, None))
+    cshape = lead + ((dim,) if bits == 8 else (dim // 2,))
+    cdtype = torch.int8 if bits == 8 else torch.uint8
+    if codes is None:
+        codes = torch.empty(cshape, dtype=cdtype, device=dev)
+    else:
+        _need(codes, "codes", cdtype, dev, rows * cshape[-1])
+    if scales is None:
+        scales = torch.empty(lead + (dim // G,), dtype=torch.float32, device=dev)
+    else:
+        _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if rotated_out is not None:
+        _need(rotated_out, "rotated_out", torch.float32, dev, x.numel())
+    _check(lib.hadq_rotate_quantize(_ptr(x), rows, dim, block, _ptr(signs), bits, group,
+                                    _ptr(codes), _ptr(scales), _ptr(rotated_out), _stream(stream)))
+    return codes, scales
+
+
+def hadq_dequant_rotate_inv(codes: torch.Tensor, scales: torch.Tensor, dim: int, block: int = -1,
+                            signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                            out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                            stream=None) -> torch.Tensor:
+    """Dequantise codes and undo the rotation; returns ``[..., dim]`` bf16 or fp32."""
+    lib = load_library()
+    if not codes.is_cuda or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous CUDA tensor")
+    dev = codes.device
+    per_row = dim if bits == 8 else dim // 2
+    if per_row <= 0:
+        _check(lib.hadq_plan(1, 0, dim, block, bits, group, 0, 1, None))
+    rows = codes.numel() // per_row
+    lead = tuple(codes.shape[:-1]) if codes.shape[-1] == per_row else (rows,)
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(1, rows, dim, block, bits, group, 0, 1, None))
+    _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        out = torch.empty(lead + (dim,), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev, rows * dim)
+    code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_dequant_rotate_inv(_ptr(codes), _ptr(scales), rows, dim, block, _ptr(signs), bits,
+                                       group, _ptr(out), code, _stream(stream)))
+    return out

@@ -1,0 +1,423 @@
+// C ABI of libhadq: argument checks, kernel choice and launches.
+//
+// Every entry point validates its arguments on the host, picks one of three
+// kernel families (blocked, 4096-point, generic), launches one kernel on the
+// caller's stream and returns.  Nothing here allocates device memory and
+// nothing synchronises.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "../../include/hadq.h"
+#include "hadq_blocked.cuh"
+#include "hadq_full4096.cuh"
+#include "hadq_generic.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<int64_t> g_launches{0};
+
+hadq_status fail(hadq_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+hadq_status fail(hadq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+int ilog2(int64_t v) {
+  int r = 0;
+  while ((int64_t(1) << r) < v) ++r;
+  return r;
+}
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct Shape {
+  int64_t rows;
+  int dim, B, G, bits;
+  bool has_signs;
+};
+
+// Size checks shared by both directions.  On success fills B and G.
+hadq_status check_sizes(int64_t rows, int32_t dim, int32_t block, int32_t bits, int32_t group,
+                        Shape* s) {
+  if (rows < 0) return fail(HADQ_ERR_INVALID_ARG, "rows must be >= 0 (got %lld)", (long long)rows);
+  if (dim < 1 || dim > HADQ_MAX_DIM)
+    return fail(HADQ_ERR_INVALID_ARG, "dim must be in [1, %d] (got %d)", HADQ_MAX_DIM, dim);
+  if (bits != 4 && bits != 8) return fail(HADQ_ERR_INVALID_ARG, "bits must be 4 or 8 (got %d)", bits);
+  if (bits == 4 && (dim & 1))
+    return fail(HADQ_ERR_INVALID_ARG, "INT4 packs two codes per byte: dim must be even (got %d)", dim);
+  int B;
+  if (block == -1) {
+    if (!is_pow2(dim))
+      return fail(HADQ_ERR_INVALID_ARG, "block -1 (whole row) needs a power-of-two dim (got %d)", dim);
+    B = dim;
+  } else {
+    if (!is_pow2(block)) return fail(HADQ_ERR_INVALID_ARG, "block must be -1 or a power of two (got %d)", block);
+    if (dim % block) return fail(HADQ_ERR_INVALID_ARG, "block %d does not divide dim %d", block, dim);
+    B = block;
+  }
+  int G;
+  if (group == -1) {
+    G = dim;
+  } else {
+    if (group < 1) return fail(HADQ_ERR_INVALID_ARG, "group must be -1 or >= 1 (got %d)", group);
+    if (dim % group) return fail(HADQ_ERR_INVALID_ARG, "group %d does not divide dim %d", group, dim);
+    G = group;
+  }
+  s->rows = rows;
+  s->dim = dim;
+  s->B = B;
+  s->G = G;
+  s->bits = bits;
+  return HADQ_OK;
+}
+
+bool blocked_group_ok(int G, int B) { return (is_pow2(G) && G >= 8 && G <= B) || (G % B == 0); }
+
+hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
+  if (s.rows == 0) return HADQ_PATH_NONE;
+  if (aligned16 && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) && s.dim % 32 == 0 &&
+      s.dim <= 16384 && blocked_group_ok(s.G, s.B))
+    return HADQ_PATH_BLOCKED;
+  if (direction == 0 && aligned16 && s.B == 4096 && s.dim == 4096 && is_pow2(s.G) && s.G >= 64)
+    return HADQ_PATH_FULL4096;
+  return HADQ_PATH_GENERIC;
+}
+
+int sm_count() {
+  static std::mutex mu;
+  static std::unordered_map<int, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  cache[dev] = n;
+  return n;
+}
+
+// Resident CTAs per SM for (kernel, threads, dynamic smem), cached per device.
+int resident(const void* fn, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<std::string, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  char key[96];
+  snprintf(key, sizeof key, "%d:%p:%d:%zu", dev, fn, threads, smem);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  cache[key] = n;
+  return n;
+}
+
+hadq_status after_launch(const char* what) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(HADQ_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return HADQ_OK;
+}
+
+// ----------------------------------------------------------------- blocked
+
+struct BlockedPlan {
+  int threads, rpi, tpr;
+  int64_t nslabs;
+  size_t smem;
+};
+
+BlockedPlan blocked_plan(const Shape& s) {
+  BlockedPlan p;
+  p.tpr = s.dim / 32;
+  p.rpi = p.tpr <= 256 ? 256 / p.tpr : 1;
+  const int t = p.rpi * p.tpr;
+  p.threads = (t + 31) / 32 * 32;
+  p.nslabs = (s.rows + p.rpi - 1) / p.rpi;
+  p.smem = s.G > s.B ? size_t(3) * p.rpi * (s.dim / s.G) * sizeof(uint32_t) : 0;
+  return p;
+}
+
+template <int LOG_B, int BITS, int MAXT>
+const void* rq_blocked_fn(bool signs) {
+  return signs ? (const void*)hadq::rq_blocked_kernel<LOG_B, BITS, true, MAXT>
+               : (const void*)hadq::rq_blocked_kernel<LOG_B, BITS, false, MAXT>;
+}
+
+template <int LOG_B, int BITS, int MAXT>
+const void* dq_blocked_fn(bool signs, bool f32) {
+  if (signs) return f32 ? (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, true, true, MAXT>
+                        : (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, true, false, MAXT>;
+  return f32 ? (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, false, true, MAXT>
+             : (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, false, false, MAXT>;
+}
+
+template <int LOG_B, int BITS, int MAXT>
+const void* pick_blocked_b(int direction, bool signs, bool f32) {
+  return direction == 0 ? rq_blocked_fn<LOG_B, BITS, MAXT>(signs) : dq_blocked_fn<LOG_B, BITS, MAXT>(signs, f32);
+}
+
+template <int BITS, int MAXT>
+const void* pick_blocked_t(int direction, int B, bool signs, bool f32) {
+  switch (B) {
+    case 32: return pick_blocked_b<5, BITS, MAXT>(direction, signs, f32);
+    case 64: return pick_blocked_b<6, BITS, MAXT>(direction, signs, f32);
+    case 128: return pick_blocked_b<7, BITS, MAXT>(direction, signs, f32);
+    default: return pick_blocked_b<8, BITS, MAXT>(direction, signs, f32);
+  }
+}
+
+const void* pick_blocked(int direction, int bits, int B, bool signs, bool f32, int threads) {
+  if (threads <= 256)
+    return bits == 8 ? pick_blocked_t<8, 256>(direction, B, signs, f32) : pick_blocked_t<4, 256>(direction, B, signs, f32);
+  return bits == 8 ? pick_blocked_t<8, 512>(direction, B, signs, f32) : pick_blocked_t<4, 512>(direction, B, signs, f32);
+}
+
+hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, bool f32,
+                           cudaStream_t stream) {
+  const BlockedPlan p = blocked_plan(s);
+  a.rows = s.rows;
+  a.nslabs = p.nslabs;
+  a.dim = s.dim;
+  a.group = s.G;
+  a.rpi = p.rpi;
+  a.tpr = p.tpr;
+  const void* fn = pick_blocked(direction, s.bits, s.B, s.has_signs, f32, p.threads);
+  const size_t smem = direction == 0 ? p.smem : 0;
+  const int64_t cap = int64_t(resident(fn, p.threads, smem)) * sm_count();
+  const unsigned grid = (unsigned)(p.nslabs < cap ? p.nslabs : cap);
+  void* args[] = {&a};
+  cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(p.threads), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "blocked kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("blocked kernel");
+}
+
+// ------------------------------------------------------------------ 4096
+
+template <int BITS, bool SIGNS>
+const void* full_fn(int logG) {
+  switch (logG) {
+    case 6: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 6>;
+    case 7: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 7>;
+    case 8: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 8>;
+    case 9: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 9>;
+    case 10: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 10>;
+    case 11: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 11>;
+    default: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 12>;
+  }
+}
+
+hadq_status launch_full4096(const Shape& s, hadq::FullArgs a, cudaStream_t stream) {
+  a.rows = s.rows;
+  const int lg = ilog2(s.G);
+  const void* fn = s.bits == 8 ? (s.has_signs ? full_fn<8, true>(lg) : full_fn<8, false>(lg))
+                               : (s.has_signs ? full_fn<4, true>(lg) : full_fn<4, false>(lg));
+  const int64_t cap = int64_t(resident(fn, 64, 0)) * sm_count();
+  const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
+  void* args[] = {&a};
+  cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(64), args, 0, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "4096-point kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("4096-point kernel");
+}
+
+// --------------------------------------------------------------- generic
+
+hadq_status launch_generic(int direction, const Shape& s, hadq::GenericArgs a, bool f32,
+                           cudaStream_t stream) {
+  a.rows = s.rows;
+  a.dim = s.dim;
+  a.block = s.B;
+  a.group = s.G;
+  const void* fn;
+  size_t smem;
+  if (direction == 0) {
+    fn = s.bits == 8 ? (const void*)hadq::rq_generic_kernel<8> : (const void*)hadq::rq_generic_kernel<4>;
+    smem = size_t(s.dim) * 4 + ((size_t(s.dim) + 15) & ~size_t(15));
+  } else {
+    fn = s.bits == 8 ? (const void*)hadq::dq_generic_kernel<8> : (const void*)hadq::dq_generic_kernel<4>;
+    smem = size_t(s.dim) * 4;
+  }
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(HADQ_ERR_CUDA, "generic kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                  cudaGetErrorString(e));
+    }
+  }
+  const int64_t cap = int64_t(resident(fn, 256, smem)) * sm_count();
+  const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
+  cudaError_t e;
+  if (direction == 0) {
+    void* args[] = {&a};
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+  } else {
+    bool out_f32 = f32;
+    void* args[] = {&a, &out_f32};
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "generic kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("generic kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+hadq_status hadq_plan(int32_t direction, int64_t rows, int32_t dim, int32_t block, int32_t bits,
+                      int32_t group, int32_t has_signs, int32_t aligned16, hadq_path* path) {
+  if (direction != 0 && direction != 1)
+    return fail(HADQ_ERR_INVALID_ARG, "direction must be 0 or 1 (got %d)", direction);
+  Shape s;
+  hadq_status st = check_sizes(rows, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  s.has_signs = has_signs != 0;
+  if (path) *path = choose_path(direction, s, aligned16 != 0);
+  return HADQ_OK;
+}
+
+hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32_t block,
+                                 const int8_t* signs, int32_t bits, int32_t group, void* codes,
+                                 float* scales, float* rotated_out, hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = check_sizes(rows, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  s.has_signs = signs != nullptr;
+  if (rows == 0) return HADQ_OK;
+  if (!x || !codes || !scales)
+    return fail(HADQ_ERR_INVALID_ARG, "x, codes and scales must not be NULL");
+  if (!aligned(x, 2)) return fail(HADQ_ERR_MISALIGNED, "x must be 2-byte aligned");
+  if (!aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  if (rotated_out && !aligned(rotated_out, 4))
+    return fail(HADQ_ERR_MISALIGNED, "rotated_out must be 4-byte aligned");
+  const bool a16 = aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)) &&
+                   (!rotated_out || aligned(rotated_out, 16));
+  const hadq_path path = choose_path(0, s, a16);
+  const double qmax = double((1 << (bits - 1)) - 1);
+  const float scale_mul = (float)(1.0 / (std::sqrt(double(s.B)) * qmax));
+  const float rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == HADQ_PATH_BLOCKED) {
+    hadq::BlockedArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.signs = signs;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.rot = rotated_out;
+    a.scale_mul = scale_mul;
+    a.rsqrt_b = rsqrt_b;
+    return launch_blocked(0, s, a, false, cs);
+  }
+  if (path == HADQ_PATH_FULL4096) {
+    hadq::FullArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.signs = signs;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.rot = rotated_out;
+    a.scale_mul = scale_mul;
+    a.rsqrt_b = rsqrt_b;
+    return launch_full4096(s, a, cs);
+  }
+  hadq::GenericArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.signs = signs;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.rot = rotated_out;
+  a.scale_mul = scale_mul;
+  a.rsqrt_b = rsqrt_b;
+  return launch_generic(0, s, a, false, cs);
+}
+
+hadq_status hadq_dequant_rotate_inv(const void* codes, const float* scales, int64_t rows,
+                                    int32_t dim, int32_t block, const int8_t* signs, int32_t bits,
+                                    int32_t group, void* out, hadq_out_dtype out_dtype,
+                                    hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = check_sizes(rows, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
+    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
+  s.has_signs = signs != nullptr;
+  if (rows == 0) return HADQ_OK;
+  if (!codes || !scales || !out) return fail(HADQ_ERR_INVALID_ARG, "codes, scales and out must not be NULL");
+  const bool f32 = out_dtype == HADQ_OUT_F32;
+  if (!aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  if (!aligned(out, f32 ? 4 : 2)) return fail(HADQ_ERR_MISALIGNED, "out must be aligned to its element size");
+  const bool a16 = aligned(codes, 16) && aligned(out, 16) && (!signs || aligned(signs, 16));
+  const hadq_path path = choose_path(1, s, a16);
+  const float rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == HADQ_PATH_BLOCKED) {
+    hadq::BlockedArgs a{};
+    a.codes_in = static_cast<const uint8_t*>(codes);
+    a.scales_in = scales;
+    a.signs = signs;
+    a.rot = f32 ? static_cast<float*>(out) : nullptr;
+    a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+    a.rsqrt_b = rsqrt_b;
+    return launch_blocked(1, s, a, f32, cs);
+  }
+  hadq::GenericArgs a{};
+  a.codes_in = static_cast<const uint8_t*>(codes);
+  a.scales_in = scales;
+  a.signs = signs;
+  a.rot = f32 ? static_cast<float*>(out) : nullptr;
+  a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+  a.rsqrt_b = rsqrt_b;
+  return launch_generic(1, s, a, f32, cs);
+}
+
+const char* hadq_status_str(hadq_status st) {
+  switch (st) {
+    case HADQ_OK: return "ok";
+    case HADQ_ERR_INVALID_ARG: return "invalid argument";
+    case HADQ_ERR_UNSUPPORTED: return "unsupported combination";
+    case HADQ_ERR_MISALIGNED: return "misaligned pointer";
+    case HADQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* hadq_last_error(void) { return g_last_error.c_str(); }
+
+int64_t hadq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int32_t hadq_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+// Device helpers shared by the rotate+quantise and dequantise kernels.
+//
+// Conventions used in every kernel:
+//  * A row of `dim` bfloat16 values is cut into Hadamard blocks of B = 2^LOG_B
+//    elements.  The transform inside a block is the Sylvester H_B, which is the
+//    tensor product of one 2-point butterfly per bit of the element index, so
+//    the stages can run in any order and on any placement of the index bits
+//    (registers, lanes, shared memory).  The 1/sqrt(B) normalisation is never
+//    applied to the data: it cancels in the codes (q = y / (max|y|/qmax)) and
+//    is folded into the stored scale and into the optional float output.
+//  * Codes are produced with the float "magic number" rounding: for |t| < 2^22,
+//    fmaf(v, inv, 1.5*2^23) rounds v*inv to the nearest integer, ties to even,
+//    and its low bits hold that integer in two's complement.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace hadq {
+
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+
+// Below this group maximum qmax/max would overflow float; such groups take a
+// rescaled path (all their values are then subnormal-sized).
+constexpr float kTinyMax = 1.0e-36f;
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Sign mask for the bf16 pair (s0 -> low half, s1 -> high half): XOR-ing it into
+// the packed pair flips the sign of the elements whose sign entry is negative.
+__device__ __forceinline__ uint32_t pair_sign_mask(int8_t s0, int8_t s1) {
+  return (s0 < 0 ? 0x00008000u : 0u) | (s1 < 0 ? 0x80000000u : 0u);
+}
+
+// Round-to-nearest-even bf16 pair from two floats (finite inputs).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a = (a + 0x7fffu + ((a >> 16) & 1u)) >> 16;
+  b = (b + 0x7fffu + ((b >> 16) & 1u)) & 0xffff0000u;
+  return a | b;
+}
+
+// One radix-2 butterfly.
+__device__ __forceinline__ void bfly(float& a, float& b) {
+  float s = a + b;
+  b = a - b;
+  a = s;
+}
+
+// Two butterflies on packed float pairs (a0,a1) and (b0,b1) with the sm_100
+// paired-FP32 add/sub: (a0,a1) <- (a0+b0, a1+b1), (b0,b1) <- (a0-b0, a1-b1).
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  uint64_t A, Bv, S, D;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(Bv) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(S) : "l"(A), "l"(Bv));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(Bv));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(S));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(D));
+}
+
+// In-register butterfly stage over register-index bit `h` (stride h) of an
+// array of N floats.  Pairs whose partners are two apart or more use the
+// paired add/sub on neighbouring registers.
+template <int N, int H>
+__device__ __forceinline__ void reg_stage(float (&v)[N]) {
+  if constexpr (H == 1) {
+#pragma unroll
+    for (int i = 0; i < N; i += 2) bfly(v[i], v[i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 2 * H) {
+#pragma unroll
+      for (int t = 0; t < H; t += 2) bfly2(v[i + t], v[i + t + 1], v[i + t + H], v[i + t + H + 1]);
+    }
+  }
+}
+
+// All in-register stages over register-index bits [0, LOG_N).
+template <int N, int LOG_N>
+__device__ __forceinline__ void reg_fwht(float (&v)[N]) {
+  if constexpr (LOG_N >= 1) reg_stage<N, 1>(v);
+  if constexpr (LOG_N >= 2) reg_stage<N, 2>(v);
+  if constexpr (LOG_N >= 3) reg_stage<N, 4>(v);
+  if constexpr (LOG_N >= 4) reg_stage<N, 8>(v);
+  if constexpr (LOG_N >= 5) reg_stage<N, 16>(v);
+  if constexpr (LOG_N >= 6) reg_stage<N, 32>(v);
+  if constexpr (LOG_N >= 7) reg_stage<N, 64>(v);
+}
+
+// Butterfly stage across lanes: partner = lane ^ m.  The lane whose bit is set
+// keeps (partner - own), the other keeps (own + partner).
+template <int N>
+__device__ __forceinline__ void lane_stage(float (&v)[N], int m, float sgn) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    float p = __shfl_xor_sync(0xffffffffu, v[i], m);
+    v[i] = fmaf(v[i], sgn, p);
+  }
+}
+
+// Code of t = v*inv as the low bits of a float's bit pattern (see header note).
+__device__ __forceinline__ uint32_t magic_code(float v, float inv) {
+  return __float_as_uint(fmaf(v, inv, kMagic));
+}
+
+// Four codes (low byte of each) -> one word of int8 codes.
+__device__ __forceinline__ uint32_t pack_i8x4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
+  uint32_t lo = __byte_perm(c0, c1, 0x0040);
+  uint32_t hi = __byte_perm(c2, c3, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// Two words of int8 codes (elements 0..3 and 4..7, values in [-8, 7]) -> one
+// word of int4 codes, element 0 in bits 0..3.
+__device__ __forceinline__ uint32_t nibble_pack(uint32_t b03, uint32_t b47) {
+  uint32_t x = b03 & 0x0f0f0f0fu;
+  uint32_t y = b47 & 0x0f0f0f0fu;
+  x |= x >> 4;  // byte 0 = e0 | e1 << 4, byte 2 = e2 | e3 << 4
+  y |= y >> 4;
+  return __byte_perm(x, y, 0x6420);
+}
+
+// Eight codes (low nibble of each) -> one word of int4 codes, element 0 in bits 0..3.
+__device__ __forceinline__ uint32_t pack_i4x8(const uint32_t (&c)[8]) {
+  return nibble_pack(pack_i8x4(c[0], c[1], c[2], c[3]), pack_i8x4(c[4], c[5], c[6], c[7]));
+}
+
+// Codes of eight values against one group maximum `m` (of the same, unnormalised
+// values): t = v * qmax / m, rounded half to even.  Groups whose maximum is so
+// small that qmax/m would overflow are rescaled by 2^64 first (exact).
+__device__ __forceinline__ void quantize8(const float* v, float m, float qmax, uint32_t (&cc)[8]) {
+  if (m >= kTinyMax) {
+    const float inv = qmax / m;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cc[k] = magic_code(v[k], inv);
+  } else {
+    const float pre = 18446744073709551616.0f;  // 2^64
+    const float inv = m > 0.0f ? qmax / (m * pre) : 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cc[k] = magic_code(v[k] * pre, inv);
+  }
+}
+
+// Sign-extended int4 nibble k of word w, as float.
+__device__ __forceinline__ float i4_at(uint32_t w, int k) {
+  return (float)(((int32_t)(w << (28 - 4 * k))) >> 28);
+}
+
+__device__ __forceinline__ float i8_at(uint32_t w, int k) {
+  return (float)(((int32_t)(w << (24 - 8 * k))) >> 24);
+}
+
+}  // namespace hadq

@@ -1,0 +1,148 @@
+/*
+ * hadq.h -- C ABI of the fused Hadamard rotate + quantize library (libhadq.so)
+ *
+ * The library implements the online rotate-then-quantize step of QuaRot-style
+ * rotation quantisation and its inverse, as CUDA kernels for sm_100a (B200).
+ *
+ *   forward:  y = (x * s) H_B   per B-wide block of each row       (rotation)
+ *             scale_g = max_{i in g} |y_i| / qmax,  qmax = 2^(bits-1) - 1
+ *             q_i = clamp(round_half_even(y_i / scale_g), -qmax, qmax)
+ *   inverse:  x_hat = ((q * scale_g) H_B) * s
+ *
+ * Sources (page title, section):
+ *   - H_B is the normalised Sylvester matrix H_1 = [1],
+ *     H_2n = [[H, H], [H, -H]] / sqrt(2) ("Hartmann rotation, lightweight QAT,
+ *     streaming attention", section 1, the Hadamard rotation of Q and K:
+ *     Q_rot = Q H^T, and H H^T = I so Q_rot K_rot^T = Q K^T).
+ *   - Block-diagonal H for widths that are not a power of two: rows are cut
+ *     into B-wide blocks rotated independently ("Rotation quantisation: the
+ *     outlier nemesis", section 2.1; block_size -1 means no blocking in the
+ *     msModelSlim QuaRot YAML configuration).
+ *   - Random +-1 signs before H (randomised Hadamard, "QuaRot hands-on",
+ *     section 2.1).
+ *   - Symmetric absmax scale, round, clip ("Rotation quantisation: the outlier
+ *     nemesis", section 2.2 quant_error; "Hartmann rotation", section 1,
+ *     scale = max|x| / 127); per-group scales (same page, section 6.2).
+ *   - INT4 codes take half a byte and the KV cache is dequantised when read
+ *     ("QuaRot hands-on", sections 2.2 and 2.3).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major, contiguous, on the current CUDA device.  The
+ *     caller owns every buffer; the library never allocates device memory.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *     Argument checks run on the host before any launch; on an error nothing
+ *     is launched and no output is touched.
+ *   - HADQ_ERR_CUDA reports a launch failure (cudaGetLastError after the
+ *     launch); hadq_last_error() gives the text.  Faults during execution are
+ *     reported by the next synchronising CUDA call, as for any kernel.
+ *   - rows == 0 is a valid empty call: HADQ_OK, nothing launched, pointers
+ *     may be NULL.
+ *   - Inputs must be finite.  Non-finite inputs give unspecified codes (no
+ *     fault).
+ *   - Calls that touch the same output buffers must be ordered by the caller.
+ */
+#ifndef HADQ_H
+#define HADQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The same type as cudaStream_t (a pointer to the runtime's stream object). */
+struct CUstream_st;
+typedef struct CUstream_st *hadq_stream_t;
+
+typedef enum {
+  HADQ_OK = 0,
+  HADQ_ERR_INVALID_ARG = 1,  /* out-of-range size, NULL pointer, bad enum     */
+  HADQ_ERR_UNSUPPORTED = 2,  /* valid maths, no kernel for it (not used now)  */
+  HADQ_ERR_MISALIGNED = 3,   /* pointer not aligned to its element size       */
+  HADQ_ERR_CUDA = 4          /* the CUDA runtime reported an error            */
+} hadq_status;
+
+typedef enum { HADQ_OUT_BF16 = 0, HADQ_OUT_F32 = 1 } hadq_out_dtype;
+
+/* Which kernel family a call dispatches to (see hadq_plan). */
+typedef enum {
+  HADQ_PATH_NONE = 0,      /* empty call, nothing launched                  */
+  HADQ_PATH_BLOCKED = 1,   /* register butterflies, blocks of 8..256        */
+  HADQ_PATH_FULL4096 = 2,  /* one 4096-point block per row, smem transposes */
+  HADQ_PATH_GENERIC = 3    /* shared-memory kernel, any valid combination   */
+} hadq_path;
+
+enum { HADQ_MAX_DIM = 32768 };
+
+/*
+ * hadq_rotate_quantize -- fused rotate + quantise of a [rows, dim] bf16 tensor.
+ *
+ *   x           device, bfloat16 [rows, dim], 2-byte aligned (16 for the fast
+ *               paths; others fall back to the generic kernel).
+ *   rows        >= 0.
+ *   dim         1 .. HADQ_MAX_DIM; even when bits == 4.
+ *   block       Hadamard block B: -1 = whole row (dim must be a power of two),
+ *               else a power of two (1 allowed = no rotation) dividing dim.
+ *   signs       device, int8 [dim], negative entry = -1, else +1; or NULL for
+ *               no sign flip.  Applied to x before H.
+ *   bits        4 or 8.
+ *   group       scale group G in columns: -1 = one scale per row, else any
+ *               divisor of dim.  Independent of block.
+ *   codes       device output.  bits 8: int8 [rows, dim].  bits 4: uint8
+ *               [rows, dim/2], element 2j in the low nibble of byte j, 4-bit
+ *               two's complement, values in [-7, 7].
+ *   scales      device output, float32 [rows, dim/G], 4-byte aligned.
+ *               scale = max|y| / qmax of the group; 0 for an all-zero group
+ *               (whose codes are then 0).
+ *   rotated_out device output float32 [rows, dim] (4-byte aligned) receiving y
+ *               itself, or NULL.  Meant for checking; costs 4 bytes/element.
+ */
+hadq_status hadq_rotate_quantize(const void *x, int64_t rows, int32_t dim, int32_t block,
+                                 const int8_t *signs, int32_t bits, int32_t group,
+                                 void *codes, float *scales, float *rotated_out,
+                                 hadq_stream_t stream);
+
+/*
+ * hadq_dequant_rotate_inv -- x_hat = ((q * scale) H_B) * s for [rows, dim].
+ *
+ *   codes, scales  as produced by hadq_rotate_quantize with the same dim,
+ *                  block, signs, bits and group (device pointers).  INT4 code
+ *                  -8 is accepted and dequantised as -8 * scale.
+ *   out            device output [rows, dim]: bfloat16 (round to nearest
+ *                  even, 2-byte aligned) or float32 (4-byte aligned),
+ *                  chosen by out_dtype.
+ *   Other arguments and rules as for hadq_rotate_quantize.
+ */
+hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int64_t rows,
+                                    int32_t dim, int32_t block, const int8_t *signs,
+                                    int32_t bits, int32_t group, void *out,
+                                    hadq_out_dtype out_dtype, hadq_stream_t stream);
+
+/*
+ * hadq_plan -- host-only: validate the sizes of a call and report the kernel
+ * family it would use.  direction 0 = rotate_quantize, 1 = dequant_rotate_inv.
+ * `aligned16` says whether every pointer of the call is 16-byte aligned.
+ * Returns the same status the call would return for these sizes (pointer
+ * checks aside) and writes the path to *path.  Touches no GPU.
+ */
+hadq_status hadq_plan(int32_t direction, int64_t rows, int32_t dim, int32_t block,
+                      int32_t bits, int32_t group, int32_t has_signs, int32_t aligned16,
+                      hadq_path *path);
+
+/* Static description of a status code. */
+const char *hadq_status_str(hadq_status status);
+
+/* Detail of the most recent failure in the calling host thread ("" if none). */
+const char *hadq_last_error(void);
+
+/* Number of kernel launches issued by this process so far (all threads). */
+int64_t hadq_launch_count(void);
+
+/* ABI version, currently 1. */
+int32_t hadq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HADQ_H */

@@ -1,0 +1,104 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+* Rotated values y (float32 from the GPU) and dequantised reconstructions in
+  float32: |g - o| <= 1e-5 * max(|o|, rms of o over the row).  The row-RMS floor
+  keeps entries near zero from failing on absolute rounding noise.
+* Scales: |g - o| <= max(1e-5 * |o|, 2^-149) (exact 0 for an all-zero group);
+  the floor is one float32 subnormal step, the storage resolution of a scale
+  below 2^-126.
+* Codes: bit-exact, except where the oracle's pre-round value y/scale lies
+  within 1e-4 of a rounding boundary k + 0.5; such a code may differ by one.
+  The number of mismatches must be at most 1e-5 of the elements, with at least
+  one such mismatch tolerated on small cases.
+* bf16 reconstructions: within one bf16 ulp of the oracle rounded to bf16
+  (round to nearest, ties to even).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+
+REL_TOL = 1e-5
+BOUNDARY = 1e-4
+MISMATCH_RATE = 1e-5
+
+
+def gpu_codes_to_int(codes: np.ndarray, bits: int, dim: int) -> np.ndarray:
+    c = np.asarray(codes)
+    if bits == 8:
+        return c.reshape(-1, dim).astype(np.int64)
+    return O.unpack_int4(c.reshape(-1, dim // 2))
+
+
+def check_values(g: np.ndarray, o: np.ndarray, what: str, tol: float = REL_TOL) -> float:
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    assert g.shape == o.shape, (what, g.shape, o.shape)
+    if o.size == 0:
+        return 0.0
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True))
+    ref = np.maximum(np.abs(o), rms)
+    err = np.abs(g - o)
+    bad = err > tol * ref
+    if np.any(bad):
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} values off; first at {tuple(i)}: "
+                             f"gpu {g[tuple(i)]!r} oracle {o[tuple(i)]!r}")
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return float(np.nanmax(np.where(ref > 0, err / ref, 0.0)))
+
+
+def check_scales(g: np.ndarray, o: np.ndarray) -> float:
+    g = np.asarray(g, dtype=np.float64).reshape(o.shape)
+    o = np.asarray(o, dtype=np.float64)
+    zero = o == 0
+    assert np.all(g[zero] == 0), "all-zero groups must have scale 0"
+    err = np.abs(g - o)
+    ok = err <= np.maximum(REL_TOL * np.abs(o), 2.0 ** -149)
+    assert np.all(ok), f"scales: {int((~ok).sum())} off, max rel err {(err / np.abs(o))[~ok].max():.3e}"
+    with np.errstate(invalid="ignore", divide="ignore"):
+        rel = np.where(zero, 0.0, err / np.abs(o))
+    return float(rel.max()) if rel.size else 0.0
+
+
+def check_codes(g_q: np.ndarray, o_q: np.ndarray, pre_round: np.ndarray) -> int:
+    """Returns the number of (allowed) boundary mismatches."""
+    g_q = np.asarray(g_q).reshape(o_q.shape)
+    mism = g_q != o_q
+    n = int(mism.sum())
+    if n:
+        d = O.half_boundary_distance(pre_round[mism])
+        far = d > BOUNDARY
+        if np.any(far):
+            idx = np.argwhere(mism)[np.argmax(far)]
+            raise AssertionError(f"codes: {int(far.sum())} mismatches away from a .5 boundary; e.g. "
+                                 f"at {tuple(idx)} gpu {g_q[tuple(idx)]} oracle {o_q[tuple(idx)]} "
+                                 f"pre-round {pre_round[tuple(idx)]!r}")
+        assert np.all(np.abs(g_q[mism] - o_q[mism]) == 1)
+    allowed = max(1.0, MISMATCH_RATE * o_q.size)
+    assert n <= allowed, f"codes: {n} boundary mismatches > {allowed:g} allowed"
+    return n
+
+
+def bf16_bits_rne(x: np.ndarray) -> np.ndarray:
+    """float64 -> bf16 bits with one rounding (to nearest, ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                       # x = m * 2^e, 0.5 <= |m| < 1
+    normal = np.ldexp(np.round(m * 256.0) / 256.0, e)   # 8 significant bits
+    sub = np.round(x * 2.0 ** 133) * 2.0 ** -133        # bf16 subnormal grid
+    y = np.where(np.abs(x) < 2.0 ** -126, sub, normal).astype(np.float32)  # exact
+    return (y.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _ordered(bits: np.ndarray) -> np.ndarray:
+    b = bits.astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def check_bf16(g_bits: np.ndarray, o: np.ndarray, what: str) -> int:
+    ref = bf16_bits_rne(o)
+    d = np.abs(_ordered(np.asarray(g_bits, dtype=np.uint16).reshape(ref.shape)) - _ordered(ref))
+    assert np.all(d <= 1), f"{what}: {int((d > 1).sum())} values more than 1 bf16 ulp off"
+    return int(d.max()) if d.size else 0

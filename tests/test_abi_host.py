@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+that include/hadq.h declares, and rejects bad arguments before any launch.
+
+No call here reaches a kernel: every call either fails validation or is an
+empty (rows == 0) call, both of which return before touching CUDA.
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from hadamard_rotation_outlier_b200 import binding as B
+from hadamard_rotation_outlier_b200.build import LIB, ROOT, build
+
+HEADER = os.path.join(ROOT, "include", "hadq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hadq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert names == sorted(B.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (hadq_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(lib):
+    assert B.hadq_version() == 1
+    assert B.hadq_status_str(B.HADQ_OK) == "ok"
+    assert "invalid" in B.hadq_status_str(B.HADQ_ERR_INVALID_ARG)
+    assert "misaligned" in B.hadq_status_str(B.HADQ_ERR_MISALIGNED)
+    assert B.hadq_status_str(99) == "unknown status"
+
+
+@pytest.mark.parametrize("args,msg", [
+    ((0, -1, 128, -1, 8, -1), "rows"),
+    ((0, 4, 0, -1, 8, -1), "dim"),
+    ((0, 4, 32769, 128, 8, -1), "dim"),
+    ((0, 4, 128, -1, 5, -1), "bits"),
+    ((0, 4, 127, 1, 4, -1), "even"),
+    ((0, 4, 96, -1, 8, -1), "power-of-two dim"),
+    ((0, 4, 128, 48, 8, -1), "power of two"),
+    ((0, 4, 96, 64, 8, -1), "does not divide"),
+    ((0, 4, 128, 128, 8, 0), "group"),
+    ((0, 4, 128, 128, 8, 48), "does not divide"),
+    ((2, 4, 128, 128, 8, -1), "direction"),
+])
+def test_plan_rejects(lib, args, msg):
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_plan(*args)
+    assert e.value.status == B.HADQ_ERR_INVALID_ARG
+    assert msg in str(e.value)
+
+
+@pytest.mark.parametrize("direction,rows,dim,block,bits,group,signs,a16,path", [
+    (0, 0, 128, -1, 8, -1, False, True, "none"),
+    (0, 524288, 128, -1, 8, -1, False, True, "blocked"),          # Q/K heads, INT8
+    (0, 256, 4096, 128, 4, -1, False, True, "blocked"),           # per-token over 32 blocks
+    (0, 16384, 4096, -1, 4, -1, True, True, "full4096"),          # full 4096 + signs
+    (0, 2097152, 128, 128, 4, 128, False, True, "blocked"),       # KV cache
+    (1, 2097152, 128, 128, 4, 128, False, True, "blocked"),       # KV dequant
+    (0, 32768, 11008, 128, 4, 128, True, True, "blocked"),        # 86 blocks of 128
+    (0, 10, 128, -1, 8, -1, False, False, "generic"),             # unaligned pointers
+    (0, 10, 4096, -1, 4, 32, False, True, "generic"),             # small groups on 4096
+    (0, 10, 8192, -1, 4, -1, False, True, "generic"),             # 8192-point block
+    (0, 10, 32768, 128, 4, 128, False, True, "generic"),          # wider than 16384
+    (0, 10, 12, 4, 8, 3, False, True, "generic"),
+    (1, 10, 4096, -1, 4, -1, True, True, "generic"),              # 4096 dequant
+])
+def test_plan_paths(lib, direction, rows, dim, block, bits, group, signs, a16, path):
+    assert B.hadq_plan(direction, rows, dim, block, bits, group, signs, a16) == path
+
+
+def test_invalid_calls_return_before_launch(lib):
+    n0 = B.hadq_launch_count()
+    vp = ctypes.c_void_p
+    fake = vp(0x10000)
+    # NULL outputs
+    st = lib.hadq_rotate_quantize(fake, 4, 128, -1, None, 8, -1, None, fake, None, None)
+    assert st == B.HADQ_ERR_INVALID_ARG and "NULL" in B.hadq_last_error()
+    # misaligned bf16 input / scales / outputs
+    st = lib.hadq_rotate_quantize(vp(0x10001), 4, 128, -1, None, 8, -1, fake, fake, None, None)
+    assert st == B.HADQ_ERR_MISALIGNED
+    st = lib.hadq_rotate_quantize(fake, 4, 128, -1, None, 8, -1, fake, vp(0x10002), None, None)
+    assert st == B.HADQ_ERR_MISALIGNED
+    st = lib.hadq_rotate_quantize(fake, 4, 128, -1, None, 8, -1, fake, fake, vp(0x10002), None)
+    assert st == B.HADQ_ERR_MISALIGNED
+    st = lib.hadq_dequant_rotate_inv(fake, fake, 4, 128, -1, None, 8, -1, vp(0x10002), B.HADQ_OUT_F32,
+                                     None)
+    assert st == B.HADQ_ERR_MISALIGNED
+    st = lib.hadq_dequant_rotate_inv(fake, fake, 4, 128, -1, None, 8, -1, fake, 7, None)
+    assert st == B.HADQ_ERR_INVALID_ARG
+    st = lib.hadq_dequant_rotate_inv(None, fake, 4, 128, -1, None, 8, -1, fake, B.HADQ_OUT_BF16, None)
+    assert st == B.HADQ_ERR_INVALID_ARG
+    # bad sizes with otherwise valid pointers
+    st = lib.hadq_rotate_quantize(fake, 4, 100, 64, None, 8, -1, fake, fake, None, None)
+    assert st == B.HADQ_ERR_INVALID_ARG and "does not divide" in B.hadq_last_error()
+    assert B.hadq_launch_count() == n0
+
+
+def test_empty_call_is_a_noop(lib):
+    n0 = B.hadq_launch_count()
+    assert lib.hadq_rotate_quantize(None, 0, 128, -1, None, 8, -1, None, None, None, None) == B.HADQ_OK
+    assert lib.hadq_dequant_rotate_inv(None, None, 0, 4096, -1, None, 4, -1, None, B.HADQ_OUT_BF16,
+                                       None) == B.HADQ_OK
+    assert B.hadq_launch_count() == n0
+    # sizes are still validated for empty calls
+    assert lib.hadq_rotate_quantize(None, 0, 100, 64, None, 8, -1, None, None, None, None) == \
+        B.HADQ_ERR_INVALID_ARG
+
+
+def test_last_error_is_cleared_by_a_good_call(lib):
+    lib.hadq_rotate_quantize(None, 0, 100, 64, None, 8, -1, None, None, None, None)
+    assert B.hadq_last_error()
+    lib.hadq_rotate_quantize(None, 0, 128, 64, None, 8, -1, None, None, None, None)
+    assert B.hadq_last_error() == ""

@@ -1,0 +1,205 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Oracle-sized cases: every kernel family, block and group sizes inside and
+across blocks, signs, INT4 and INT8, ragged row counts, odd shapes on the
+generic kernel, unaligned pointers, degenerate groups.  Each case compares
+rotated values, scales and codes, then feeds the GPU codes and scales to both
+dequantisers and compares the reconstructions (float32 and bf16).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hadamard_rotation_outlier_b200 import binding as B
+from hadamard_rotation_outlier_b200 import synthetic as S
+from hadamard_rotation_outlier_b200.steps import bf16_tensor_to_bits, bits_to_bf16_tensor
+
+from parity import check_bf16, check_codes, check_scales, check_values, gpu_codes_to_int
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+def oracle_method(dim, block):
+    B_ = dim if block == -1 else block
+    return "dense" if B_ <= 4096 else "fwht"
+
+
+def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", outliers=(),
+             x_bits=None, offset=0, check_dequant=True):
+    if x_bits is None:
+        x_bits = S.random_bf16(rows, dim, seed, dist=dist, outlier_cols=outliers)
+    s = S.random_signs(dim, seed) if with_signs else None
+    meth = oracle_method(dim, block)
+    ref = O.rotate_quantize(x_bits, block=block, signs=s, bits=bits, group=group, method=meth)
+
+    if offset:  # a view starting `offset` elements into a larger buffer: unaligned pointers
+        xb = bits_to_bf16_tensor(np.concatenate([np.zeros(offset, np.uint16), x_bits.ravel()]), DEV)
+        x = xb[offset:].view(rows, dim)
+    else:
+        x = bits_to_bf16_tensor(x_bits, DEV)
+    sg = None if s is None else torch.from_numpy(s).to(DEV)
+    rot = torch.empty((rows, dim), dtype=torch.float32, device=DEV)
+    codes, scales = B.hadq_rotate_quantize(x, block=block, signs=sg, bits=bits, group=group,
+                                           rotated_out=rot)
+    torch.cuda.synchronize()
+    check_values(rot.cpu().numpy(), ref["rotated"], "rotated")
+    check_scales(scales.cpu().numpy(), ref["scales"])
+    check_codes(gpu_codes_to_int(codes.cpu().numpy(), bits, dim), ref["q"], ref["pre_round"])
+
+    # the same codes without the optional float output (the timed configuration)
+    codes2, scales2 = B.hadq_rotate_quantize(x, block=block, signs=sg, bits=bits, group=group)
+    torch.cuda.synchronize()
+    assert torch.equal(codes2, codes) and torch.equal(scales2, scales)
+
+    if check_dequant:
+        g_codes = codes.cpu().numpy()
+        g_scales = scales.cpu().numpy()
+        o_rec = O.dequant_rotate_inv(g_codes, g_scales, dim, block=block, signs=s, bits=bits,
+                                     group=group, method=meth)
+        f32 = B.hadq_dequant_rotate_inv(codes, scales, dim, block=block, signs=sg, bits=bits,
+                                        group=group, out_dtype=torch.float32)
+        b16 = B.hadq_dequant_rotate_inv(codes, scales, dim, block=block, signs=sg, bits=bits,
+                                        group=group, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        check_values(f32.cpu().numpy(), o_rec, "dequant fp32")
+        check_bf16(bf16_tensor_to_bits(b16), o_rec, "dequant bf16")
+    return codes, scales
+
+
+# (rows, dim, block, group, bits, signs, expected forward path)
+CASES = [
+    (300, 128, -1, -1, 8, False, "blocked"),        # Q/K heads, INT8, per row
+    (301, 128, 128, 128, 4, False, "blocked"),      # KV rows, INT4, group 128
+    (37, 4096, 128, -1, 4, False, "blocked"),       # per-token scale over 32 blocks
+    (9, 11008, 128, 128, 4, True, "blocked"),       # 86 blocks, signs
+    (5, 11008, 128, -1, 8, True, "blocked"),        # 86 blocks, one scale per row
+    (65, 256, 32, 8, 4, False, "blocked"),          # groups smaller than a block
+    (70, 512, 64, 16, 8, True, "blocked"),
+    (33, 1024, 256, 64, 4, True, "blocked"),
+    (17, 768, 256, -1, 8, False, "blocked"),        # row of three 256-blocks
+    (40, 2048, 32, 256, 8, False, "blocked"),       # groups of 8 blocks
+    (3, 16384, 128, -1, 4, True, "blocked"),        # widest blocked row (512 threads)
+    (6, 8192, 256, 1024, 8, True, "blocked"),
+    (129, 64, 64, 32, 4, False, "blocked"),
+    (21, 4096, -1, -1, 4, True, "full4096"),        # full 4096 + signs, per token
+    (19, 4096, -1, 128, 8, False, "full4096"),
+    (7, 4096, 4096, 64, 4, True, "full4096"),
+    (11, 4096, -1, 1024, 8, True, "full4096"),
+    (8, 4096, -1, 2048, 4, False, "full4096"),
+    (13, 4096, -1, 512, 4, False, "full4096"),
+    (10, 4096, -1, 256, 8, True, "full4096"),
+    (5, 12, 4, 3, 8, False, "generic"),             # odd group, tiny block
+    (9, 4096, -1, 32, 4, True, "generic"),          # groups too small for the 4096 path
+    (4, 8192, -1, -1, 4, True, "generic"),          # 8192-point block
+    (6, 100, 4, 10, 4, False, "generic"),
+    (3, 2048, -1, -1, 8, True, "generic"),
+    (12, 24, 8, 8, 4, False, "generic"),
+    (2, 32768, 128, 128, 4, False, "generic"),      # widest row
+    (1, 1, 1, 1, 8, False, "generic"),
+    (50, 64, 16, 16, 8, True, "generic"),
+    (3, 6, 2, 6, 4, False, "generic"),
+]
+
+
+@pytest.mark.parametrize("rows,dim,block,group,bits,signs,path", CASES)
+def test_parity_shapes(rows, dim, block, group, bits, signs, path):
+    assert B.hadq_plan(0, rows, dim, block, bits, group, signs, True) == path
+    run_case(rows, dim, block, group, bits, signs, seed=rows * 7 + dim, outliers=[dim // 3])
+
+
+@pytest.mark.parametrize("dist", ["normal", "student_t3"])
+def test_parity_distributions(dist):
+    run_case(64, 1024, 128, 128, 4, True, seed=5, dist=dist)
+
+
+def test_unaligned_pointer_takes_generic_path_and_matches():
+    run_case(31, 128, -1, -1, 8, False, seed=3, offset=1, check_dequant=False)
+    run_case(9, 4096, -1, -1, 4, True, seed=4, offset=3, check_dequant=False)
+
+
+def test_zero_rows_and_zero_groups():
+    for dim, block, group, bits in [(128, -1, -1, 8), (256, 128, 64, 4), (4096, -1, -1, 4),
+                                    (4096, 128, -1, 4), (12, 4, 3, 8)]:
+        x = np.zeros((4, dim), np.uint16)
+        x[1] = S.random_bf16(1, dim, 9)[0]
+        codes, scales = run_case(4, dim, block, group, bits, False, x_bits=x)
+        sc = scales.cpu().numpy().reshape(4, -1)
+        assert np.all(sc[0] == 0) and np.all(sc[2:] == 0)
+        assert not torch.any(codes[0].to(torch.int32)) and not torch.any(codes[2:].to(torch.int32))
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device=DEV)
+    codes, scales = B.hadq_rotate_quantize(x, block=-1, bits=8)
+    assert codes.shape == (0, 128) and scales.shape == (0, 1)
+
+
+def test_tiny_and_subnormal_groups():
+    """Groups whose maximum is subnormal-sized: qmax/max would overflow float32."""
+    for dim, block, group in [(128, 128, 128), (4096, -1, -1), (12, 4, 3)]:
+        rng = np.random.default_rng(dim)
+        x = rng.integers(1, 0x7F, size=(3, dim)).astype(np.uint16)       # subnormal bf16
+        x |= (rng.integers(0, 2, size=(3, dim)) << 15).astype(np.uint16)  # random signs
+        x[2] = S.random_bf16(1, dim, 3)[0]
+        run_case(3, dim, block, group, 4, False, x_bits=x)
+        run_case(3, dim, block, group, 8, False, x_bits=x)
+
+
+def test_exact_ties_round_half_even():
+    # block 1 (no rotation): scale = 7/7 = 1, values on .5 exactly.
+    y = np.array([[7, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5]], dtype=np.float32)
+    x = S.f32_to_bf16_bits(np.repeat(y, 40, axis=0).reshape(40, 8))
+    for group in (8, -1):
+        codes, _ = B.hadq_rotate_quantize(bits_to_bf16_tensor(x, DEV), block=1, bits=4, group=group)
+        q = gpu_codes_to_int(codes.cpu().numpy(), 4, 8)
+        np.testing.assert_array_equal(q, np.tile([7, 0, 2, 2, 0, -2, -2, 4], (40, 1)))
+    # through 32-wide blocks: y = H x with x = 2*e_0 gives +-2/sqrt(32); add a
+    # block where the quantiser sees exact halves after an exact transform.
+    x = np.zeros((2, 32), np.float32)
+    x[0, 0] = 14.0           # y = 14/sqrt(32) everywhere -> all codes 7
+    x[1, :2] = [3.0, 1.0]    # y in {4, 2}/sqrt(32): INT4 codes 7 and 3.5 -> 4 (even)
+    codes, _ = B.hadq_rotate_quantize(bits_to_bf16_tensor(S.f32_to_bf16_bits(x), DEV), block=32,
+                                      bits=4, group=32)
+    q = gpu_codes_to_int(codes.cpu().numpy(), 4, 32)
+    assert np.all(q[0] == 7)
+    assert set(np.abs(q[1]).tolist()) == {7, 4}
+
+
+def test_hand_worked_examples_on_gpu(golden_hand):
+    g = golden_hand
+    x = bits_to_bf16_tensor(S.f32_to_bf16_bits(np.array([g["ex1_x"]], np.float32)), DEV)
+    codes, scales = B.hadq_rotate_quantize(x, block=-1, bits=4)
+    assert codes.cpu().numpy().ravel().tolist() == [int(v) for v in g["ex1_int4_bytes"]]
+    assert scales.item() == pytest.approx(5 / 7, rel=1e-6)
+    codes, _ = B.hadq_rotate_quantize(x, block=-1, bits=8)
+    assert codes.cpu().numpy().ravel().tolist() == [int(v) for v in g["ex1_int8_q"]]
+    sg = torch.tensor(g["ex2_signs"], dtype=torch.int8, device=DEV)
+    codes, _ = B.hadq_rotate_quantize(x, block=-1, signs=sg, bits=4)
+    assert codes.cpu().numpy().ravel().tolist() == [int(v) for v in g["ex2_int4_bytes"]]
+
+
+def test_non_default_stream_and_launch_count():
+    x_bits = S.random_bf16(64, 128, 2)
+    x = bits_to_bf16_tensor(x_bits, DEV)
+    st = torch.cuda.Stream()
+    n0 = B.hadq_launch_count()
+    with torch.cuda.stream(st):
+        codes, scales = B.hadq_rotate_quantize(x, block=-1, bits=8, stream=st)
+    st.synchronize()
+    assert B.hadq_launch_count() == n0 + 1
+    ref = O.rotate_quantize(x_bits, block=-1, bits=8)
+    check_codes(gpu_codes_to_int(codes.cpu().numpy(), 8, 128), ref["q"], ref["pre_round"])
+
+
+def test_binding_rejects_bad_tensors():
+    x = torch.zeros((4, 128), dtype=torch.float32, device=DEV)
+    with pytest.raises(TypeError):
+        B.hadq_rotate_quantize(x)
+    x = torch.zeros((4, 100), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_rotate_quantize(x, block=64, bits=4)
+    assert e.value.status == B.HADQ_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        B.hadq_rotate_quantize(torch.zeros((128, 4), dtype=torch.bfloat16, device=DEV).t(), bits=8)
