@@ -16,7 +16,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libhadq.so")
-SOURCES = [os.path.join(PKG, "csrc", "hadq_api.cu")]
+SOURCES = sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")))
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -39,20 +39,39 @@ def needs_build() -> bool:
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile the library if it is missing or stale; return its path."""
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), "-shared", "-Xcompiler", "-fPIC", "-O3", "-lineinfo", "-std=c++17",
-           *ARCH, "-o", tmp, *SOURCES]
+def _compile(src: str, obj: str, verbose: bool):
+    cmd = [nvcc_path(), "-c", "-Xcompiler", "-fPIC", "-O3", "-lineinfo", "-std=c++17", *ARCH,
+           "-o", obj, src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    return subprocess.run(cmd, capture_output=True, text=True)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library if it is missing or stale; return its path.
+
+    Each kernel family is its own translation unit; they compile in parallel
+    and link into one shared library.
+    """
+    if not force and not needs_build():
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    objs = [os.path.join(objdir, os.path.basename(src)[:-3] + ".o") for src in SOURCES]
+    with ThreadPoolExecutor(len(SOURCES)) as ex:
+        results = list(ex.map(lambda so: _compile(so[0], so[1], verbose), zip(SOURCES, objs)))
+    for src, res in zip(SOURCES, results):
+        if res.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {os.path.basename(src)} ({res.returncode}):\n"
+                               f"{res.stderr[-8000:]}")
+        if verbose:
+            sys.stderr.write(res.stderr)
+    tmp = LIB + ".tmp"
+    res = subprocess.run([nvcc_path(), "-shared", *ARCH, "-o", tmp, *objs], capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr[-8000:]}")
-    if verbose:
-        sys.stderr.write(res.stderr)
+        raise RuntimeError(f"nvcc link failed ({res.returncode}):\n{res.stderr[-8000:]}")
     os.replace(tmp, LIB)
     return LIB
 

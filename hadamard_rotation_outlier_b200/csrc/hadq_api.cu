@@ -15,8 +15,10 @@
 
 #include "../../include/hadq.h"
 #include "hadq_blocked.cuh"
+#include "hadq_chunk.cuh"
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
+#include "hadq_kernels.h"
 
 namespace {
 
@@ -85,8 +87,15 @@ hadq_status check_sizes(int64_t rows, int32_t dim, int32_t block, int32_t bits, 
 
 bool blocked_group_ok(int G, int B) { return (is_pow2(G) && G >= 8 && G <= B) || (G % B == 0); }
 
+bool chunk_ok(int direction, const Shape& s) {
+  if (direction != 0 || s.B < 8 || s.B > 128 || s.dim % 128) return false;
+  if (is_pow2(s.G) && s.G >= 8 && s.G <= 128) return true;
+  return s.G % 128 == 0 && s.dim <= 128 * hadq::kCT;  // a slab holds whole rows
+}
+
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
+  if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
   if (aligned16 && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) && s.dim % 32 == 0 &&
       s.dim <= 16384 && blocked_group_ok(s.G, s.B))
     return HADQ_PATH_BLOCKED;
@@ -158,41 +167,6 @@ BlockedPlan blocked_plan(const Shape& s) {
   return p;
 }
 
-template <int LOG_B, int BITS, int MAXT>
-const void* rq_blocked_fn(bool signs) {
-  return signs ? (const void*)hadq::rq_blocked_kernel<LOG_B, BITS, true, MAXT>
-               : (const void*)hadq::rq_blocked_kernel<LOG_B, BITS, false, MAXT>;
-}
-
-template <int LOG_B, int BITS, int MAXT>
-const void* dq_blocked_fn(bool signs, bool f32) {
-  if (signs) return f32 ? (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, true, true, MAXT>
-                        : (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, true, false, MAXT>;
-  return f32 ? (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, false, true, MAXT>
-             : (const void*)hadq::dq_blocked_kernel<LOG_B, BITS, false, false, MAXT>;
-}
-
-template <int LOG_B, int BITS, int MAXT>
-const void* pick_blocked_b(int direction, bool signs, bool f32) {
-  return direction == 0 ? rq_blocked_fn<LOG_B, BITS, MAXT>(signs) : dq_blocked_fn<LOG_B, BITS, MAXT>(signs, f32);
-}
-
-template <int BITS, int MAXT>
-const void* pick_blocked_t(int direction, int B, bool signs, bool f32) {
-  switch (B) {
-    case 32: return pick_blocked_b<5, BITS, MAXT>(direction, signs, f32);
-    case 64: return pick_blocked_b<6, BITS, MAXT>(direction, signs, f32);
-    case 128: return pick_blocked_b<7, BITS, MAXT>(direction, signs, f32);
-    default: return pick_blocked_b<8, BITS, MAXT>(direction, signs, f32);
-  }
-}
-
-const void* pick_blocked(int direction, int bits, int B, bool signs, bool f32, int threads) {
-  if (threads <= 256)
-    return bits == 8 ? pick_blocked_t<8, 256>(direction, B, signs, f32) : pick_blocked_t<4, 256>(direction, B, signs, f32);
-  return bits == 8 ? pick_blocked_t<8, 512>(direction, B, signs, f32) : pick_blocked_t<4, 512>(direction, B, signs, f32);
-}
-
 hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, bool f32,
                            cudaStream_t stream) {
   const BlockedPlan p = blocked_plan(s);
@@ -202,7 +176,7 @@ hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, b
   a.group = s.G;
   a.rpi = p.rpi;
   a.tpr = p.tpr;
-  const void* fn = pick_blocked(direction, s.bits, s.B, s.has_signs, f32, p.threads);
+  const void* fn = hadq::blocked_kernel_ptr(direction, s.bits, s.B, s.has_signs, f32, p.threads);
   const size_t smem = direction == 0 ? p.smem : 0;
   const int64_t cap = int64_t(resident(fn, p.threads, smem)) * sm_count();
   const unsigned grid = (unsigned)(p.nslabs < cap ? p.nslabs : cap);
@@ -216,26 +190,43 @@ hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, b
   return after_launch("blocked kernel");
 }
 
-// ------------------------------------------------------------------ 4096
+// ----------------------------------------------------------------- chunk
 
-template <int BITS, bool SIGNS>
-const void* full_fn(int logG) {
-  switch (logG) {
-    case 6: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 6>;
-    case 7: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 7>;
-    case 8: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 8>;
-    case 9: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 9>;
-    case 10: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 10>;
-    case 11: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 11>;
-    default: return (const void*)hadq::rq_full4096_kernel<BITS, SIGNS, 12>;
+hadq_status launch_chunk(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+  a.cpr = s.dim / hadq::kCK;
+  a.nchunks = s.rows * a.cpr;
+  a.slab_chunks = s.G > hadq::kCK ? (hadq::kCT / a.cpr) * a.cpr : hadq::kCT;
+  a.nslabs = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
+  a.G = s.G;
+  a.dim = s.dim;
+  a.log_g = s.G <= hadq::kCK ? ilog2(s.G) : -1;
+  a.gpc = s.G > hadq::kCK ? s.G / hadq::kCK : 1;
+  const void* fn = hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK);
+  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "chunk kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                cudaGetErrorString(e));
   }
+  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  const unsigned grid = (unsigned)(a.nslabs < cap ? a.nslabs : cap);
+  void* args[] = {&a};
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "chunk kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("chunk kernel");
 }
+
+// ------------------------------------------------------------------ 4096
 
 hadq_status launch_full4096(const Shape& s, hadq::FullArgs a, cudaStream_t stream) {
   a.rows = s.rows;
   const int lg = ilog2(s.G);
-  const void* fn = s.bits == 8 ? (s.has_signs ? full_fn<8, true>(lg) : full_fn<8, false>(lg))
-                               : (s.has_signs ? full_fn<4, true>(lg) : full_fn<4, false>(lg));
+  const void* fn = hadq::full4096_kernel_ptr(s.bits, s.has_signs, lg);
   const int64_t cap = int64_t(resident(fn, 64, 0)) * sm_count();
   const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
   void* args[] = {&a};
@@ -259,11 +250,11 @@ hadq_status launch_generic(int direction, const Shape& s, hadq::GenericArgs a, b
   const void* fn;
   size_t smem;
   if (direction == 0) {
-    fn = s.bits == 8 ? (const void*)hadq::rq_generic_kernel<8> : (const void*)hadq::rq_generic_kernel<4>;
+    fn = hadq::generic_kernel_ptr(0, s.bits);
     smem = size_t(s.dim) * 4 + ((size_t(s.dim) + 15) & ~size_t(15));
   } else {
-    fn = s.bits == 8 ? (const void*)hadq::dq_generic_kernel<8> : (const void*)hadq::dq_generic_kernel<4>;
-    smem = size_t(s.dim) * 4;
+    fn = hadq::generic_kernel_ptr(1, s.bits);
+    smem = size_t(s.dim) * 4 + ((size_t(s.dim / s.B) + 15) & ~size_t(15));
   }
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -340,6 +331,17 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.scale_mul = scale_mul;
     a.rsqrt_b = rsqrt_b;
     return launch_blocked(0, s, a, false, cs);
+  }
+  if (path == HADQ_PATH_CHUNK) {
+    hadq::ChunkArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.signs = signs;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.rot = rotated_out;
+    a.scale_mul = scale_mul;
+    a.rsqrt_b = rsqrt_b;
+    return launch_chunk(s, a, cs);
   }
   if (path == HADQ_PATH_FULL4096) {
     hadq::FullArgs a{};

@@ -236,11 +236,25 @@ __global__ void __launch_bounds__(MAXT, MAXT == 256 ? 3 : 1) dq_blocked_kernel(B
     const bool active = lane_ok && row < a.rows;
     const int64_t base = row * dim + col0;
 
-    float v[32];
+    // Blocks with a scale below 2^-100 would run the butterflies on subnormal
+    // values (each add rounding to the 2^-149 grid); they run at 2^64 times
+    // their value instead and are scaled back once at the end (exact factors).
+    float sc[4];
+    bool tiny = false;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = c * B + 8 * T * j + 8 * q;
-      const float s = active ? __ldg(a.scales_in + row * ngroups + e / G) * a.rsqrt_b : 0.0f;
+      sc[j] = active ? __ldg(a.scales_in + row * ngroups + e / G) : 0.0f;
+      tiny |= sc[j] < kTinyScale && sc[j] != 0.0f;
+    }
+#pragma unroll
+    for (int b = 0; b < LOG_T; ++b) tiny |= __shfl_xor_sync(0xffffffffu, (int)tiny, 1 << b) != 0;
+    const float pre = tiny ? kUp64 : 1.0f;
+
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float s = sc[j] * pre * a.rsqrt_b;
       if constexpr (BITS == 8) {
         uint2 w = active ? __ldg(reinterpret_cast<const uint2*>(a.codes_in + base + 8 * T * j)) : make_uint2(0, 0);
 #pragma unroll
@@ -258,6 +272,10 @@ __global__ void __launch_bounds__(MAXT, MAXT == 256 ? 3 : 1) dq_blocked_kernel(B
     reg_fwht<32, 5>(v);
 #pragma unroll
     for (int b = 0; b < LOG_T; ++b) lane_stage<32>(v, 1 << b, sgn[b]);
+    if (tiny) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= kDown64;
+    }
 
     if (active) {
 #pragma unroll

@@ -1,0 +1,286 @@
+// Chunk path: Hadamard blocks of B = 8..128 columns, dim a multiple of 128.
+//
+// Every thread owns one 128-element chunk of a row (chunks never cross rows),
+// so all log2(B) butterfly stages run in registers with no shuffles.  A CTA of
+// 128 threads walks over slabs of consecutive chunks, which are contiguous in
+// memory.  Each slab is staged through shared memory:
+//
+//   load   16-byte cp.async copies, consecutive lanes on consecutive 16-byte
+//          pieces (fully coalesced), into chunk slots padded to 272 bytes so
+//          that a thread reading its own chunk row-wise is bank-conflict free.
+//          Two stages: the next slab streams in while this one is computed.
+//   store  each thread writes its codes back into its own slot; after a
+//          barrier the CTA copies the slab's codes out with coalesced 16-byte
+//          stores (they too are contiguous in memory).
+//
+// Scale groups: G = 2^g with 8 <= G <= 128 reduce inside the thread; groups of
+// several chunks (G a multiple of 128) reduce with one shared-memory max per
+// slab, and then a slab holds whole rows so that no group straddles two slabs.
+#pragma once
+
+#include "hadq_common.cuh"
+
+namespace hadq {
+
+constexpr int kCK = 128;     // elements per chunk (one thread)
+constexpr int kCT = 128;     // threads per CTA
+constexpr int kCPad = 272;   // bytes per chunk slot in shared memory (256 + 16)
+
+struct ChunkArgs {
+  const uint16_t* x;         // forward input (bf16)
+  const uint8_t* codes_in;   // inverse input
+  const float* scales_in;
+  const int8_t* signs;
+  uint8_t* codes;
+  float* scales;
+  float* rot;                // forward: optional fp32 y; inverse: fp32 output
+  uint16_t* out_bf16;
+  int64_t nchunks;           // rows * dim / 128
+  int64_t nslabs;
+  int cpr;                   // chunks per row
+  int slab_chunks;           // chunks per slab (<= 128)
+  int G;
+  int log_g;                 // log2(G) when G <= 128, else -1
+  int gpc;                   // chunks per group when G > 128, else 1
+  int dim;
+  float scale_mul;
+  float rsqrt_b;
+};
+
+// Shared-memory layout shared by host and device.
+__host__ __device__ constexpr int chunk_stage_bytes() { return kCT * kCPad; }
+__host__ __device__ inline int chunk_mask_words(int dim) { return dim / 2 + 4 * (dim / 128); }
+__host__ __device__ inline size_t chunk_smem_bytes(int dim, bool signs) {
+  return size_t(2) * chunk_stage_bytes() + 2 * kCT * sizeof(uint32_t) +
+         (signs ? size_t(chunk_mask_words(dim)) * sizeof(uint32_t) : 0);
+}
+
+// Pair sign masks are stored with 4 padding words after every 64, so that
+// threads reading the masks of consecutive chunks hit different banks.
+__device__ __forceinline__ int mask_slot(int pair) { return pair + 4 * (pair >> 6); }
+
+
+// Copies `nch` chunks of `bytes_per_chunk` (16 * PPC) bytes starting at `src`
+// into padded slots of `dst`.  Consecutive threads take consecutive 16-byte
+// pieces, so every warp reads 512 contiguous bytes.  Full slabs use a fully
+// unrolled loop with constant strides.
+template <int PPC>
+__device__ __forceinline__ void chunk_load(const uint8_t* src, int nch, uint8_t* dst) {
+  const int tid = threadIdx.x;
+  if (nch == kCT) {
+    constexpr int STEP = kCT / PPC;  // chunks covered by one pass of the CTA
+    const uint8_t* s0 = src + 16 * tid;
+    uint8_t* d0 = dst + (tid / PPC) * kCPad + 16 * (tid % PPC);
+#pragma unroll
+    for (int i = 0; i < PPC; ++i) cp_async16(d0 + i * STEP * kCPad, s0 + i * 16 * kCT);
+  } else {
+    for (int g = tid; g < nch * PPC; g += kCT) cp_async16(dst + (g / PPC) * kCPad + 16 * (g % PPC), src + 16 * g);
+  }
+}
+
+// Copies `nch` chunk results of 16 * PPC bytes from padded slots to `dst`.
+template <int PPC>
+__device__ __forceinline__ void chunk_store(const uint8_t* src, int nch, uint8_t* dst) {
+  const int tid = threadIdx.x;
+  if (nch == kCT) {
+    constexpr int STEP = kCT / PPC;
+    const uint8_t* s0 = src + (tid / PPC) * kCPad + 16 * (tid % PPC);
+    uint8_t* d0 = dst + 16 * tid;
+#pragma unroll
+    for (int i = 0; i < PPC; ++i)
+      *reinterpret_cast<uint4*>(d0 + i * 16 * kCT) = *reinterpret_cast<const uint4*>(s0 + i * STEP * kCPad);
+  } else {
+    for (int g = tid; g < nch * PPC; g += kCT)
+      *reinterpret_cast<uint4*>(dst + 16 * g) = *reinterpret_cast<const uint4*>(src + (g / PPC) * kCPad + 16 * (g % PPC));
+  }
+}
+
+__device__ __forceinline__ int slab_count(int64_t nchunks, int64_t slab, int slab_chunks) {
+  const int64_t left = nchunks - slab * slab_chunks;
+  return left < slab_chunks ? (int)left : slab_chunks;
+}
+
+// Codes of the 128 values of one chunk into its shared-memory slot: vector p
+// (8 values) uses multiplier inv[p] (all equal when the group covers the chunk).
+template <int BITS>
+__device__ __forceinline__ void chunk_codes(const float (&v)[kCK], const float (&inv)[16], uint8_t* slot) {
+#pragma unroll
+  for (int p = 0; p < 16; p += 2) {
+    uint32_t c[16];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      magic_code2(v[8 * p + k], v[8 * p + k + 1], inv[p], c[k], c[k + 1]);
+      magic_code2(v[8 * p + 8 + k], v[8 * p + 9 + k], inv[p + 1], c[8 + k], c[9 + k]);
+    }
+    if constexpr (BITS == 8) {
+      *reinterpret_cast<uint4*>(slot + 8 * p) =
+          make_uint4(pack_i8x4(c[0], c[1], c[2], c[3]), pack_i8x4(c[4], c[5], c[6], c[7]),
+                     pack_i8x4(c[8], c[9], c[10], c[11]), pack_i8x4(c[12], c[13], c[14], c[15]));
+    } else {
+      const uint32_t a0[8] = {c[0], c[1], c[2], c[3], c[4], c[5], c[6], c[7]};
+      const uint32_t a1[8] = {c[8], c[9], c[10], c[11], c[12], c[13], c[14], c[15]};
+      *reinterpret_cast<uint2*>(slot + 4 * p) = make_uint2(pack_i4x8(a0), pack_i4x8(a1));
+    }
+  }
+}
+
+// Forward: bf16 -> signs -> H_B (B = 2^LOG_B, 8..128) -> group max -> codes.
+// WIDE_G: the scale group covers whole chunks (G >= 128); otherwise 8 <= G < 128.
+template <int LOG_B, int BITS, bool SIGNS, bool WIDE_G>
+__global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
+  constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
+  constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* stage0 = smem;
+  uint8_t* stage1 = smem + chunk_stage_bytes();
+  uint32_t* s_gmax = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes());  // [2][kCT]
+  uint32_t* s_msk = s_gmax + 2 * kCT;
+  const int tid = threadIdx.x;
+  const int G = a.G;
+  const bool multi = WIDE_G && G > kCK;  // groups spanning several chunks
+
+  if constexpr (SIGNS) {
+    for (int p = tid; p < a.dim / 2; p += kCT)
+      s_msk[mask_slot(p)] = pair_sign_mask(a.signs[2 * p], a.signs[2 * p + 1]);
+  }
+  for (int i = tid; i < 2 * kCT; i += kCT) s_gmax[i] = 0u;
+
+  const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
+  // Column chunk of this thread's chunk, advanced from slab to slab (sign
+  // masks only); group bookkeeping for groups spanning several chunks.
+  int colc = SIGNS ? (int)(((int64_t)blockIdx.x * a.slab_chunks + tid) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)(((int64_t)gridDim.x * a.slab_chunks) % a.cpr) : 0;
+  const int wide_slot = multi ? tid / a.gpc : 0;
+  const bool wide_lead = multi ? (tid - wide_slot * a.gpc) == 0 : true;
+  const int groups_per_slab = multi ? a.slab_chunks / a.gpc : 0;
+
+  int64_t slab = blockIdx.x;
+  if (slab < a.nslabs) chunk_load<16>(xsrc + slab * a.slab_chunks * 256, slab_count(a.nchunks, slab, a.slab_chunks), stage0);
+  cp_async_commit();
+  for (int it = 0; slab < a.nslabs; ++it, slab += gridDim.x) {
+    uint8_t* cur = (it & 1) ? stage1 : stage0;
+    cp_async_wait<0>();
+    __syncthreads();  // slab data visible; the other stage is free again
+    {
+      const int64_t nx = slab + gridDim.x;
+      if (nx < a.nslabs)
+        chunk_load<16>(xsrc + nx * a.slab_chunks * 256, slab_count(a.nchunks, nx, a.slab_chunks), (it & 1) ? stage0 : stage1);
+      cp_async_commit();
+    }
+    const int nch = slab_count(a.nchunks, slab, a.slab_chunks);
+    const int64_t ch = slab * a.slab_chunks + tid;
+    const bool active = tid < nch;
+    const int col0 = colc * kCK;
+    if constexpr (SIGNS) {
+      colc += col_step;
+      if (colc >= a.cpr) colc -= a.cpr;
+    }
+    uint8_t* mine = cur + tid * kCPad;
+
+    float v[kCK];
+    float pm[16];
+    if (active) {
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        const uint4 r = *reinterpret_cast<const uint4*>(mine + 16 * p);
+        uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        if constexpr (SIGNS) {
+          const uint4 m4 = *reinterpret_cast<const uint4*>(s_msk + mask_slot(col0 / 2 + 4 * p));
+          w[0] ^= m4.x;
+          w[1] ^= m4.y;
+          w[2] ^= m4.z;
+          w[3] ^= m4.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bf16_pair_stage1(w[i], v[8 * p + 2 * i], v[8 * p + 2 * i + 1]);
+      }
+      reg_fwht_from<kCK, 1, LOG_B>(v);
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        float m = fmaxf(fabsf(v[8 * p]), fabsf(v[8 * p + 1]));
+#pragma unroll
+        for (int k = 2; k < 8; ++k) m = fmaxf(m, fabsf(v[8 * p + k]));
+        pm[p] = m;
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < 16; ++p) pm[p] = 0.0f;
+    }
+
+    float gmax = 0.0f;  // WIDE_G: maximum of the whole group
+    if constexpr (WIDE_G) {
+      gmax = pm[0];
+#pragma unroll
+      for (int p = 1; p < 16; ++p) gmax = fmaxf(gmax, pm[p]);
+      if (multi) {
+        uint32_t* slot = s_gmax + (it & 1) * kCT + wide_slot;
+        if (active) atomicMax(slot, __float_as_uint(gmax));
+        __syncthreads();
+        gmax = __uint_as_float(*slot);
+        s_gmax[((it + 1) & 1) * kCT + tid] = 0u;  // read two slabs later, after two barriers
+      }
+    } else {
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        if (G > (8 << l)) {
+          float t[16];
+#pragma unroll
+          for (int p = 0; p < 16; ++p) t[p] = fmaxf(pm[p], pm[p ^ (1 << l)]);
+#pragma unroll
+          for (int p = 0; p < 16; ++p) pm[p] = t[p];
+        }
+      }
+    }
+
+    if (active) {
+      // scale index = (flat element index of the group's first element) / G
+      if constexpr (WIDE_G) {
+        if (wide_lead) a.scales[multi ? slab * groups_per_slab + wide_slot : ch] = gmax * a.scale_mul;
+      } else {
+        const int lg = a.log_g;
+#pragma unroll
+        for (int p = 0; p < 16; ++p)
+          if (((8 * p) & (G - 1)) == 0) a.scales[((ch * kCK) >> lg) + ((8 * p) >> lg)] = pm[p] * a.scale_mul;
+      }
+      if (a.rot) {
+        float4* dst = reinterpret_cast<float4*>(a.rot + ch * kCK);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          dst[i] = make_float4(v[4 * i] * a.rsqrt_b, v[4 * i + 1] * a.rsqrt_b, v[4 * i + 2] * a.rsqrt_b,
+                               v[4 * i + 3] * a.rsqrt_b);
+      }
+      // codes into this thread's own slot (its input is already in registers)
+      float inv[16];
+      bool tiny = false;
+      if constexpr (WIDE_G) {
+        const QInv q = make_qinv(gmax, QMAX);
+        tiny = q.tiny;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) inv[p] = q.inv;
+      } else {
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const QInv q = make_qinv(pm[p], QMAX);
+          inv[p] = q.inv;
+          tiny |= q.tiny;
+        }
+      }
+      if (tiny) {  // groups whose maximum is below kTinyMax: codes from v * 2^64 (see make_qinv)
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float m = WIDE_G ? gmax : pm[p];
+          if (m < kTinyMax) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[8 * p + k] *= 18446744073709551616.0f;
+          }
+        }
+      }
+      chunk_codes<BITS>(v, inv, mine);
+    }
+    __syncthreads();
+    chunk_store<CB / 16>(cur, nch, a.codes + slab * a.slab_chunks * CB);
+  }
+  cp_async_wait<0>();
+}
+
+}  // namespace hadq

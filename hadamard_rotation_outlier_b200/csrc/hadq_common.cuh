@@ -24,6 +24,13 @@ constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 // rescaled path (all their values are then subnormal-sized).
 constexpr float kTinyMax = 1.0e-36f;
 
+// Dequantisation: blocks with a scale below kTinyScale (2^-100) are computed at
+// 2^64 times their value and scaled back once, so the butterflies never run
+// on subnormal numbers.  Both factors are exact powers of two.
+constexpr float kTinyScale = 7.888609052210118e-31f;  // 2^-100
+constexpr float kUp64 = 18446744073709551616.0f;      // 2^64
+constexpr float kDown64 = 5.421010862427522e-20f;     // 2^-64
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
@@ -60,6 +67,17 @@ __device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1
   asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(D));
 }
 
+// bf16 pair (x0 low half, x1 high half) -> first butterfly stage (x0 + x1,
+// x0 - x1) with the mixed bf16/f32 add and subtract: x1 is widened by masking,
+// x0 is read directly as a bf16 operand.  Same rounding as adding the widened
+// values.
+__device__ __forceinline__ void bf16_pair_stage1(uint32_t w, float& s, float& d) {
+  const float x1 = __uint_as_float(w & 0xffff0000u);
+  unsigned short x0 = (unsigned short)(w & 0xffffu);
+  asm("add.rn.f32.bf16 %0, %1, %2;" : "=f"(s) : "h"(x0), "f"(x1));
+  asm("sub.rn.f32.bf16 %0, %1, %2;" : "=f"(d) : "h"(x0), "f"(x1));
+}
+
 // In-register butterfly stage over register-index bit `h` (stride h) of an
 // array of N floats.  Pairs whose partners are two apart or more use the
 // paired add/sub on neighbouring registers.
@@ -75,6 +93,18 @@ __device__ __forceinline__ void reg_stage(float (&v)[N]) {
       for (int t = 0; t < H; t += 2) bfly2(v[i + t], v[i + t + 1], v[i + t + H], v[i + t + H + 1]);
     }
   }
+}
+
+// In-register stages over register-index bits [FIRST, LOG_N).
+template <int N, int FIRST, int LOG_N>
+__device__ __forceinline__ void reg_fwht_from(float (&v)[N]) {
+  if constexpr (FIRST <= 0 && LOG_N >= 1) reg_stage<N, 1>(v);
+  if constexpr (FIRST <= 1 && LOG_N >= 2) reg_stage<N, 2>(v);
+  if constexpr (FIRST <= 2 && LOG_N >= 3) reg_stage<N, 4>(v);
+  if constexpr (FIRST <= 3 && LOG_N >= 4) reg_stage<N, 8>(v);
+  if constexpr (FIRST <= 4 && LOG_N >= 5) reg_stage<N, 16>(v);
+  if constexpr (FIRST <= 5 && LOG_N >= 6) reg_stage<N, 32>(v);
+  if constexpr (FIRST <= 6 && LOG_N >= 7) reg_stage<N, 64>(v);
 }
 
 // All in-register stages over register-index bits [0, LOG_N).
@@ -105,6 +135,16 @@ __device__ __forceinline__ uint32_t magic_code(float v, float inv) {
   return __float_as_uint(fmaf(v, inv, kMagic));
 }
 
+// Codes of two values against one multiplier with the paired fused multiply-add.
+__device__ __forceinline__ void magic_code2(float v0, float v1, float inv, uint32_t& c0, uint32_t& c1) {
+  uint64_t V, I, M, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(V) : "f"(v0), "f"(v1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(I) : "f"(inv));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(M) : "f"(kMagic));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(V), "l"(I), "l"(M));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(c0), "=r"(c1) : "l"(R));
+}
+
 // Four codes (low byte of each) -> one word of int8 codes.
 __device__ __forceinline__ uint32_t pack_i8x4(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3) {
   uint32_t lo = __byte_perm(c0, c1, 0x0040);
@@ -115,16 +155,17 @@ __device__ __forceinline__ uint32_t pack_i8x4(uint32_t c0, uint32_t c1, uint32_t
 // Two words of int8 codes (elements 0..3 and 4..7, values in [-8, 7]) -> one
 // word of int4 codes, element 0 in bits 0..3.
 __device__ __forceinline__ uint32_t nibble_pack(uint32_t b03, uint32_t b47) {
-  uint32_t x = b03 & 0x0f0f0f0fu;
-  uint32_t y = b47 & 0x0f0f0f0fu;
-  x |= x >> 4;  // byte 0 = e0 | e1 << 4, byte 2 = e2 | e3 << 4
-  y |= y >> 4;
-  return __byte_perm(x, y, 0x6420);
+  const uint32_t e = __byte_perm(b03, b47, 0x6420);  // elements 0, 2, 4, 6
+  const uint32_t o = __byte_perm(b03, b47, 0x7531);  // elements 1, 3, 5, 7
+  return (e & 0x0f0f0f0fu) | ((o << 4) & 0xf0f0f0f0u);
 }
 
-// Eight codes (low nibble of each) -> one word of int4 codes, element 0 in bits 0..3.
+// Eight codes (low nibble of each) -> one word of int4 codes, element 0 in bits
+// 0..3: bytes of the even elements, and of the odd elements shifted up a nibble.
 __device__ __forceinline__ uint32_t pack_i4x8(const uint32_t (&c)[8]) {
-  return nibble_pack(pack_i8x4(c[0], c[1], c[2], c[3]), pack_i8x4(c[4], c[5], c[6], c[7]));
+  const uint32_t e = pack_i8x4(c[0], c[2], c[4], c[6]);
+  const uint32_t o = pack_i8x4(c[1], c[3], c[5], c[7]);
+  return (e & 0x0f0f0f0fu) | ((o << 4) & 0xf0f0f0f0u);
 }
 
 // Codes of eight values against one group maximum `m` (of the same, unnormalised
@@ -140,6 +181,35 @@ __device__ __forceinline__ void quantize8(const float* v, float m, float qmax, u
     const float inv = m > 0.0f ? qmax / (m * pre) : 0.0f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) cc[k] = magic_code(v[k] * pre, inv);
+  }
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only), with group commit/wait.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Code multiplier of one group: inv = qmax / m, or, for a group maximum so
+// small that this overflows, qmax / (m * 2^64) applied to v * 2^64.
+struct QInv {
+  float inv;
+  bool tiny;
+};
+__device__ __forceinline__ QInv make_qinv(float m, float qmax) {
+  if (m >= kTinyMax) return {qmax / m, false};
+  return {m > 0.0f ? qmax / (m * 18446744073709551616.0f) : 0.0f, true};
+}
+__device__ __forceinline__ void quantize8q(const float* v, QInv q, uint32_t (&cc)[8]) {
+  if (!q.tiny) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cc[k] = magic_code(v[k], q.inv);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cc[k] = magic_code(v[k] * 18446744073709551616.0f, q.inv);
   }
 }
 

@@ -42,7 +42,7 @@ __device__ __forceinline__ int code_of(float v, float m, float qmax) {
   return (int)(b - 0x4b400000u);  // bit pattern of kMagic
 }
 
-__device__ void generic_stages(float* buf, int dim, int B) {
+__device__ __forceinline__ void generic_stages(float* buf, int dim, int B) {
   for (int h = 1; h < B; h <<= 1) {
     for (int p = threadIdx.x; p < dim / 2; p += blockDim.x) {
       const int i = ((p & ~(h - 1)) << 1) | (p & (h - 1));
@@ -107,11 +107,23 @@ __global__ void __launch_bounds__(256) rq_generic_kernel(GenericArgs a) {
 template <int BITS>
 __global__ void __launch_bounds__(256) dq_generic_kernel(GenericArgs a, bool out_f32) {
   extern __shared__ __align__(16) float sbuf[];
-  const int dim = a.dim, G = a.group;
+  const int dim = a.dim, G = a.group, B = a.block;
   const int ngroups = dim / G;
+  const int nblk = dim / B;
+  uint8_t* sflag = reinterpret_cast<uint8_t*>(sbuf + dim);  // per block: computed at 2^64 scale
 
   for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
     const int64_t base = row * dim;
+    const float* srow = a.scales_in + row * ngroups;
+    for (int b = threadIdx.x; b < nblk; b += blockDim.x) {
+      bool tiny = false;
+      for (int g = (b * B) / G; g <= ((b + 1) * B - 1) / G; ++g) {
+        const float sc = srow[g];
+        tiny |= sc < kTinyScale && sc != 0.0f;
+      }
+      sflag[b] = tiny;
+    }
+    __syncthreads();
     for (int i = threadIdx.x; i < dim; i += blockDim.x) {
       int qv;
       if constexpr (BITS == 8) {
@@ -120,12 +132,14 @@ __global__ void __launch_bounds__(256) dq_generic_kernel(GenericArgs a, bool out
         const uint32_t byte = a.codes_in[(base + i) >> 1];
         qv = ((int32_t)((byte >> (4 * (i & 1))) << 28)) >> 28;
       }
-      sbuf[i] = (float)qv * (a.scales_in[row * ngroups + i / G] * a.rsqrt_b);
+      const float pre = sflag[i / B] ? kUp64 : 1.0f;
+      sbuf[i] = (float)qv * (srow[i / G] * pre * a.rsqrt_b);
     }
     __syncthreads();
-    generic_stages(sbuf, dim, a.block);
+    generic_stages(sbuf, dim, B);
     for (int i = threadIdx.x; i < dim; i += blockDim.x) {
       float f = sbuf[i];
+      if (sflag[i / B]) f *= kDown64;
       if (a.signs && a.signs[i] < 0) f = -f;
       if (out_f32) {
         a.rot[base + i] = f;

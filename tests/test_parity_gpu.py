@@ -73,19 +73,23 @@ def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", o
 
 # (rows, dim, block, group, bits, signs, expected forward path)
 CASES = [
-    (300, 128, -1, -1, 8, False, "blocked"),        # Q/K heads, INT8, per row
-    (301, 128, 128, 128, 4, False, "blocked"),      # KV rows, INT4, group 128
-    (37, 4096, 128, -1, 4, False, "blocked"),       # per-token scale over 32 blocks
-    (9, 11008, 128, 128, 4, True, "blocked"),       # 86 blocks, signs
-    (5, 11008, 128, -1, 8, True, "blocked"),        # 86 blocks, one scale per row
-    (65, 256, 32, 8, 4, False, "blocked"),          # groups smaller than a block
-    (70, 512, 64, 16, 8, True, "blocked"),
-    (33, 1024, 256, 64, 4, True, "blocked"),
+    (300, 128, -1, -1, 8, False, "chunk"),          # Q/K heads, INT8, per row
+    (301, 128, 128, 128, 4, False, "chunk"),        # KV rows, INT4, group 128
+    (37, 4096, 128, -1, 4, False, "chunk"),         # per-token scale over 32 blocks
+    (9, 11008, 128, 128, 4, True, "chunk"),         # 86 blocks, signs
+    (5, 11008, 128, -1, 8, True, "chunk"),          # 86 blocks, one scale per row
+    (300, 256, 32, 8, 4, False, "chunk"),           # groups smaller than a block
+    (70, 512, 64, 16, 8, True, "chunk"),
+    (140, 384, 16, 32, 4, True, "chunk"),           # groups wider than blocks, inside a chunk
+    (40, 2048, 32, 256, 8, False, "chunk"),         # groups of two chunks
+    (3, 16384, 128, -1, 4, True, "chunk"),          # one row per slab
+    (33, 1152, 8, 64, 8, False, "chunk"),           # 8-point blocks, 9 chunks per row
+    (5, 32768, 128, 128, 4, True, "chunk"),         # widest row, groups inside chunks
+    (33, 1024, 256, 64, 4, True, "blocked"),        # 256-point blocks
     (17, 768, 256, -1, 8, False, "blocked"),        # row of three 256-blocks
-    (40, 2048, 32, 256, 8, False, "blocked"),       # groups of 8 blocks
-    (3, 16384, 128, -1, 4, True, "blocked"),        # widest blocked row (512 threads)
     (6, 8192, 256, 1024, 8, True, "blocked"),
-    (129, 64, 64, 32, 4, False, "blocked"),
+    (129, 64, 64, 32, 4, False, "blocked"),         # dim not a multiple of 128
+    (61, 96, 32, 8, 8, True, "blocked"),
     (21, 4096, -1, -1, 4, True, "full4096"),        # full 4096 + signs, per token
     (19, 4096, -1, 128, 8, False, "full4096"),
     (7, 4096, 4096, 64, 4, True, "full4096"),
@@ -99,7 +103,7 @@ CASES = [
     (6, 100, 4, 10, 4, False, "generic"),
     (3, 2048, -1, -1, 8, True, "generic"),
     (12, 24, 8, 8, 4, False, "generic"),
-    (2, 32768, 128, 128, 4, False, "generic"),      # widest row
+    (2, 32768, 128, -1, 4, False, "generic"),       # widest row, one scale per row
     (1, 1, 1, 1, 8, False, "generic"),
     (50, 64, 16, 16, 8, True, "generic"),
     (3, 6, 2, 6, 4, False, "generic"),
