@@ -214,14 +214,20 @@ def _barrier(world):
         dist.barrier()
 
 
-def _max_over_ranks(world, value: float) -> float:
+def _max_over_ranks(world, value: float, device="cuda") -> float:
+    """Max of a per-rank duration over all ranks (the job's time)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(world: int, bytes_per_step: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch (weak scaling)."""
+    return world * bytes_per_step * steps / (total_ms * 1e-3) / 1e9
 
 
 def run_ours(args):
@@ -284,7 +290,7 @@ def run_ours(args):
     if rank != 0:
         return None
     bytes_step = st.bytes_per_step
-    value = world * bytes_step * steps / (total_ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, bytes_step, steps, total_ms)
     peak, peak_kind = measured_peaks()
     q_bytes = wl.quant_bytes()
     q_ms = sum(quant_ms) / len(quant_ms)

@@ -88,7 +88,8 @@ hadq_status check_sizes(int64_t rows, int32_t dim, int32_t block, int32_t bits, 
 bool blocked_group_ok(int G, int B) { return (is_pow2(G) && G >= 8 && G <= B) || (G % B == 0); }
 
 bool chunk_ok(int direction, const Shape& s) {
-  if (direction != 0 || s.B < 8 || s.B > 128 || s.dim % 128) return false;
+  (void)direction;
+  if (s.B < 8 || s.B > 128 || s.dim % 128) return false;
   if (is_pow2(s.G) && s.G >= 8 && s.G <= 128) return true;
   return s.G % 128 == 0 && s.dim <= 128 * hadq::kCT;  // a slab holds whole rows
 }
@@ -192,16 +193,16 @@ hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, b
 
 // ----------------------------------------------------------------- chunk
 
-hadq_status launch_chunk(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool f32, cudaStream_t stream) {
   a.cpr = s.dim / hadq::kCK;
   a.nchunks = s.rows * a.cpr;
-  a.slab_chunks = s.G > hadq::kCK ? (hadq::kCT / a.cpr) * a.cpr : hadq::kCT;
-  a.nslabs = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
   a.G = s.G;
   a.dim = s.dim;
   a.log_g = s.G <= hadq::kCK ? ilog2(s.G) : -1;
   a.gpc = s.G > hadq::kCK ? s.G / hadq::kCK : 1;
-  const void* fn = hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK);
+  a.slab_chunks = (hadq::kCT / a.gpc) * a.gpc;  // a slab never splits a scale group
+  const void* fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK)
+                                  : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
@@ -210,7 +211,8 @@ hadq_status launch_chunk(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream)
                 cudaGetErrorString(e));
   }
   const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
-  const unsigned grid = (unsigned)(a.nslabs < cap ? a.nslabs : cap);
+  const int64_t want = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;  // number of slabs
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
   e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
   if (e != cudaSuccess) {
@@ -341,7 +343,7 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.rot = rotated_out;
     a.scale_mul = scale_mul;
     a.rsqrt_b = rsqrt_b;
-    return launch_chunk(s, a, cs);
+    return launch_chunk(0, s, a, false, cs);
   }
   if (path == HADQ_PATH_FULL4096) {
     hadq::FullArgs a{};
@@ -385,6 +387,16 @@ hadq_status hadq_dequant_rotate_inv(const void* codes, const float* scales, int6
   const hadq_path path = choose_path(1, s, a16);
   const float rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == HADQ_PATH_CHUNK) {
+    hadq::ChunkArgs a{};
+    a.codes_in = static_cast<const uint8_t*>(codes);
+    a.scales_in = scales;
+    a.signs = signs;
+    a.rot = f32 ? static_cast<float*>(out) : nullptr;
+    a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+    a.rsqrt_b = rsqrt_b;
+    return launch_chunk(1, s, a, f32, cs);
+  }
   if (path == HADQ_PATH_BLOCKED) {
     hadq::BlockedArgs a{};
     a.codes_in = static_cast<const uint8_t*>(codes);

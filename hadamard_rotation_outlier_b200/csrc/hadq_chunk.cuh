@@ -36,9 +36,8 @@ struct ChunkArgs {
   float* rot;                // forward: optional fp32 y; inverse: fp32 output
   uint16_t* out_bf16;
   int64_t nchunks;           // rows * dim / 128
-  int64_t nslabs;
   int cpr;                   // chunks per row
-  int slab_chunks;           // chunks per slab (<= 128)
+  int slab_chunks;           // chunks per slab (<= 128, a multiple of gpc)
   int G;
   int log_g;                 // log2(G) when G <= 128, else -1
   int gpc;                   // chunks per group when G > 128, else 1
@@ -46,6 +45,13 @@ struct ChunkArgs {
   float scale_mul;
   float rsqrt_b;
 };
+
+// Slabs are dealt round-robin (slab s goes to CTA s mod gridDim.x): at any
+// moment the CTAs of the grid work on one compact window of memory, which
+// measured faster than giving each CTA a contiguous range.
+__device__ __forceinline__ int64_t nslabs_of(const ChunkArgs& a) {
+  return (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
+}
 
 // Shared-memory layout shared by host and device.
 __host__ __device__ constexpr int chunk_stage_bytes() { return kCT * kCPad; }
@@ -95,8 +101,9 @@ __device__ __forceinline__ void chunk_store(const uint8_t* src, int nch, uint8_t
   }
 }
 
-__device__ __forceinline__ int slab_count(int64_t nchunks, int64_t slab, int slab_chunks) {
-  const int64_t left = nchunks - slab * slab_chunks;
+// Chunks of the slab starting at chunk c (the last slab may be short).
+__device__ __forceinline__ int slab_count(int64_t c, int64_t nchunks, int slab_chunks) {
+  const int64_t left = nchunks - c;
   return left < slab_chunks ? (int)left : slab_chunks;
 }
 
@@ -146,6 +153,7 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
   for (int i = tid; i < 2 * kCT; i += kCT) s_gmax[i] = 0u;
 
   const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
+  const int64_t nslabs = nslabs_of(a);
   // Column chunk of this thread's chunk, advanced from slab to slab (sign
   // masks only); group bookkeeping for groups spanning several chunks.
   int colc = SIGNS ? (int)(((int64_t)blockIdx.x * a.slab_chunks + tid) % a.cpr) : 0;
@@ -155,20 +163,22 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
   const int groups_per_slab = multi ? a.slab_chunks / a.gpc : 0;
 
   int64_t slab = blockIdx.x;
-  if (slab < a.nslabs) chunk_load<16>(xsrc + slab * a.slab_chunks * 256, slab_count(a.nchunks, slab, a.slab_chunks), stage0);
+  if (slab < nslabs) chunk_load<16>(xsrc + slab * a.slab_chunks * 256, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), stage0);
   cp_async_commit();
-  for (int it = 0; slab < a.nslabs; ++it, slab += gridDim.x) {
+  for (int it = 0; slab < nslabs; ++it, slab += gridDim.x) {
     uint8_t* cur = (it & 1) ? stage1 : stage0;
+    const int64_t c = slab * a.slab_chunks;
     cp_async_wait<0>();
     __syncthreads();  // slab data visible; the other stage is free again
     {
       const int64_t nx = slab + gridDim.x;
-      if (nx < a.nslabs)
-        chunk_load<16>(xsrc + nx * a.slab_chunks * 256, slab_count(a.nchunks, nx, a.slab_chunks), (it & 1) ? stage0 : stage1);
+      if (nx < nslabs)
+        chunk_load<16>(xsrc + nx * a.slab_chunks * 256, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
+                       (it & 1) ? stage0 : stage1);
       cp_async_commit();
     }
-    const int nch = slab_count(a.nchunks, slab, a.slab_chunks);
-    const int64_t ch = slab * a.slab_chunks + tid;
+    const int nch = slab_count(c, a.nchunks, a.slab_chunks);
+    const int64_t ch = c + tid;
     const bool active = tid < nch;
     const int col0 = colc * kCK;
     if constexpr (SIGNS) {
@@ -278,7 +288,169 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
       chunk_codes<BITS>(v, inv, mine);
     }
     __syncthreads();
-    chunk_store<CB / 16>(cur, nch, a.codes + slab * a.slab_chunks * CB);
+    chunk_store<CB / 16>(cur, nch, a.codes + c * CB);
+  }
+  cp_async_wait<0>();
+}
+
+// Inverse: codes * scale -> H_B -> signs -> bf16 (or fp32).
+//
+// When every Hadamard block lies inside one scale group (G >= B), the
+// butterflies run on the integer codes themselves (exact in float32: the sums
+// stay at or below 128 * 127) and each vector is scaled once afterwards, by
+// scale / sqrt(B).  Otherwise (G < B) the codes are scaled first.
+template <int LOG_B, int BITS, bool SIGNS, bool SCALE_FIRST, bool OUT_F32>
+__global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
+  constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint8_t* stage0 = smem;
+  uint8_t* stage1 = smem + chunk_stage_bytes();
+  uint32_t* s_msk = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes()) + 2 * kCT;
+  const int tid = threadIdx.x;
+  const int G = a.G;
+
+  if constexpr (SIGNS) {
+    for (int p = tid; p < a.dim / 2; p += kCT)
+      s_msk[mask_slot(p)] = pair_sign_mask(a.signs[2 * p], a.signs[2 * p + 1]);
+  }
+  const int64_t nslabs = nslabs_of(a);
+  int colc = SIGNS ? (int)(((int64_t)blockIdx.x * a.slab_chunks + tid) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)(((int64_t)gridDim.x * a.slab_chunks) % a.cpr) : 0;
+
+  int64_t slab = blockIdx.x;
+  if (slab < nslabs)
+    chunk_load<CB / 16>(a.codes_in + slab * a.slab_chunks * CB, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), stage0);
+  cp_async_commit();
+  for (int it = 0; slab < nslabs; ++it, slab += gridDim.x) {
+    uint8_t* cur = (it & 1) ? stage1 : stage0;
+    const int64_t c = slab * a.slab_chunks;
+    cp_async_wait<0>();
+    __syncthreads();
+    {
+      const int64_t nx = slab + gridDim.x;
+      if (nx < nslabs)
+        chunk_load<CB / 16>(a.codes_in + nx * a.slab_chunks * CB, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
+                            (it & 1) ? stage0 : stage1);
+      cp_async_commit();
+    }
+    const int nch = slab_count(c, a.nchunks, a.slab_chunks);
+    const int64_t ch = c + tid;
+    const bool active = tid < nch;
+    const int col0 = colc * kCK;
+    if constexpr (SIGNS) {
+      colc += col_step;
+      if (colc >= a.cpr) colc -= a.cpr;
+    }
+    uint8_t* mine = cur + tid * kCPad;
+
+    if (active) {
+      // per-vector scale (a group covers >= 8 columns)
+      float sc[16];
+      if (G >= kCK) {
+        const float s0 = __ldg(a.scales_in + (a.gpc == 1 ? ch : ch / a.gpc));
+#pragma unroll
+        for (int p = 0; p < 16; ++p) sc[p] = s0;
+      } else {
+        const int lg = a.log_g;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) sc[p] = __ldg(a.scales_in + (((ch * kCK) + 8 * p) >> lg));
+      }
+      // Scales below 2^-100 would give subnormal factors (scale / sqrt(B)) or
+      // butterflies on subnormal values: those take factors at 2^64 scale and
+      // one exact 2^-64 rescale at the end.
+      bool tiny = false;
+#pragma unroll
+      for (int p = 0; p < 16; ++p) tiny |= sc[p] < kTinyScale && sc[p] != 0.0f;
+      float v[kCK];
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        if constexpr (BITS == 8) {
+          const uint2 r = *reinterpret_cast<const uint2*>(mine + 8 * p);
+          i8x4_to_float(r.x, v + 8 * p);
+          i8x4_to_float(r.y, v + 8 * p + 4);
+        } else {
+          i4x8_to_float(*reinterpret_cast<const uint32_t*>(mine + 4 * p), v + 8 * p);
+        }
+      }
+      const float pre = tiny ? kUp64 : 1.0f;
+      if constexpr (SCALE_FIRST) {
+        // the whole chunk runs at 2^64 scale when any of its scales is tiny
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float f = (sc[p] * pre) * a.rsqrt_b;
+#pragma unroll
+          for (int k = 0; k < 8; k += 2) mul2(v[8 * p + k], v[8 * p + k + 1], f);
+        }
+        reg_fwht<kCK, LOG_B>(v);
+        if (tiny) {
+#pragma unroll
+          for (int i = 0; i < kCK; i += 2) mul2(v[i], v[i + 1], kDown64);
+        }
+      } else {
+        // butterflies on the integer codes (exact), then one factor per vector
+        reg_fwht<kCK, LOG_B>(v);
+        if (!tiny) {
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const float f = sc[p] * a.rsqrt_b;
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) mul2(v[8 * p + k], v[8 * p + k + 1], f);
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {
+            const bool t = sc[p] < kTinyScale;
+            const float f = (sc[p] * (t ? kUp64 : 1.0f)) * a.rsqrt_b;
+            const float g = t ? kDown64 : 1.0f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[8 * p + k] = (v[8 * p + k] * f) * g;
+          }
+        }
+      }
+      if constexpr (OUT_F32) {
+        float* dst = a.rot + ch * kCK;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t lo = __float_as_uint(v[8 * p + 2 * i]), hi = __float_as_uint(v[8 * p + 2 * i + 1]);
+            if constexpr (SIGNS) {
+              const uint32_t m = s_msk[mask_slot(col0 / 2 + 4 * p + i)];
+              lo ^= m << 16;
+              hi ^= m & 0x80000000u;
+            }
+            o[2 * i] = lo;
+            o[2 * i + 1] = hi;
+          }
+          reinterpret_cast<uint4*>(dst + 8 * p)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+          reinterpret_cast<uint4*>(dst + 8 * p)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t r;
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v[8 * p + 2 * i + 1]), "f"(v[8 * p + 2 * i]));
+            o[i] = r;
+          }
+          if constexpr (SIGNS) {
+            const uint4 m4 = *reinterpret_cast<const uint4*>(s_msk + mask_slot(col0 / 2 + 4 * p));
+            o[0] ^= m4.x;
+            o[1] ^= m4.y;
+            o[2] ^= m4.z;
+            o[3] ^= m4.w;
+          }
+          *reinterpret_cast<uint4*>(mine + 16 * p) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+    }
+    if constexpr (!OUT_F32) {
+      __syncthreads();
+      chunk_store<16>(cur, nch, reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256);
+    }
   }
   cp_async_wait<0>();
 }

@@ -213,6 +213,47 @@ __device__ __forceinline__ void quantize8q(const float* v, QInv q, uint32_t (&cc
   }
 }
 
+// Paired FP32 ops on two registers with one shared operand.
+__device__ __forceinline__ void add2(float& a, float& b, float c) {
+  uint64_t X, C, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(C) : "f"(c));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(R) : "l"(X), "l"(C));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(R));
+}
+__device__ __forceinline__ void mul2(float& a, float& b, float c) {
+  uint64_t X, C, R;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(X) : "f"(a), "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(C) : "f"(c));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(R) : "l"(X), "l"(C));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(R));
+}
+
+// Codes to floats without integer-to-float conversions: a biased code u
+// (0 <= u < 256) placed in the low mantissa byte of 2^23 gives the float
+// 2^23 + u exactly; subtracting 2^23 + bias recovers the signed code.
+// Eight int4 codes of word w -> v[0..7].
+__device__ __forceinline__ void i4x8_to_float(uint32_t w, float* v) {
+  const uint32_t x = w ^ 0x88888888u;           // nibble n -> n + 8 in [0, 15]
+  const uint32_t e = x & 0x0f0f0f0fu;           // elements 0, 2, 4, 6
+  const uint32_t o = (x >> 4) & 0x0f0f0f0fu;    // elements 1, 3, 5, 7
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(__byte_perm(e, 0x4b000000u, 0x7440 + i));
+    v[2 * i + 1] = __uint_as_float(__byte_perm(o, 0x4b000000u, 0x7440 + i));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) add2(v[i], v[i + 1], -8388616.0f);  // -(2^23 + 8)
+}
+// Four int8 codes of word w -> v[0..3].
+__device__ __forceinline__ void i8x4_to_float(uint32_t w, float* v) {
+  const uint32_t x = w ^ 0x80808080u;           // n -> n + 128 in [0, 255]
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(__byte_perm(x, 0x4b000000u, 0x7440 + i));
+#pragma unroll
+  for (int i = 0; i < 4; i += 2) add2(v[i], v[i + 1], -8388736.0f);  // -(2^23 + 128)
+}
+
 // Sign-extended int4 nibble k of word w, as float.
 __device__ __forceinline__ float i4_at(uint32_t w, int k) {
   return (float)(((int32_t)(w << (28 - 4 * k))) >> 28);

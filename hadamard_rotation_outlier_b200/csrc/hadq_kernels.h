@@ -8,6 +8,12 @@ namespace hadq {
 const void* blocked_kernel_ptr(int direction, int bits, int B, bool signs, bool f32, int threads);
 // wide_g: the scale group covers whole 128-column chunks (G >= 128).
 const void* chunk_kernel_ptr(int bits, int B, bool signs, bool wide_g);
+// scale_first: some Hadamard block spans several scale groups (G < B).
+const void* dq_chunk_kernel_ptr_8(int B, bool signs, bool scale_first, bool f32);
+const void* dq_chunk_kernel_ptr_4(int B, bool signs, bool scale_first, bool f32);
+inline const void* dq_chunk_kernel_ptr(int bits, int B, bool signs, bool scale_first, bool f32) {
+  return bits == 8 ? dq_chunk_kernel_ptr_8(B, signs, scale_first, f32) : dq_chunk_kernel_ptr_4(B, signs, scale_first, f32);
+}
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);
 const void* generic_kernel_ptr(int direction, int bits);
 

@@ -77,7 +77,8 @@ def test_plan_rejects(lib, args, msg):
     (0, 256, 4096, 128, 4, -1, False, True, "chunk"),             # per-token over 32 blocks
     (0, 16384, 4096, -1, 4, -1, True, True, "full4096"),          # full 4096 + signs
     (0, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV cache
-    (1, 2097152, 128, 128, 4, 128, False, True, "blocked"),       # KV dequant
+    (1, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV dequant
+    (1, 10, 1024, 256, 4, 64, False, True, "blocked"),            # 256-point dequant
     (0, 32768, 11008, 128, 4, 128, True, True, "chunk"),          # 86 blocks of 128
     (0, 10, 1024, 256, 4, 64, True, True, "blocked"),             # 256-point blocks
     (0, 10, 96, 32, 8, -1, False, True, "blocked"),               # dim not a multiple of 128
