@@ -200,8 +200,11 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   a.dim = s.dim;
   a.log_g = s.G <= hadq::kCK ? ilog2(s.G) : -1;
   a.gpc = s.G > hadq::kCK ? s.G / hadq::kCK : 1;
-  a.slab_chunks = (hadq::kCT / a.gpc) * a.gpc;  // a slab never splits a scale group
-  const void* fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK)
+  // Warp teams (slabs of 32 chunks) unless a scale group spans a chunk count
+  // that does not divide 32; the dequantiser needs no group reduction.
+  const int team = (direction == 1 || (32 % a.gpc) == 0) ? 32 : hadq::kCT;
+  a.slab_chunks = team == 32 ? 32 : (hadq::kCT / a.gpc) * a.gpc;  // a slab never splits a group
+  const void* fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK, team)
                                   : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -211,7 +214,8 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
                 cudaGetErrorString(e));
   }
   const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
-  const int64_t want = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;  // number of slabs
+  const int64_t teams = team == 32 ? hadq::kCT / 32 : 1;
+  const int64_t want = ((a.nchunks + a.slab_chunks - 1) / a.slab_chunks + teams - 1) / teams;  // CTAs for one slab per team
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
   e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);

@@ -1,21 +1,28 @@
 // Chunk path: Hadamard blocks of B = 8..128 columns, dim a multiple of 128.
 //
 // Every thread owns one 128-element chunk of a row (chunks never cross rows),
-// so all log2(B) butterfly stages run in registers with no shuffles.  A CTA of
-// 128 threads walks over slabs of consecutive chunks, which are contiguous in
-// memory.  Each slab is staged through shared memory:
+// so all log2(B) butterfly stages run in registers with no shuffles.
 //
+// Teams.  Work is dealt in slabs of consecutive chunks, which are contiguous
+// in memory.  A slab belongs to a team: one warp (32 chunks) whenever no scale
+// group spans more than a warp's chunks, otherwise the whole CTA (128 threads).
+// A warp team synchronises with __syncwarp only, so warps never wait on each
+// other.  Slabs are dealt round-robin over all teams of the grid, so at any
+// moment the grid works on one compact window of memory.
+//
+// Each slab is staged through shared memory:
 //   load   16-byte cp.async copies, consecutive lanes on consecutive 16-byte
 //          pieces (fully coalesced), into chunk slots padded to 272 bytes so
 //          that a thread reading its own chunk row-wise is bank-conflict free.
-//          Two stages: the next slab streams in while this one is computed.
-//   store  each thread writes its codes back into its own slot; after a
-//          barrier the CTA copies the slab's codes out with coalesced 16-byte
+//          Two stages per team: the next slab streams in while this one is
+//          computed.
+//   store  each thread writes its results back into its own slot; after a
+//          team barrier the team copies them out with coalesced 16-byte
 //          stores (they too are contiguous in memory).
 //
 // Scale groups: G = 2^g with 8 <= G <= 128 reduce inside the thread; groups of
-// several chunks (G a multiple of 128) reduce with one shared-memory max per
-// slab, and then a slab holds whole rows so that no group straddles two slabs.
+// gpc = G/128 chunks reduce with lane shuffles (warp team, gpc divides 32) or
+// one shared-memory max per slab (CTA team); a slab always holds whole groups.
 #pragma once
 
 #include "hadq_common.cuh"
@@ -37,7 +44,7 @@ struct ChunkArgs {
   uint16_t* out_bf16;
   int64_t nchunks;           // rows * dim / 128
   int cpr;                   // chunks per row
-  int slab_chunks;           // chunks per slab (<= 128, a multiple of gpc)
+  int slab_chunks;           // chunks per slab: 32 (warp team) or <= 128, a multiple of gpc
   int G;
   int log_g;                 // log2(G) when G <= 128, else -1
   int gpc;                   // chunks per group when G > 128, else 1
@@ -46,14 +53,9 @@ struct ChunkArgs {
   float rsqrt_b;
 };
 
-// Slabs are dealt round-robin (slab s goes to CTA s mod gridDim.x): at any
-// moment the CTAs of the grid work on one compact window of memory, which
-// measured faster than giving each CTA a contiguous range.
-__device__ __forceinline__ int64_t nslabs_of(const ChunkArgs& a) {
-  return (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
-}
-
-// Shared-memory layout shared by host and device.
+// Shared-memory layout shared by host and device: two stages of kCT slots
+// (split per team), a [2][kCT] group-max area (CTA teams) and the pair sign
+// masks of one row.
 __host__ __device__ constexpr int chunk_stage_bytes() { return kCT * kCPad; }
 __host__ __device__ inline int chunk_mask_words(int dim) { return dim / 2 + 4 * (dim / 128); }
 __host__ __device__ inline size_t chunk_smem_bytes(int dim, bool signs) {
@@ -65,38 +67,51 @@ __host__ __device__ inline size_t chunk_smem_bytes(int dim, bool signs) {
 // threads reading the masks of consecutive chunks hit different banks.
 __device__ __forceinline__ int mask_slot(int pair) { return pair + 4 * (pair >> 6); }
 
+// A team of TEAM threads (32: one warp, 128: the CTA) owning one slab at a time.
+template <int TEAM>
+struct Team {
+  static_assert(TEAM == 32 || TEAM == kCT, "warp or CTA teams");
+  static constexpr int PER_CTA = kCT / TEAM;
+  __device__ static int index() { return TEAM == 32 ? (int)(threadIdx.x >> 5) : 0; }
+  __device__ static int tid() { return (int)threadIdx.x & (TEAM - 1); }
+  __device__ static void sync() {
+    if constexpr (TEAM == 32) __syncwarp(); else __syncthreads();
+  }
+  // this team's two stages of TEAM slots
+  __device__ static uint8_t* stage(uint8_t* smem, int s) { return smem + (index() * 2 + s) * TEAM * kCPad; }
+  __device__ static int64_t first() { return (int64_t)blockIdx.x * PER_CTA + index(); }
+  __device__ static int64_t stride() { return (int64_t)gridDim.x * PER_CTA; }
+};
 
-// Copies `nch` chunks of `bytes_per_chunk` (16 * PPC) bytes starting at `src`
-// into padded slots of `dst`.  Consecutive threads take consecutive 16-byte
-// pieces, so every warp reads 512 contiguous bytes.  Full slabs use a fully
+// Copies `nch` chunks of 16 * PPC bytes starting at `src` into padded slots of
+// `dst`.  Consecutive team threads take consecutive 16-byte pieces, so every
+// warp reads 512 contiguous bytes per instruction.  Full slabs use a fully
 // unrolled loop with constant strides.
-template <int PPC>
-__device__ __forceinline__ void chunk_load(const uint8_t* src, int nch, uint8_t* dst) {
-  const int tid = threadIdx.x;
-  if (nch == kCT) {
-    constexpr int STEP = kCT / PPC;  // chunks covered by one pass of the CTA
-    const uint8_t* s0 = src + 16 * tid;
-    uint8_t* d0 = dst + (tid / PPC) * kCPad + 16 * (tid % PPC);
+template <int PPC, int TEAM>
+__device__ __forceinline__ void chunk_load(const uint8_t* src, int nch, uint8_t* dst, int tt) {
+  if (nch == TEAM) {
+    constexpr int STEP = TEAM / PPC;  // chunks covered by one pass of the team
+    const uint8_t* s0 = src + 16 * tt;
+    uint8_t* d0 = dst + (tt / PPC) * kCPad + 16 * (tt % PPC);
 #pragma unroll
-    for (int i = 0; i < PPC; ++i) cp_async16(d0 + i * STEP * kCPad, s0 + i * 16 * kCT);
+    for (int i = 0; i < PPC; ++i) cp_async16(d0 + i * STEP * kCPad, s0 + i * 16 * TEAM);
   } else {
-    for (int g = tid; g < nch * PPC; g += kCT) cp_async16(dst + (g / PPC) * kCPad + 16 * (g % PPC), src + 16 * g);
+    for (int g = tt; g < nch * PPC; g += TEAM) cp_async16(dst + (g / PPC) * kCPad + 16 * (g % PPC), src + 16 * g);
   }
 }
 
 // Copies `nch` chunk results of 16 * PPC bytes from padded slots to `dst`.
-template <int PPC>
-__device__ __forceinline__ void chunk_store(const uint8_t* src, int nch, uint8_t* dst) {
-  const int tid = threadIdx.x;
-  if (nch == kCT) {
-    constexpr int STEP = kCT / PPC;
-    const uint8_t* s0 = src + (tid / PPC) * kCPad + 16 * (tid % PPC);
-    uint8_t* d0 = dst + 16 * tid;
+template <int PPC, int TEAM>
+__device__ __forceinline__ void chunk_store(const uint8_t* src, int nch, uint8_t* dst, int tt) {
+  if (nch == TEAM) {
+    constexpr int STEP = TEAM / PPC;
+    const uint8_t* s0 = src + (tt / PPC) * kCPad + 16 * (tt % PPC);
+    uint8_t* d0 = dst + 16 * tt;
 #pragma unroll
     for (int i = 0; i < PPC; ++i)
-      *reinterpret_cast<uint4*>(d0 + i * 16 * kCT) = *reinterpret_cast<const uint4*>(s0 + i * STEP * kCPad);
+      *reinterpret_cast<uint4*>(d0 + i * 16 * TEAM) = *reinterpret_cast<const uint4*>(s0 + i * STEP * kCPad);
   } else {
-    for (int g = tid; g < nch * PPC; g += kCT)
+    for (int g = tt; g < nch * PPC; g += TEAM)
       *reinterpret_cast<uint4*>(dst + 16 * g) = *reinterpret_cast<const uint4*>(src + (g / PPC) * kCPad + 16 * (g % PPC));
   }
 }
@@ -131,61 +146,69 @@ __device__ __forceinline__ void chunk_codes(const float (&v)[kCK], const float (
   }
 }
 
+// Loads the pair sign masks of one row into shared memory (all threads).
+__device__ __forceinline__ void load_sign_masks(const int8_t* signs, int dim, uint32_t* s_msk) {
+  for (int p = threadIdx.x; p < dim / 2; p += kCT) s_msk[mask_slot(p)] = pair_sign_mask(signs[2 * p], signs[2 * p + 1]);
+}
+
 // Forward: bf16 -> signs -> H_B (B = 2^LOG_B, 8..128) -> group max -> codes.
 // WIDE_G: the scale group covers whole chunks (G >= 128); otherwise 8 <= G < 128.
-template <int LOG_B, int BITS, bool SIGNS, bool WIDE_G>
+// TEAM: 32 (warp teams; groups of at most 32 chunks, gpc dividing 32) or 128.
+template <int LOG_B, int BITS, bool SIGNS, bool WIDE_G, int TEAM>
 __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
+  using T = Team<TEAM>;
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* stage0 = smem;
-  uint8_t* stage1 = smem + chunk_stage_bytes();
-  uint32_t* s_gmax = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes());  // [2][kCT]
+  uint32_t* s_gmax = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes());  // [2][kCT], CTA teams
   uint32_t* s_msk = s_gmax + 2 * kCT;
-  const int tid = threadIdx.x;
+  const int tt = T::tid();
   const int G = a.G;
   const bool multi = WIDE_G && G > kCK;  // groups spanning several chunks
 
-  if constexpr (SIGNS) {
-    for (int p = tid; p < a.dim / 2; p += kCT)
-      s_msk[mask_slot(p)] = pair_sign_mask(a.signs[2 * p], a.signs[2 * p + 1]);
+  if constexpr (SIGNS) load_sign_masks(a.signs, a.dim, s_msk);
+  if constexpr (TEAM == kCT) {
+    for (int i = threadIdx.x; i < 2 * kCT; i += kCT) s_gmax[i] = 0u;
   }
-  for (int i = tid; i < 2 * kCT; i += kCT) s_gmax[i] = 0u;
+  __syncthreads();  // masks and group-max area ready (the only CTA-wide barrier of warp teams)
 
   const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
-  const int64_t nslabs = nslabs_of(a);
+  const int64_t nslabs = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
   // Column chunk of this thread's chunk, advanced from slab to slab (sign
   // masks only); group bookkeeping for groups spanning several chunks.
-  int colc = SIGNS ? (int)(((int64_t)blockIdx.x * a.slab_chunks + tid) % a.cpr) : 0;
-  const int col_step = SIGNS ? (int)(((int64_t)gridDim.x * a.slab_chunks) % a.cpr) : 0;
-  const int wide_slot = multi ? tid / a.gpc : 0;
-  const bool wide_lead = multi ? (tid - wide_slot * a.gpc) == 0 : true;
+  int colc = SIGNS ? (int)((T::first() * a.slab_chunks + tt) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)((T::stride() * a.slab_chunks) % a.cpr) : 0;
+  const int gslot = multi ? tt / a.gpc : 0;         // group of this chunk inside its slab
+  const bool glead = multi ? (tt - gslot * a.gpc) == 0 : true;
   const int groups_per_slab = multi ? a.slab_chunks / a.gpc : 0;
+  uint8_t* st0 = T::stage(smem, 0);
+  uint8_t* st1 = T::stage(smem, 1);
 
-  int64_t slab = blockIdx.x;
-  if (slab < nslabs) chunk_load<16>(xsrc + slab * a.slab_chunks * 256, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), stage0);
+  int64_t slab = T::first();
+  if (slab < nslabs)
+    chunk_load<16, TEAM>(xsrc + slab * a.slab_chunks * 256, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), st0, tt);
   cp_async_commit();
-  for (int it = 0; slab < nslabs; ++it, slab += gridDim.x) {
-    uint8_t* cur = (it & 1) ? stage1 : stage0;
+  for (int it = 0; slab < nslabs; ++it, slab += T::stride()) {
+    uint8_t* cur = (it & 1) ? st1 : st0;
     const int64_t c = slab * a.slab_chunks;
     cp_async_wait<0>();
-    __syncthreads();  // slab data visible; the other stage is free again
+    T::sync();  // slab data visible; the other stage is free again
     {
-      const int64_t nx = slab + gridDim.x;
+      const int64_t nx = slab + T::stride();
       if (nx < nslabs)
-        chunk_load<16>(xsrc + nx * a.slab_chunks * 256, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
-                       (it & 1) ? stage0 : stage1);
+        chunk_load<16, TEAM>(xsrc + nx * a.slab_chunks * 256, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
+                             (it & 1) ? st0 : st1, tt);
       cp_async_commit();
     }
     const int nch = slab_count(c, a.nchunks, a.slab_chunks);
-    const int64_t ch = c + tid;
-    const bool active = tid < nch;
+    const int64_t ch = c + tt;
+    const bool active = tt < nch;
     const int col0 = colc * kCK;
     if constexpr (SIGNS) {
       colc += col_step;
       if (colc >= a.cpr) colc -= a.cpr;
     }
-    uint8_t* mine = cur + tid * kCPad;
+    uint8_t* mine = cur + tt * kCPad;
 
     float v[kCK];
     float pm[16];
@@ -222,12 +245,17 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
       gmax = pm[0];
 #pragma unroll
       for (int p = 1; p < 16; ++p) gmax = fmaxf(gmax, pm[p]);
-      if (multi) {
-        uint32_t* slot = s_gmax + (it & 1) * kCT + wide_slot;
-        if (active) atomicMax(slot, __float_as_uint(gmax));
-        __syncthreads();
-        gmax = __uint_as_float(*slot);
-        s_gmax[((it + 1) & 1) * kCT + tid] = 0u;  // read two slabs later, after two barriers
+      if constexpr (TEAM == 32) {
+        // groups of gpc consecutive lanes (gpc divides 32): butterfly max
+        for (int b = 1; b < a.gpc; b <<= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, b));
+      } else {
+        if (multi) {
+          uint32_t* slot = s_gmax + (it & 1) * kCT + gslot;
+          if (active) atomicMax(slot, __float_as_uint(gmax));
+          __syncthreads();
+          gmax = __uint_as_float(*slot);
+          s_gmax[((it + 1) & 1) * kCT + tt] = 0u;  // read two slabs later, after two barriers
+        }
       }
     } else {
 #pragma unroll
@@ -245,7 +273,7 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
     if (active) {
       // scale index = (flat element index of the group's first element) / G
       if constexpr (WIDE_G) {
-        if (wide_lead) a.scales[multi ? slab * groups_per_slab + wide_slot : ch] = gmax * a.scale_mul;
+        if (glead) a.scales[multi ? slab * groups_per_slab + gslot : ch] = gmax * a.scale_mul;
       } else {
         const int lg = a.log_g;
 #pragma unroll
@@ -287,69 +315,80 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
       }
       chunk_codes<BITS>(v, inv, mine);
     }
-    __syncthreads();
-    chunk_store<CB / 16>(cur, nch, a.codes + c * CB);
+    T::sync();
+    chunk_store<CB / 16, TEAM>(cur, nch, a.codes + c * CB, tt);
   }
   cp_async_wait<0>();
 }
 
-// Inverse: codes * scale -> H_B -> signs -> bf16 (or fp32).
+// Inverse: codes * scale -> H_B -> signs -> bf16 (or fp32), warp teams.
 //
 // When every Hadamard block lies inside one scale group (G >= B), the
 // butterflies run on the integer codes themselves (exact in float32: the sums
 // stay at or below 128 * 127) and each vector is scaled once afterwards, by
-// scale / sqrt(B).  Otherwise (G < B) the codes are scaled first.
+// scale / sqrt(B).  Otherwise (G < B) the codes are scaled first.  With one
+// scale per chunk (G >= 128) the scale of the next slab is loaded one slab
+// ahead.
 template <int LOG_B, int BITS, bool SIGNS, bool SCALE_FIRST, bool OUT_F32>
 __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
+  using T = Team<32>;
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* stage0 = smem;
-  uint8_t* stage1 = smem + chunk_stage_bytes();
   uint32_t* s_msk = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes()) + 2 * kCT;
-  const int tid = threadIdx.x;
+  const int tt = T::tid();
   const int G = a.G;
+  const bool one_scale = G >= kCK;
 
   if constexpr (SIGNS) {
-    for (int p = tid; p < a.dim / 2; p += kCT)
-      s_msk[mask_slot(p)] = pair_sign_mask(a.signs[2 * p], a.signs[2 * p + 1]);
-  }
-  const int64_t nslabs = nslabs_of(a);
-  int colc = SIGNS ? (int)(((int64_t)blockIdx.x * a.slab_chunks + tid) % a.cpr) : 0;
-  const int col_step = SIGNS ? (int)(((int64_t)gridDim.x * a.slab_chunks) % a.cpr) : 0;
-
-  int64_t slab = blockIdx.x;
-  if (slab < nslabs)
-    chunk_load<CB / 16>(a.codes_in + slab * a.slab_chunks * CB, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), stage0);
-  cp_async_commit();
-  for (int it = 0; slab < nslabs; ++it, slab += gridDim.x) {
-    uint8_t* cur = (it & 1) ? stage1 : stage0;
-    const int64_t c = slab * a.slab_chunks;
-    cp_async_wait<0>();
+    load_sign_masks(a.signs, a.dim, s_msk);
     __syncthreads();
+  }
+  const int64_t nslabs = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
+  int colc = SIGNS ? (int)((T::first() * a.slab_chunks + tt) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)((T::stride() * a.slab_chunks) % a.cpr) : 0;
+  uint8_t* st0 = T::stage(smem, 0);
+  uint8_t* st1 = T::stage(smem, 1);
+  auto chunk_scale = [&](int64_t ch) { return __ldg(a.scales_in + (a.gpc == 1 ? ch : ch / a.gpc)); };
+
+  int64_t slab = T::first();
+  float sc_next = 0.0f;
+  if (slab < nslabs) {
+    const int64_t c0 = slab * a.slab_chunks;
+    chunk_load<CB / 16, 32>(a.codes_in + c0 * CB, slab_count(c0, a.nchunks, a.slab_chunks), st0, tt);
+    if (one_scale && c0 + tt < a.nchunks) sc_next = chunk_scale(c0 + tt);
+  }
+  cp_async_commit();
+  for (int it = 0; slab < nslabs; ++it, slab += T::stride()) {
+    uint8_t* cur = (it & 1) ? st1 : st0;
+    const int64_t c = slab * a.slab_chunks;
+    const float sc_cur = sc_next;
+    cp_async_wait<0>();
+    T::sync();
     {
-      const int64_t nx = slab + gridDim.x;
-      if (nx < nslabs)
-        chunk_load<CB / 16>(a.codes_in + nx * a.slab_chunks * CB, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
-                            (it & 1) ? stage0 : stage1);
+      const int64_t nx = slab + T::stride();
+      if (nx < nslabs) {
+        const int64_t cn = nx * a.slab_chunks;
+        chunk_load<CB / 16, 32>(a.codes_in + cn * CB, slab_count(cn, a.nchunks, a.slab_chunks), (it & 1) ? st0 : st1, tt);
+        if (one_scale && cn + tt < a.nchunks) sc_next = chunk_scale(cn + tt);
+      }
       cp_async_commit();
     }
     const int nch = slab_count(c, a.nchunks, a.slab_chunks);
-    const int64_t ch = c + tid;
-    const bool active = tid < nch;
+    const int64_t ch = c + tt;
+    const bool active = tt < nch;
     const int col0 = colc * kCK;
     if constexpr (SIGNS) {
       colc += col_step;
       if (colc >= a.cpr) colc -= a.cpr;
     }
-    uint8_t* mine = cur + tid * kCPad;
+    uint8_t* mine = cur + tt * kCPad;
 
     if (active) {
       // per-vector scale (a group covers >= 8 columns)
       float sc[16];
-      if (G >= kCK) {
-        const float s0 = __ldg(a.scales_in + (a.gpc == 1 ? ch : ch / a.gpc));
+      if (one_scale) {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) sc[p] = s0;
+        for (int p = 0; p < 16; ++p) sc[p] = sc_cur;
       } else {
         const int lg = a.log_g;
 #pragma unroll
@@ -363,13 +402,18 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
       for (int p = 0; p < 16; ++p) tiny |= sc[p] < kTinyScale && sc[p] != 0.0f;
       float v[kCK];
 #pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        if constexpr (BITS == 8) {
-          const uint2 r = *reinterpret_cast<const uint2*>(mine + 8 * p);
-          i8x4_to_float(r.x, v + 8 * p);
-          i8x4_to_float(r.y, v + 8 * p + 4);
-        } else {
-          i4x8_to_float(*reinterpret_cast<const uint32_t*>(mine + 4 * p), v + 8 * p);
+      for (int q4 = 0; q4 < CB / 16; ++q4) {
+        const uint4 r = *reinterpret_cast<const uint4*>(mine + 16 * q4);
+        if constexpr (BITS == 8) {  // 16 codes: elements 16 q4 .. 16 q4 + 15
+          i8x4_to_float(r.x, v + 16 * q4);
+          i8x4_to_float(r.y, v + 16 * q4 + 4);
+          i8x4_to_float(r.z, v + 16 * q4 + 8);
+          i8x4_to_float(r.w, v + 16 * q4 + 12);
+        } else {                    // 32 codes: elements 32 q4 .. 32 q4 + 31
+          i4x8_to_float(r.x, v + 32 * q4);
+          i4x8_to_float(r.y, v + 32 * q4 + 8);
+          i4x8_to_float(r.z, v + 32 * q4 + 16);
+          i4x8_to_float(r.w, v + 32 * q4 + 24);
         }
       }
       const float pre = tiny ? kUp64 : 1.0f;
@@ -448,8 +492,8 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
       }
     }
     if constexpr (!OUT_F32) {
-      __syncthreads();
-      chunk_store<16>(cur, nch, reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256);
+      T::sync();
+      chunk_store<16, 32>(cur, nch, reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256, tt);
     }
   }
   cp_async_wait<0>();

@@ -6,8 +6,10 @@ namespace hadq {
 
 // direction 0 = rotate+quantise, 1 = dequantise+inverse; threads = CTA size.
 const void* blocked_kernel_ptr(int direction, int bits, int B, bool signs, bool f32, int threads);
-// wide_g: the scale group covers whole 128-column chunks (G >= 128).
-const void* chunk_kernel_ptr(int bits, int B, bool signs, bool wide_g);
+// wide_g: the scale group covers whole 128-column chunks (G >= 128);
+// team: 32 (warp teams) or 128 (CTA teams, for groups of more than 32 chunks
+// or of a chunk count that does not divide 32).
+const void* chunk_kernel_ptr(int bits, int B, bool signs, bool wide_g, int team);
 // scale_first: some Hadamard block spans several scale groups (G < B).
 const void* dq_chunk_kernel_ptr_8(int B, bool signs, bool scale_first, bool f32);
 const void* dq_chunk_kernel_ptr_4(int B, bool signs, bool scale_first, bool f32);

@@ -81,7 +81,9 @@ CASES = [
     (300, 256, 32, 8, 4, False, "chunk"),           # groups smaller than a block
     (70, 512, 64, 16, 8, True, "chunk"),
     (140, 384, 16, 32, 4, True, "chunk"),           # groups wider than blocks, inside a chunk
-    (40, 2048, 32, 256, 8, False, "chunk"),         # groups of two chunks
+    (40, 2048, 32, 256, 8, False, "chunk"),         # groups of two chunks (warp shuffle)
+    (20, 6144, 64, 2048, 8, True, "chunk"),         # groups of 16 chunks (warp shuffle)
+    (30, 768, 128, 384, 4, False, "chunk"),         # groups of 3 chunks (CTA shared-memory max)
     (3, 16384, 128, -1, 4, True, "chunk"),          # one row per slab
     (33, 1152, 8, 64, 8, False, "chunk"),           # 8-point blocks, 9 chunks per row
     (5, 32768, 128, 128, 4, True, "chunk"),         # widest row, groups inside chunks
