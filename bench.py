@@ -41,7 +41,8 @@ METRIC = "fused Hadamard+quantize GB/s (bf16 in→int4/int8 out), % of B200 HBM 
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
-                "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel", "none": None}
+                "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
+                "wide4096": "rq_wide4096_kernel", "none": None}
 
 
 def parse_args(argv=None):

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libhadq.so")
 
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
-PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk"}
+PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
 MAX_DIM = 32768
 
 EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_plan", "hadq_status_str",

@@ -97,6 +97,7 @@ bool chunk_ok(int direction, const Shape& s) {
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
+  if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096) return HADQ_PATH_WIDE4096;
   if (aligned16 && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) && s.dim % 32 == 0 &&
       s.dim <= 16384 && blocked_group_ok(s.G, s.B))
     return HADQ_PATH_BLOCKED;
@@ -206,7 +207,7 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   a.slab_chunks = team == 32 ? 32 : (hadq::kCT / a.gpc) * a.gpc;  // a slab never splits a group
   const void* fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK, team)
                                   : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
-  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs);
+  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, direction == 0 && team != 32);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -225,6 +226,35 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
     return fail(HADQ_ERR_CUDA, "chunk kernel launch failed: %s", cudaGetErrorString(e));
   }
   return after_launch("chunk kernel");
+}
+
+hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+  a.cpr = s.dim / hadq::kCK;
+  a.nchunks = s.rows * a.cpr;
+  a.slab_chunks = 32;
+  a.G = s.G;
+  a.dim = s.dim;
+  a.log_g = -1;
+  a.gpc = 32;
+  const void* fn = hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
+  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "4096-block kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                cudaGetErrorString(e));
+  }
+  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  const int64_t want = (a.nchunks / 32 + 3) / 4;  // one block per warp
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  void* args[] = {&a};
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "4096-block kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("4096-block kernel");
 }
 
 // ------------------------------------------------------------------ 4096
@@ -348,6 +378,17 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.scale_mul = scale_mul;
     a.rsqrt_b = rsqrt_b;
     return launch_chunk(0, s, a, false, cs);
+  }
+  if (path == HADQ_PATH_WIDE4096) {
+    hadq::ChunkArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.signs = signs;
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.rot = rotated_out;
+    a.scale_mul = scale_mul;
+    a.rsqrt_b = rsqrt_b;
+    return launch_wide4096(s, a, cs);
   }
   if (path == HADQ_PATH_FULL4096) {
     hadq::FullArgs a{};

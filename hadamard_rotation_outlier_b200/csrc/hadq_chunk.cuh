@@ -53,19 +53,41 @@ struct ChunkArgs {
   float rsqrt_b;
 };
 
-// Shared-memory layout shared by host and device: two stages of kCT slots
-// (split per team), a [2][kCT] group-max area (CTA teams) and the pair sign
-// masks of one row.
+// Shared-memory layout shared by host and device:
+//   [two stages of kCT slots][sign table, sign bits (SIGNS)][group max (CTA teams)]
+// The sign vector is kept as packed bits (one per column) plus a 256-entry
+// table mapping a byte of 8 sign bits to the four XOR masks of its bf16 pairs,
+// so the layout stays near 74 KB for any width (three CTAs per SM).
 __host__ __device__ constexpr int chunk_stage_bytes() { return kCT * kCPad; }
-__host__ __device__ inline int chunk_mask_words(int dim) { return dim / 2 + 4 * (dim / 128); }
-__host__ __device__ inline size_t chunk_smem_bytes(int dim, bool signs) {
-  return size_t(2) * chunk_stage_bytes() + 2 * kCT * sizeof(uint32_t) +
-         (signs ? size_t(chunk_mask_words(dim)) * sizeof(uint32_t) : 0);
+constexpr int kSignTabBytes = 256 * 16;
+__host__ __device__ inline int sign_bits_bytes(int dim) { return ((dim / 8) + 15) & ~15; }
+__host__ __device__ inline size_t chunk_smem_bytes(int dim, bool signs, bool cta_team) {
+  return size_t(2) * chunk_stage_bytes() + (signs ? size_t(kSignTabBytes + sign_bits_bytes(dim)) : 0) +
+         (cta_team ? size_t(2 * kCT * sizeof(uint32_t)) : 0);
 }
 
-// Pair sign masks are stored with 4 padding words after every 64, so that
-// threads reading the masks of consecutive chunks hit different banks.
-__device__ __forceinline__ int mask_slot(int pair) { return pair + 4 * (pair >> 6); }
+// Builds the sign table and the packed sign bits of one row (all threads; the
+// caller synchronises).  Bit b of word w is set when signs[32 w + b] < 0.
+__device__ __forceinline__ void load_sign_tables(const int8_t* signs, int dim, uint4* s_tab, uint32_t* s_bits) {
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    uint32_t m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = (((uint32_t)e >> (2 * k)) & 1u) << 15 | (((uint32_t)e >> (2 * k + 1)) & 1u) << 31;
+    s_tab[e] = make_uint4(m[0], m[1], m[2], m[3]);
+  }
+  for (int w = threadIdx.x; w < dim / 32; w += blockDim.x) {
+    uint32_t b = 0;
+    for (int i = 0; i < 32; ++i) b |= (uint32_t)(signs[32 * w + i] < 0) << i;
+    s_bits[w] = b;
+  }
+}
+
+// XOR masks of the 4 bf16 pairs of 8-column vector p of a chunk whose 128 sign
+// bits are `sb`.
+__device__ __forceinline__ uint4 sign_masks8(const uint4* s_tab, const uint4& sb, int p) {
+  const uint32_t w = (p >> 2) == 0 ? sb.x : (p >> 2) == 1 ? sb.y : (p >> 2) == 2 ? sb.z : sb.w;
+  return s_tab[__byte_perm(w, 0, 0x4440 + (p & 3))];
+}
 
 // A team of TEAM threads (32: one warp, 128: the CTA) owning one slab at a time.
 template <int TEAM>
@@ -146,11 +168,6 @@ __device__ __forceinline__ void chunk_codes(const float (&v)[kCK], const float (
   }
 }
 
-// Loads the pair sign masks of one row into shared memory (all threads).
-__device__ __forceinline__ void load_sign_masks(const int8_t* signs, int dim, uint32_t* s_msk) {
-  for (int p = threadIdx.x; p < dim / 2; p += kCT) s_msk[mask_slot(p)] = pair_sign_mask(signs[2 * p], signs[2 * p + 1]);
-}
-
 // Forward: bf16 -> signs -> H_B (B = 2^LOG_B, 8..128) -> group max -> codes.
 // WIDE_G: the scale group covers whole chunks (G >= 128); otherwise 8 <= G < 128.
 // TEAM: 32 (warp teams; groups of at most 32 chunks, gpc dividing 32) or 128.
@@ -160,13 +177,15 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* s_gmax = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes());  // [2][kCT], CTA teams
-  uint32_t* s_msk = s_gmax + 2 * kCT;
+  uint4* s_tab = reinterpret_cast<uint4*>(smem + 2 * chunk_stage_bytes());
+  uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes() + kSignTabBytes);
+  uint32_t* s_gmax = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes() +
+                                                 (SIGNS ? kSignTabBytes + sign_bits_bytes(a.dim) : 0));  // [2][kCT], CTA teams
   const int tt = T::tid();
   const int G = a.G;
   const bool multi = WIDE_G && G > kCK;  // groups spanning several chunks
 
-  if constexpr (SIGNS) load_sign_masks(a.signs, a.dim, s_msk);
+  if constexpr (SIGNS) load_sign_tables(a.signs, a.dim, s_tab, s_bits);
   if constexpr (TEAM == kCT) {
     for (int i = threadIdx.x; i < 2 * kCT; i += kCT) s_gmax[i] = 0u;
   }
@@ -213,12 +232,14 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
     float v[kCK];
     float pm[16];
     if (active) {
+      uint4 sb = make_uint4(0, 0, 0, 0);
+      if constexpr (SIGNS) sb = *reinterpret_cast<const uint4*>(s_bits + col0 / 32);
 #pragma unroll
       for (int p = 0; p < 16; ++p) {
         const uint4 r = *reinterpret_cast<const uint4*>(mine + 16 * p);
         uint32_t w[4] = {r.x, r.y, r.z, r.w};
         if constexpr (SIGNS) {
-          const uint4 m4 = *reinterpret_cast<const uint4*>(s_msk + mask_slot(col0 / 2 + 4 * p));
+          const uint4 m4 = sign_masks8(s_tab, sb, p);
           w[0] ^= m4.x;
           w[1] ^= m4.y;
           w[2] ^= m4.z;
@@ -334,13 +355,14 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
   using T = Team<32>;
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* s_msk = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes()) + 2 * kCT;
+  uint4* s_tab = reinterpret_cast<uint4*>(smem + 2 * chunk_stage_bytes());
+  uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes() + kSignTabBytes);
   const int tt = T::tid();
   const int G = a.G;
   const bool one_scale = G >= kCK;
 
   if constexpr (SIGNS) {
-    load_sign_masks(a.signs, a.dim, s_msk);
+    load_sign_tables(a.signs, a.dim, s_tab, s_bits);
     __syncthreads();
   }
   const int64_t nslabs = (a.nchunks + a.slab_chunks - 1) / a.slab_chunks;
@@ -451,18 +473,22 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
           }
         }
       }
+      uint4 sb = make_uint4(0, 0, 0, 0);
+      if constexpr (SIGNS) sb = *reinterpret_cast<const uint4*>(s_bits + col0 / 32);
       if constexpr (OUT_F32) {
         float* dst = a.rot + ch * kCK;
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
           uint32_t o[8];
+          uint4 m4 = make_uint4(0, 0, 0, 0);
+          if constexpr (SIGNS) m4 = sign_masks8(s_tab, sb, p);
+          const uint32_t mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t lo = __float_as_uint(v[8 * p + 2 * i]), hi = __float_as_uint(v[8 * p + 2 * i + 1]);
             if constexpr (SIGNS) {
-              const uint32_t m = s_msk[mask_slot(col0 / 2 + 4 * p + i)];
-              lo ^= m << 16;
-              hi ^= m & 0x80000000u;
+              lo ^= mm[i] << 16;
+              hi ^= mm[i] & 0x80000000u;
             }
             o[2 * i] = lo;
             o[2 * i + 1] = hi;
@@ -481,7 +507,7 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
             o[i] = r;
           }
           if constexpr (SIGNS) {
-            const uint4 m4 = *reinterpret_cast<const uint4*>(s_msk + mask_slot(col0 / 2 + 4 * p));
+            const uint4 m4 = sign_masks8(s_tab, sb, p);
             o[0] ^= m4.x;
             o[1] ^= m4.y;
             o[2] ^= m4.z;
@@ -495,6 +521,141 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
       T::sync();
       chunk_store<16, 32>(cur, nch, reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256, tt);
     }
+  }
+  cp_async_wait<0>();
+}
+
+// Forward for 4096-column Hadamard blocks, one block per warp (one scale per
+// block, G = 4096).  Lane c first owns chunk c (block columns 128c..128c+127)
+// and runs index bits 0..6 in registers, exactly as in rq_chunk_kernel.  Index
+// bits 7..11 are the lane number, so the warp then transposes its block
+// through its own shared-memory slots, in two halves of 64 columns per chunk
+// so that it fits in the slab's 32 x 272-byte slots.  Afterwards lane t holds
+// columns 64h + 2t + j of every chunk c in register 4c + 2h + j: bits 7..11
+// are register bits 2..6, run as five more paired-FP32 stages.  Codes are
+// written back into the slots in natural order and leave with the usual
+// coalesced copy-out.
+template <int BITS, bool SIGNS>
+__global__ void __launch_bounds__(kCT, 3) rq_wide4096_kernel(ChunkArgs a) {
+  using T = Team<32>;
+  constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
+  constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint4* s_tab = reinterpret_cast<uint4*>(smem + 2 * chunk_stage_bytes());
+  uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + 2 * chunk_stage_bytes() + kSignTabBytes);
+  const int tt = T::tid();
+
+  if constexpr (SIGNS) {
+    load_sign_tables(a.signs, a.dim, s_tab, s_bits);
+    __syncthreads();
+  }
+  const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
+  const int64_t nslabs = a.nchunks / 32;  // one 4096-column block per slab
+  int colc = SIGNS ? (int)((T::first() * 32 + tt) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)((T::stride() * 32) % a.cpr) : 0;
+  uint8_t* st0 = T::stage(smem, 0);
+  uint8_t* st1 = T::stage(smem, 1);
+
+  int64_t slab = T::first();
+  if (slab < nslabs) chunk_load<16, 32>(xsrc + slab * 32 * 256, 32, st0, tt);
+  cp_async_commit();
+  for (int it = 0; slab < nslabs; ++it, slab += T::stride()) {
+    uint8_t* cur = (it & 1) ? st1 : st0;
+    const int64_t c0 = slab * 32;
+    cp_async_wait<0>();
+    T::sync();
+    {
+      const int64_t nx = slab + T::stride();
+      if (nx < nslabs) chunk_load<16, 32>(xsrc + nx * 32 * 256, 32, (it & 1) ? st0 : st1, tt);
+      cp_async_commit();
+    }
+    const int col0 = colc * kCK;
+    if constexpr (SIGNS) {
+      colc += col_step;
+      if (colc >= a.cpr) colc -= a.cpr;
+    }
+    uint8_t* mine = cur + tt * kCPad;
+
+    float v[kCK];
+    uint4 sb = make_uint4(0, 0, 0, 0);
+    if constexpr (SIGNS) sb = *reinterpret_cast<const uint4*>(s_bits + col0 / 32);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const uint4 r = *reinterpret_cast<const uint4*>(mine + 16 * p);
+      uint32_t w[4] = {r.x, r.y, r.z, r.w};
+      if constexpr (SIGNS) {
+        const uint4 m4 = sign_masks8(s_tab, sb, p);
+        w[0] ^= m4.x;
+        w[1] ^= m4.y;
+        w[2] ^= m4.z;
+        w[3] ^= m4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bf16_pair_stage1(w[i], v[8 * p + 2 * i], v[8 * p + 2 * i + 1]);
+    }
+    reg_fwht_from<kCK, 1, 7>(v);  // index bits 0..6
+
+    // transpose inside the warp, one 64-column half of every chunk at a time
+    float u[kCK];
+    float* slotf = reinterpret_cast<float*>(cur);  // slot c = 68 floats
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      __syncwarp();  // the slots are free (input read / previous half read)
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        *reinterpret_cast<float4*>(slotf + tt * 68 + 4 * q) =
+            make_float4(v[64 * h + 4 * q], v[64 * h + 4 * q + 1], v[64 * h + 4 * q + 2], v[64 * h + 4 * q + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float2 f = *reinterpret_cast<const float2*>(slotf + c * 68 + 2 * tt);
+        u[4 * c + 2 * h] = f.x;
+        u[4 * c + 2 * h + 1] = f.y;
+      }
+    }
+    // index bits 7..11 = register bits 2..6
+    reg_stage<kCK, 4>(u);
+    reg_stage<kCK, 8>(u);
+    reg_stage<kCK, 16>(u);
+    reg_stage<kCK, 32>(u);
+    reg_stage<kCK, 64>(u);
+
+    float m = fmaxf(fabsf(u[0]), fabsf(u[1]));
+#pragma unroll
+    for (int i = 2; i < kCK; ++i) m = fmaxf(m, fabsf(u[i]));
+#pragma unroll
+    for (int b = 1; b < 32; b <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, b));
+    if (tt == 0) a.scales[slab] = m * a.scale_mul;
+    if (a.rot) {
+      float* rr = a.rot + c0 * kCK + 2 * tt;
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          *reinterpret_cast<float2*>(rr + c * kCK + 64 * h) =
+              make_float2(u[4 * c + 2 * h] * a.rsqrt_b, u[4 * c + 2 * h + 1] * a.rsqrt_b);
+    }
+    const QInv q = make_qinv(m, QMAX);
+    if (q.tiny) {
+#pragma unroll
+      for (int i = 0; i < kCK; ++i) u[i] *= 18446744073709551616.0f;
+    }
+    __syncwarp();  // every lane has read the second half
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t c0w, c1w;
+        magic_code2(u[4 * c + 2 * h], u[4 * c + 2 * h + 1], q.inv, c0w, c1w);
+        if constexpr (BITS == 8) {  // columns 64h + 2t, 64h + 2t + 1 -> bytes
+          *reinterpret_cast<uint16_t*>(cur + c * kCPad + 64 * h + 2 * tt) = (uint16_t)__byte_perm(c0w, c1w, 0x0040);
+        } else {                    // -> one byte, even column in the low nibble
+          cur[c * kCPad + 32 * h + tt] = (uint8_t)((c0w & 0xfu) | ((c1w & 0xfu) << 4));
+        }
+      }
+    }
+    T::sync();
+    chunk_store<CB / 16, 32>(cur, 32, a.codes + c0 * CB, tt);
   }
   cp_async_wait<0>();
 }

@@ -26,6 +26,11 @@ const void* chunk_fn_g(int B, bool wide_g, int team) {
 
 }  // namespace
 
+const void* wide4096_kernel_ptr(int bits, bool signs) {
+  if (bits == 8) return signs ? (const void*)rq_wide4096_kernel<8, true> : (const void*)rq_wide4096_kernel<8, false>;
+  return signs ? (const void*)rq_wide4096_kernel<4, true> : (const void*)rq_wide4096_kernel<4, false>;
+}
+
 const void* chunk_kernel_ptr(int bits, int B, bool signs, bool wide_g, int team) {
   return bits == 8 ? (signs ? chunk_fn_g<8, true>(B, wide_g, team) : chunk_fn_g<8, false>(B, wide_g, team))
                    : (signs ? chunk_fn_g<4, true>(B, wide_g, team) : chunk_fn_g<4, false>(B, wide_g, team));

@@ -70,8 +70,10 @@ typedef enum {
   HADQ_PATH_BLOCKED = 1,   /* register butterflies, blocks of 8..256        */
   HADQ_PATH_FULL4096 = 2,  /* one 4096-point block per row, smem transposes */
   HADQ_PATH_GENERIC = 3,   /* shared-memory kernel, any valid combination   */
-  HADQ_PATH_CHUNK = 4      /* one 128-column chunk per thread, blocks <= 128,
+  HADQ_PATH_CHUNK = 4,     /* one 128-column chunk per thread, blocks <= 128,
                               slabs staged through shared memory            */
+  HADQ_PATH_WIDE4096 = 5   /* 4096-column blocks with one scale per block:
+                              one block per warp, in-warp transpose         */
 } hadq_path;
 
 enum { HADQ_MAX_DIM = 32768 };

@@ -92,7 +92,10 @@ CASES = [
     (6, 8192, 256, 1024, 8, True, "blocked"),
     (129, 64, 64, 32, 4, False, "blocked"),         # dim not a multiple of 128
     (61, 96, 32, 8, 8, True, "blocked"),
-    (21, 4096, -1, -1, 4, True, "full4096"),        # full 4096 + signs, per token
+    (21, 4096, -1, -1, 4, True, "wide4096"),        # full 4096 + signs, per token
+    (22, 4096, -1, -1, 8, False, "wide4096"),
+    (5, 8192, 4096, 4096, 8, True, "wide4096"),     # two 4096-blocks per row, scale per block
+    (3, 12288, 4096, 4096, 4, False, "wide4096"),
     (19, 4096, -1, 128, 8, False, "full4096"),
     (7, 4096, 4096, 64, 4, True, "full4096"),
     (11, 4096, -1, 1024, 8, True, "full4096"),
