@@ -234,8 +234,8 @@ class L2Flush:
     def __init__(self, device):
         import torch
         self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
-        self.sink = torch.zeros((), dtype=torch.int64, device=device)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.sink = torch.zeros((), dtype=torch.float32, device=device)
 
     def __call__(self):
         self.w.fill_(1)

@@ -248,13 +248,21 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) bf16_pair_stage1(w[i], v[8 * p + 2 * i], v[8 * p + 2 * i + 1]);
       }
-      reg_fwht_from<kCK, 1, LOG_B>(v);
+      if constexpr (WIDE_G) {
+        // one group covers the chunk: fuse the maximum into the last stage
+        reg_fwht_from<kCK, 1, LOG_B - 1>(v);
+        pm[0] = reg_stage_absmax<kCK, (1 << (LOG_B - 1))>(v);
 #pragma unroll
-      for (int p = 0; p < 16; ++p) {
-        float m = fmaxf(fabsf(v[8 * p]), fabsf(v[8 * p + 1]));
+        for (int p = 1; p < 16; ++p) pm[p] = pm[0];
+      } else {
+        reg_fwht_from<kCK, 1, LOG_B>(v);
 #pragma unroll
-        for (int k = 2; k < 8; ++k) m = fmaxf(m, fabsf(v[8 * p + k]));
-        pm[p] = m;
+        for (int p = 0; p < 16; ++p) {
+          float m = fmaxf(fabsf(v[8 * p]), fabsf(v[8 * p + 1]));
+#pragma unroll
+          for (int k = 2; k < 8; ++k) m = fmaxf(m, fabsf(v[8 * p + k]));
+          pm[p] = m;
+        }
       }
     } else {
 #pragma unroll
@@ -264,8 +272,6 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
     float gmax = 0.0f;  // WIDE_G: maximum of the whole group
     if constexpr (WIDE_G) {
       gmax = pm[0];
-#pragma unroll
-      for (int p = 1; p < 16; ++p) gmax = fmaxf(gmax, pm[p]);
       if constexpr (TEAM == 32) {
         // groups of gpc consecutive lanes (gpc divides 32): butterfly max
         for (int b = 1; b < a.gpc; b <<= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, b));
@@ -530,9 +536,10 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
 // and runs index bits 0..6 in registers, exactly as in rq_chunk_kernel.  Index
 // bits 7..11 are the lane number, so the warp then transposes its block
 // through its own shared-memory slots, in two halves of 64 columns per chunk
-// so that it fits in the slab's 32 x 272-byte slots.  Afterwards lane t holds
-// columns 64h + 2t + j of every chunk c in register 4c + 2h + j: bits 7..11
-// are register bits 2..6, run as five more paired-FP32 stages.  Codes are
+// (column bit 1 clear, then set) so that it fits in the slab's 32 x 272-byte
+// slots.
+// Afterwards lane t holds columns 4t + j of every chunk c in register 4c + j:
+// bits 7..11 are register bits 2..6, run as five more paired-FP32 stages.  Codes are
 // written back into the slots in natural order and leave with the usual
 // coalesced copy-out.
 template <int BITS, bool SIGNS>
@@ -595,7 +602,10 @@ __global__ void __launch_bounds__(kCT, 3) rq_wide4096_kernel(ChunkArgs a) {
     }
     reg_fwht_from<kCK, 1, 7>(v);  // index bits 0..6
 
-    // transpose inside the warp, one 64-column half of every chunk at a time
+    // transpose inside the warp: first the columns with bit 1 clear, then those
+    // with bit 1 set (64 per chunk, whole register pairs so that the written
+    // half frees its registers); afterwards register 4c + j of lane t holds
+    // column 4t + j of chunk c
     float u[kCK];
     float* slotf = reinterpret_cast<float*>(cur);  // slot c = 68 floats
 #pragma unroll
@@ -604,11 +614,11 @@ __global__ void __launch_bounds__(kCT, 3) rq_wide4096_kernel(ChunkArgs a) {
 #pragma unroll
       for (int q = 0; q < 16; ++q)
         *reinterpret_cast<float4*>(slotf + tt * 68 + 4 * q) =
-            make_float4(v[64 * h + 4 * q], v[64 * h + 4 * q + 1], v[64 * h + 4 * q + 2], v[64 * h + 4 * q + 3]);
+            make_float4(v[8 * q + 2 * h], v[8 * q + 2 * h + 1], v[8 * q + 4 + 2 * h], v[8 * q + 5 + 2 * h]);
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float2 f = *reinterpret_cast<const float2*>(slotf + c * 68 + 2 * tt);
+        const float2 f = *reinterpret_cast<const float2*>(slotf + c * 68 + 2 * tt);  // columns 4t + 2h, + 1
         u[4 * c + 2 * h] = f.x;
         u[4 * c + 2 * h + 1] = f.y;
       }
@@ -618,22 +628,16 @@ __global__ void __launch_bounds__(kCT, 3) rq_wide4096_kernel(ChunkArgs a) {
     reg_stage<kCK, 8>(u);
     reg_stage<kCK, 16>(u);
     reg_stage<kCK, 32>(u);
-    reg_stage<kCK, 64>(u);
-
-    float m = fmaxf(fabsf(u[0]), fabsf(u[1]));
-#pragma unroll
-    for (int i = 2; i < kCK; ++i) m = fmaxf(m, fabsf(u[i]));
+    float m = reg_stage_absmax<kCK, 64>(u);
 #pragma unroll
     for (int b = 1; b < 32; b <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, b));
     if (tt == 0) a.scales[slab] = m * a.scale_mul;
     if (a.rot) {
-      float* rr = a.rot + c0 * kCK + 2 * tt;
+      float* rr = a.rot + c0 * kCK + 4 * tt;
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          *reinterpret_cast<float2*>(rr + c * kCK + 64 * h) =
-              make_float2(u[4 * c + 2 * h] * a.rsqrt_b, u[4 * c + 2 * h + 1] * a.rsqrt_b);
+        *reinterpret_cast<float4*>(rr + c * kCK) =
+            make_float4(u[4 * c] * a.rsqrt_b, u[4 * c + 1] * a.rsqrt_b, u[4 * c + 2] * a.rsqrt_b, u[4 * c + 3] * a.rsqrt_b);
     }
     const QInv q = make_qinv(m, QMAX);
     if (q.tiny) {
@@ -643,15 +647,16 @@ __global__ void __launch_bounds__(kCT, 3) rq_wide4096_kernel(ChunkArgs a) {
     __syncwarp();  // every lane has read the second half
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t c0w, c1w;
-        magic_code2(u[4 * c + 2 * h], u[4 * c + 2 * h + 1], q.inv, c0w, c1w);
-        if constexpr (BITS == 8) {  // columns 64h + 2t, 64h + 2t + 1 -> bytes
-          *reinterpret_cast<uint16_t*>(cur + c * kCPad + 64 * h + 2 * tt) = (uint16_t)__byte_perm(c0w, c1w, 0x0040);
-        } else {                    // -> one byte, even column in the low nibble
-          cur[c * kCPad + 32 * h + tt] = (uint8_t)((c0w & 0xfu) | ((c1w & 0xfu) << 4));
-        }
+      uint32_t cc[4];
+      magic_code2(u[4 * c], u[4 * c + 1], q.inv, cc[0], cc[1]);
+      magic_code2(u[4 * c + 2], u[4 * c + 3], q.inv, cc[2], cc[3]);
+      const uint32_t b4 = pack_i8x4(cc[0], cc[1], cc[2], cc[3]);  // columns 4t .. 4t + 3
+      if constexpr (BITS == 8) {
+        *reinterpret_cast<uint32_t*>(cur + c * kCPad + 4 * tt) = b4;
+      } else {
+        const uint32_t e = __byte_perm(b4, 0, 0x0020);  // columns 4t, 4t + 2
+        const uint32_t o = __byte_perm(b4, 0, 0x0031);  // columns 4t + 1, 4t + 3
+        *reinterpret_cast<uint16_t*>(cur + c * kCPad + 2 * tt) = (uint16_t)((e & 0x0f0fu) | ((o << 4) & 0xf0f0u));
       }
     }
     T::sync();

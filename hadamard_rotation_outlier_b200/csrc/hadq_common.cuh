@@ -119,6 +119,33 @@ __device__ __forceinline__ void reg_fwht(float (&v)[N]) {
   if constexpr (LOG_N >= 7) reg_stage<N, 64>(v);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// The last butterfly stage (stride H, paired FP32) fused with the maximum of
+// |y| over its outputs: max(|a + b|, |a - b|) = |a| + |b|, and the rounded
+// value of whichever of a + b, a - b has that magnitude equals the rounded
+// |a| + |b|, so the maximum is exact.  Returns the maximum over all N outputs.
+template <int N, int H>
+__device__ __forceinline__ float reg_stage_absmax(float (&v)[N]) {
+  static_assert(H >= 2, "paired stage");
+  float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < N; i += 2 * H) {
+#pragma unroll
+    for (int t = 0; t < H; t += 2) {
+      const float s0 = fabsf(v[i + t]) + fabsf(v[i + t + H]);
+      const float s1 = fabsf(v[i + t + 1]) + fabsf(v[i + t + H + 1]);
+      if (((i + t) / 2) & 1) m1 = max3(m1, s0, s1); else m0 = max3(m0, s0, s1);
+      bfly2(v[i + t], v[i + t + 1], v[i + t + H], v[i + t + H + 1]);
+    }
+  }
+  return fmaxf(m0, m1);
+}
+
 // Butterfly stage across lanes: partner = lane ^ m.  The lane whose bit is set
 // keeps (partner - own), the other keeps (own + partner).
 template <int N>
