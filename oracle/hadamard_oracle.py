@@ -52,6 +52,8 @@ __all__ = [
     "dequant_rotate_inv",
     "quant_error",
     "half_boundary_distance",
+    "dequant_rotated",
+    "kv_decode_attention",
 ]
 
 
@@ -274,6 +276,64 @@ def dequant_rotate_inv(codes: np.ndarray, scales: np.ndarray, dim: int, block: i
     s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
     yhat = (q.reshape(q.shape[0], dim // G, G) * s[..., None]).reshape(q.shape)
     return inverse_rotate(yhat, block=block, signs=signs, method=method)
+
+
+def dequant_rotated(codes: np.ndarray, scales: np.ndarray, dim: int, bits: int = 4,
+                    group: int = -1) -> np.ndarray:
+    """q * scale, left in the rotated basis (no inverse rotation), float64 [..., dim].
+
+    The dequantisation of [Outlier nemesis] §2.2 (``x_q * scale``) applied to
+    stored codes; [QuaRot hands-on] §2.2 reads the 4-bit KV cache this way.
+    """
+    q = np.asarray(codes).astype(np.int64) if bits == 8 else unpack_int4(codes)
+    lead = q.shape[:-1]
+    G = _group_size(dim, group)
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(lead + (dim // G,))
+    return (q.reshape(lead + (dim // G, G)) * s[..., None]).reshape(lead + (dim,))
+
+
+def kv_decode_attention(q_bits: np.ndarray, k_codes: np.ndarray, k_scales: np.ndarray,
+                        v_codes: np.ndarray, v_scales: np.ndarray, dim: int, block: int = -1,
+                        signs=None, bits: int = 4, group: int = -1,
+                        softmax_scale: float | None = None) -> np.ndarray:
+    """Decode attention of one new query token per head over a quantised,
+    rotated KV cache, float64.
+
+    * [QuaRot hands-on] §2.2: K and V are rotated online and stored in 4 bits,
+      then dequantised when they are read for attention.
+    * [Hartmann rotation] §1: Q_rot K_rot^T = Q K^T, so the scores come from
+      the rotated query against the rotated keys, without undoing the
+      rotation of K.
+    * P V_rot = (P V) H: the output is computed in the rotated basis and
+      transformed back once ([QuaRot hands-on] §2.3), with H and the signs
+      of :func:`inverse_rotate`.
+
+    Shapes: ``q_bits`` bf16 bits [batch, n_q_heads, dim]; codes [batch,
+    n_kv_heads, tokens, dim] (INT8) or [..., dim/2] (INT4); scales [batch,
+    n_kv_heads, tokens, dim/G].  Query head h reads KV head h // (n_q_heads /
+    n_kv_heads).  Returns float64 [batch, n_q_heads, dim].
+    """
+    q = bf16_bits_to_f64(q_bits)
+    nb, nqh, d = q.shape
+    assert d == dim
+    kr = dequant_rotated(k_codes, k_scales, dim, bits, group)   # [b, hk, T, d]
+    vr = dequant_rotated(v_codes, v_scales, dim, bits, group)
+    nkh = kr.shape[1]
+    if nqh % nkh:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    g = nqh // nkh
+    if softmax_scale is None:
+        softmax_scale = 1.0 / np.sqrt(dim)
+    qr = rotate(q, block=block, signs=signs)
+    out = np.empty((nb, nqh, dim))
+    for b in range(nb):
+        for h in range(nqh):
+            kv = h // g
+            s = softmax_scale * (kr[b, kv] @ qr[b, h])
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            out[b, h] = p @ vr[b, kv]
+    return inverse_rotate(out, block=block, signs=signs)
 
 
 def quant_error(x: np.ndarray, bits: int = 4) -> float:

@@ -11,6 +11,7 @@ import math
 import numpy as np
 import pytest
 import scipy.linalg
+import scipy.special
 
 import oracle as O
 from hadamard_rotation_outlier_b200 import synthetic as S
@@ -359,3 +360,107 @@ def test_planted_mistakes_are_caught(golden_hand):
         return x @ (O.sylvester(4) * 2)
 
     assert not np.allclose(unnormalised(np.array([g["ex1_x"]]))[0], g["ex1_y"])
+
+
+# ------------------------------------------------- decode attention over the KV cache
+
+def _random_kv_codes(rng, nb, nkh, T, dim, bits, G):
+    qmax = 2 ** (bits - 1) - 1
+    q = rng.integers(-qmax, qmax + 1, size=(nb, nkh, T, dim))
+    codes = q.astype(np.int8) if bits == 8 else O.pack_int4(q)
+    scales = rng.uniform(0.01, 0.2, size=(nb, nkh, T, dim // G)).astype(np.float32)
+    return q, codes, scales
+
+
+def _scipy_unrotate(yrot, dim, B, signs):
+    # x = (y @ H_B) * s with H_B from scipy's Sylvester construction.
+    H = scipy.linalg.hadamard(B).astype(np.float64) / math.sqrt(B)
+    x = (yrot.reshape(yrot.shape[:-1] + (dim // B, B)) @ H).reshape(yrot.shape)
+    if signs is not None:
+        x = x * np.where(np.asarray(signs) < 0, -1.0, 1.0)
+    return x
+
+
+@pytest.mark.parametrize("bits,G,B,with_signs", [(4, 128, 128, False), (8, 64, 128, True),
+                                                 (4, 32, 64, True), (4, 128, -1, False)])
+def test_decode_attention_matches_unrotated_attention(bits, G, B, with_signs):
+    # Q_rot K_rot^T = Q K^T: the oracle's rotated-basis attention must equal
+    # textbook attention on the un-rotated K, V (undone with scipy's H) and the
+    # raw query, with scipy's softmax.  Consecutive query heads share a KV head.
+    rng = np.random.default_rng(11 + bits + G)
+    nb, nqh, nkh, T, dim = 2, 4, 2, 37, 128
+    Bn = dim if B == -1 else B
+    signs = S.random_signs(dim, 5) if with_signs else None
+    qk, kc, ks = _random_kv_codes(rng, nb, nkh, T, dim, bits, G)
+    qv, vc, vs = _random_kv_codes(rng, nb, nkh, T, dim, bits, G)
+    qbits = S.f32_to_bf16_bits(rng.normal(size=(nb, nqh, dim)).astype(np.float32))
+    got = O.kv_decode_attention(qbits, kc, ks, vc, vs, dim, B, signs, bits, G)
+
+    def deq(qcodes, sc):
+        return (qcodes.reshape(nb, nkh, T, dim // G, G) * sc.astype(np.float64)[..., None]
+                ).reshape(nb, nkh, T, dim)
+
+    K = _scipy_unrotate(deq(qk, ks), dim, Bn, signs)
+    V = _scipy_unrotate(deq(qv, vs), dim, Bn, signs)
+    x = O.bf16_bits_to_f64(qbits)
+    want = np.empty((nb, nqh, dim))
+    for b in range(nb):
+        for h in range(nqh):
+            kvh = h // (nqh // nkh)
+            p = scipy.special.softmax(K[b, kvh] @ x[b, h] / math.sqrt(dim))
+            want[b, h] = p @ V[b, kvh]
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_decode_attention_single_token_returns_its_value_row():
+    # One cached token: softmax weight 1, output = that V row un-rotated.
+    rng = np.random.default_rng(3)
+    dim = 128
+    qv, vc, vs = _random_kv_codes(rng, 1, 1, 1, dim, 4, 128)
+    _, kc, ks = _random_kv_codes(rng, 1, 1, 1, dim, 4, 128)
+    qbits = S.f32_to_bf16_bits(rng.normal(size=(1, 3, dim)).astype(np.float32))
+    got = O.kv_decode_attention(qbits, kc, ks, vc, vs, dim, 128, None, 4, 128)
+    row = _scipy_unrotate(qv[0, 0, 0] * np.float64(vs[0, 0, 0, 0]), dim, 128, None)
+    for h in range(3):
+        np.testing.assert_allclose(got[0, h], row, rtol=0, atol=1e-13)
+
+
+def test_decode_attention_zero_query_averages_values():
+    # q = 0: every score is 0, the weights are uniform, output = mean of V.
+    rng = np.random.default_rng(4)
+    dim, T = 64, 9
+    qv, vc, vs = _random_kv_codes(rng, 1, 1, T, dim, 8, 32)
+    _, kc, ks = _random_kv_codes(rng, 1, 1, T, dim, 8, 32)
+    qbits = np.zeros((1, 1, dim), np.uint16)
+    got = O.kv_decode_attention(qbits, kc, ks, vc, vs, dim, -1, None, 8, 32)
+    deq = (qv.reshape(T, 2, 32) * vs.reshape(T, 2, 1).astype(np.float64)).reshape(T, dim)
+    want = _scipy_unrotate(deq.mean(axis=0), dim, dim, None)
+    np.testing.assert_allclose(got[0, 0], want, rtol=0, atol=1e-13)
+
+
+def test_decode_attention_dominant_key_selects_its_value():
+    # One key aligned with the (rotated) query and far larger than the rest:
+    # its weight is 1 to within exp(-huge), so the output is its V row.
+    dim, T, hot = 128, 16, 11
+    H = scipy.linalg.hadamard(dim).astype(np.float64) / math.sqrt(dim)
+    x = np.zeros(dim)
+    x[0] = 1.0                              # rotated query = H[0] = all +1/sqrt(128)
+    qk = np.zeros((1, 1, T, dim), np.int64)
+    qk[0, 0, hot] = 7
+    ks = np.full((1, 1, T, 1), 1.0, np.float32)
+    qv = np.tile(np.arange(T)[:, None] % 15 - 7, (1, dim))[None, None]
+    vs = np.full((1, 1, T, 1), 0.5, np.float32)
+    qbits = S.f32_to_bf16_bits(x.astype(np.float32)[None, None])
+    got = O.kv_decode_attention(qbits, O.pack_int4(qk), ks, O.pack_int4(qv), vs, dim, -1, None, 4,
+                                -1, softmax_scale=1.0)
+    want = (H @ (qv[0, 0, hot] * 0.5))       # inverse rotation of the hot V row
+    np.testing.assert_allclose(got[0, 0], want, rtol=0, atol=1e-12)
+    assert abs(got[0, 0].sum() - want.sum()) < 1e-12
+
+
+def test_decode_attention_rejects_bad_head_ratio():
+    rng = np.random.default_rng(5)
+    _, kc, ks = _random_kv_codes(rng, 1, 2, 3, 64, 8, 64)
+    qbits = np.zeros((1, 3, 64), np.uint16)
+    with pytest.raises(ValueError):
+        O.kv_decode_attention(qbits, kc, ks, kc, ks, 64, -1, None, 8, 64)
