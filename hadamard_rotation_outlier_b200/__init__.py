@@ -15,6 +15,8 @@ from .binding import (  # noqa: F401
     MAX_DIM,
     HadqError,
     hadq_dequant_rotate_inv,
+    hadq_kv_decode_attention,
+    hadq_kv_decode_workspace_size,
     hadq_last_error,
     hadq_launch_count,
     hadq_plan,

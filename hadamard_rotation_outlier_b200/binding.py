@@ -22,8 +22,9 @@ HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
 PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
 MAX_DIM = 32768
 
-EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_plan", "hadq_status_str",
-            "hadq_last_error", "hadq_launch_count", "hadq_version")
+EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_kv_decode_attention",
+            "hadq_kv_decode_workspace_size", "hadq_plan", "hadq_status_str", "hadq_last_error",
+            "hadq_launch_count", "hadq_version")
 
 
 class HadqError(RuntimeError):
@@ -52,6 +53,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_dequant_rotate_inv.argtypes = [vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
                                             ctypes.c_int, vp]
     lib.hadq_dequant_rotate_inv.restype = ctypes.c_int
+    lib.hadq_kv_decode_attention.argtypes = [vp, vp, vp, vp, vp, c_i32, c_i32, c_i32, c_i64, c_i64,
+                                             c_i32, c_i32, vp, c_i32, c_i32, ctypes.c_float, vp,
+                                             ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.hadq_kv_decode_attention.restype = ctypes.c_int
+    lib.hadq_kv_decode_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i64,
+                                                  ctypes.POINTER(ctypes.c_size_t)]
+    lib.hadq_kv_decode_workspace_size.restype = ctypes.c_int
     lib.hadq_plan.argtypes = [c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
                               ctypes.POINTER(ctypes.c_int)]
     lib.hadq_plan.restype = ctypes.c_int
@@ -196,4 +204,72 @@ def hadq_dequant_rotate_inv(codes: torch.Tensor, scales: torch.Tensor, dim: int,
     code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
     _check(lib.hadq_dequant_rotate_inv(_ptr(codes), _ptr(scales), rows, dim, block, _ptr(signs), bits,
                                        group, _ptr(out), code, _stream(stream)))
+    return out
+
+
+def hadq_kv_decode_workspace_size(batch: int, n_q_heads: int, n_kv_heads: int, tokens: int) -> int:
+    """Host-only: workspace bytes :func:`hadq_kv_decode_attention` needs (any GPU)."""
+    n = ctypes.c_size_t(0)
+    _check(load_library().hadq_kv_decode_workspace_size(batch, n_q_heads, n_kv_heads, tokens,
+                                                        ctypes.byref(n)))
+    return int(n.value)
+
+
+def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: torch.Tensor,
+                             v_codes: torch.Tensor, v_scales: torch.Tensor, tokens: int | None = None,
+                             block: int = -1, signs: torch.Tensor | None = None, bits: int = 4,
+                             group: int = -1, softmax_scale: float | None = None,
+                             out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One decode step of attention over a rotated INT4 KV cache.
+
+    ``q``: bf16 ``[batch, n_q_heads, dim]``.  ``k_codes``/``v_codes``: uint8
+    ``[batch, n_kv_heads, token_stride, dim/2]``; ``k_scales``/``v_scales``:
+    float32 ``[batch, n_kv_heads, token_stride]`` (or with a trailing 1).
+    ``tokens`` (default ``token_stride``) rows of each head are attended over.
+    ``workspace``: a zero-filled uint8 CUDA tensor of at least
+    :func:`hadq_kv_decode_workspace_size` bytes, reused across calls (one is
+    allocated when omitted).  Returns ``[batch, n_q_heads, dim]`` bf16 or fp32.
+    """
+    lib = load_library()
+    if q.dtype != torch.bfloat16:
+        raise TypeError(f"q must be bfloat16, got {q.dtype}")
+    if q.dim() != 3 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("q must be a contiguous CUDA tensor [batch, n_q_heads, dim]")
+    batch, nqh, dim = q.shape
+    dev = q.device
+    if k_codes.dim() != 4 or v_codes.shape != k_codes.shape:
+        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim/2] alike")
+    nkv, stride = k_codes.shape[1], k_codes.shape[2]
+    if k_codes.shape[0] != batch:
+        raise ValueError("k_codes batch differs from q")
+    per_row = k_codes.shape[3]
+    if tokens is None:
+        tokens = stride
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, dev)
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float32, dev, batch * nkv * stride)
+    if per_row * 2 != dim:
+        raise ValueError(f"codes rows hold {per_row} bytes, expected dim/2 = {dim // 2}")
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / float(dim) ** 0.5
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        out = torch.empty((batch, nqh, dim), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev, batch * nqh * dim)
+    need = hadq_kv_decode_workspace_size(batch, nqh, nkv, tokens) if batch else 0
+    if workspace is None:
+        workspace = torch.zeros(max(need, 1), dtype=torch.uint8, device=dev)
+    else:
+        _need(workspace, "workspace", torch.uint8, dev)
+    code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_kv_decode_attention(_ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                        _ptr(v_scales), batch, nqh, nkv, tokens, stride, dim, block,
+                                        _ptr(signs), bits, group, float(softmax_scale), _ptr(out), code,
+                                        _ptr(workspace), workspace.numel(), _stream(stream)))
     return out

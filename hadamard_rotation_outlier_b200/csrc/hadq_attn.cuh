@@ -1,0 +1,544 @@
+// Decode attention over the rotated, quantised KV cache.
+//
+// One new query token per head attends over a cache whose K and V rows were
+// rotated by H_128 (after the optional sign flip) and stored as INT4 codes with
+// one float32 scale per row, i.e. the output of the rotate+quantise kernels at
+// dim 128, block 128, group 128.  The maths ("Hartmann rotation, lightweight
+// QAT, streaming attention", section 1; "QuaRot hands-on", sections 2.2-2.3):
+//
+//   q_rot = (q * s) H                     rotate the query like the keys
+//   score_t = softmax_scale * q_rot . (kcode_t * kscale_t)   (= q . k_t)
+//   p = softmax(score)                    over the cached tokens
+//   o_rot = sum_t p_t * vcode_t * vscale_t
+//   o = (o_rot H) * s                     one inverse rotation per output row
+//
+// Work split: a CTA (4 warps) serves one KV head, up to 4 of the query heads
+// that share it, and one contiguous token range (split-K).  Each warp streams
+// 16-token tiles through its own cp.async ring in shared memory and keeps an
+// online softmax (running max m, sum l, output O) in registers.  The CTA
+// merges its warps, writes one partial (m, l, O) per head to the workspace, and
+// the last CTA of a head group merges all partials, applies H and the signs
+// and writes the output.
+//
+// Tensor-core use (mma.sync; the contraction has only 4 query rows per KV
+// head, far below the 64-row minimum of a tcgen05 tile, and its operands are
+// born in registers):
+//  * QK: m16n8k32 s8 x s8 -> s32.  B = key codes as int8 (the nibble shifted
+//    into the high half of a byte, i.e. 16 * code, one shift and one mask per
+//    8 codes).  A = the scaled rotated query as a 24-bit fixed-point number
+//    cut into three signed 8-bit digits (rows = head x digit).  The integer
+//    sums are exact; score = (d0 + 2^8 d1 + 2^16 d2) * 2^-E / 16 * kscale.
+//  * PV: m16n8k16 bf16 x bf16 -> f32.  B = value codes as exact bf16 values
+//    (the nibble placed in a bf16 mantissa, then 136 subtracted).  A = p *
+//    vscale cut into three bf16 parts hi + mid + lo (rows = head x part), which
+//    together carry the full float32 value.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "hadq_common.cuh"
+
+namespace hadq {
+
+constexpr int kAttnDim = 128;
+constexpr int kAttnWarps = 4;
+constexpr int kAttnThreads = 32 * kAttnWarps;
+constexpr int kAttnHeads = 4;                                   // query heads per CTA
+constexpr int kAttnTile = 16;                                   // tokens per tile
+constexpr int kAttnStages = 4;                                  // ring depth per warp
+constexpr int kAttnKRow = 64;                                   // bytes of INT4 codes per token
+constexpr int kAttnVRow = 80;                                   // V row padded in shared memory
+constexpr int kAttnStV = kAttnTile * kAttnKRow;                 // 1024
+constexpr int kAttnStS = kAttnStV + kAttnTile * kAttnVRow;      // 2304: 16 K scales, 16 V scales
+constexpr int kAttnStageBytes = kAttnStS + 2 * kAttnTile * 4;   // 2432
+constexpr int kAttnCombPitch = kAttnDim + 4;                    // floats per head in the CTA merge
+constexpr int kAttnMaxSplits = 256;
+constexpr float kAttnSlack = 8.0f;  // log2 units the running max may trail the true max
+
+struct AttnArgs {
+  const uint16_t* q;         // [batch, nqh, 128] bf16
+  const uint8_t* k_codes;    // [batch, nkv, stride, 64]
+  const float* k_scales;     // [batch, nkv, stride]
+  const uint8_t* v_codes;
+  const float* v_scales;
+  const int8_t* signs;       // [128] or NULL
+  void* out;                 // [batch, nqh, 128] bf16 or f32
+  unsigned* counters;        // [groups]
+  float* part_ml;            // [groups][splits][4][2]  (m, l)
+  float* part_o;             // [groups][splits][4][128] (permuted order, see below)
+  int64_t tokens, stride, chunk;
+  int nqh, nkv, g, hgroups, splits;
+  float qmul;                // softmax_scale * log2(e) / sqrt(128)
+  float inv_sqrt_dim;        // 1 / sqrt(128)
+  int out_f32;
+};
+
+template <int STAGES>
+struct __align__(16) AttnSmem {
+  union {
+    uint8_t stage[kAttnWarps][STAGES][kAttnStageBytes];
+    float comb[kAttnWarps][kAttnHeads][kAttnCombPitch];
+  } u;
+  int8_t qd[4][kAttnHeads][kAttnDim];  // query digits [digit][head][dim]; digit 3 stays 0
+  float qscale[kAttnHeads];
+  float m[kAttnWarps][kAttnHeads];
+  float l[kAttnWarps][kAttnHeads];
+  int last;
+};
+
+__device__ __forceinline__ void mma_s8_16832(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// cp.async of 16 (or 4) bytes to a shared-memory address.  The _zfill forms
+// read nothing when valid == false and fill the destination with zeros (the
+// source must still be a mapped address).
+__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async16_zfill(uint32_t smem, const void* gmem, bool valid) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async4_zfill(uint32_t smem, const void* gmem, bool valid) {
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem), "l"(gmem), "r"(n) : "memory");
+}
+
+// Two INT4 codes (nibbles at bits 0-3 and 16-19 of x) -> bf16x2 holding the
+// codes exactly: the nibble with its sign bit flipped is c + 8; placed in the
+// mantissa of 128.0 it reads 136 + c, and subtracting 136 leaves c.
+__device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t x) {
+  const uint32_t t = (x & 0x000F000Fu) ^ 0x43084308u;
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(0x43084308u));
+  return r;
+}
+
+// bf16x2 of (lo, hi), round to nearest even.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Cut the float pair (x0, x1) into bf16 pairs hi + mid + lo whose sum carries
+// every bit of each float: each part is the bf16 rounding of what the
+// previous parts left, and those remainders are exact float differences.
+__device__ __forceinline__ void split3_bf16(float x0, float x1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+  hi = cvt_bf16x2(x0, x1);
+  const float r0 = x0 - __uint_as_float(hi << 16);
+  const float r1 = x1 - __uint_as_float(hi & 0xffff0000u);
+  mid = cvt_bf16x2(r0, r1);
+  const float s0 = r0 - __uint_as_float(mid << 16);
+  const float s1 = r1 - __uint_as_float(mid & 0xffff0000u);
+  lo = cvt_bf16x2(s0, s1);
+}
+
+// 8 INT4 codes of one word -> the two int8x4 registers of an s8 MMA operand:
+// even elements (low nibbles) and odd elements (high nibbles), each as 16*code.
+__device__ __forceinline__ void int4x8_to_s8x16(uint32_t w, uint32_t& even, uint32_t& odd) {
+  even = (w << 4) & 0xF0F0F0F0u;
+  odd = w & 0xF0F0F0F0u;
+}
+
+// STAGES: depth of each warp's cp.async ring (tiles in flight + 1).
+template <int STAGES>
+__global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const AttnArgs a) {
+  __shared__ AttnSmem<STAGES> sm;
+  const int tid = threadIdx.x;
+  const int w = tid >> 5;
+  const int lane = tid & 31;
+  const int g = lane >> 2;  // MMA row group
+  const int j = lane & 3;   // thread in group
+
+  const int grp = blockIdx.y;
+  const int split = blockIdx.x;
+  const int bidx = grp / (a.nkv * a.hgroups);
+  const int rem = grp - bidx * a.nkv * a.hgroups;
+  const int kvh = rem / a.hgroups;
+  const int hg = rem - kvh * a.hgroups;
+  const int head0 = kvh * a.g + hg * kAttnHeads;  // first query head of this CTA
+  const int hn = min(kAttnHeads, a.g - hg * kAttnHeads);
+  const int64_t row0 = (int64_t(bidx) * a.nkv + kvh) * a.stride;
+
+  // ---- query: rotate, scale, cut into digits (warp w handles head w) ----
+  {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (w < hn) {
+      const uint2 raw =
+          *reinterpret_cast<const uint2*>(a.q + (int64_t(bidx) * a.nqh + head0 + w) * kAttnDim + 4 * lane);
+      x[0] = bf16lo(raw.x);
+      x[1] = bf16hi(raw.x);
+      x[2] = bf16lo(raw.y);
+      x[3] = bf16hi(raw.y);
+      if (a.signs) {
+        const uint32_t sg = *reinterpret_cast<const uint32_t*>(a.signs + 4 * lane);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if ((sg >> (8 * i + 7)) & 1u) x[i] = -x[i];
+      }
+    }
+    // H_128: index bits 0-1 in registers, bits 2-6 on lane bits 0-4.
+    bfly(x[0], x[1]);
+    bfly(x[2], x[3]);
+    bfly(x[0], x[2]);
+    bfly(x[1], x[3]);
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+        x[i] = upper ? o - x[i] : x[i] + o;
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[i] *= a.qmul;
+      amax = fmaxf(amax, fabsf(x[i]));
+    }
+#pragma unroll
+    for (int m = 16; m; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    // amax < 2^E' with E' = biased exponent - 126; the fixed-point value is
+    // x * 2^(22 - E'), so |qf| <= 2^22 and the top digit stays within +-65.
+    // A query below 2^-100 in every scaled entry is taken as zero.
+    const int E = int((__float_as_uint(amax) >> 23) & 0xffu);
+    const bool zero = E < 27;
+    const float up = zero ? 0.f : __uint_as_float(uint32_t(148 - E + 127) << 23);
+    uint32_t d0 = 0, d1 = 0, d2 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int qf = __float2int_rn(x[i] * up);
+      const int e0 = (qf << 24) >> 24;
+      const int r1 = (qf - e0) >> 8;
+      const int e1 = (r1 << 24) >> 24;
+      const int e2 = (r1 - e1) >> 8;
+      d0 |= uint32_t(e0 & 0xff) << (8 * i);
+      d1 |= uint32_t(e1 & 0xff) << (8 * i);
+      d2 |= uint32_t(e2 & 0xff) << (8 * i);
+    }
+    *reinterpret_cast<uint32_t*>(&sm.qd[0][w][4 * lane]) = d0;
+    *reinterpret_cast<uint32_t*>(&sm.qd[1][w][4 * lane]) = d1;
+    *reinterpret_cast<uint32_t*>(&sm.qd[2][w][4 * lane]) = d2;
+    *reinterpret_cast<uint32_t*>(&sm.qd[3][w][4 * lane]) = 0u;
+    // 2^(E' - 22) / 16: undo the fixed point and the 16 * code of the keys.
+    if (lane == 0) sm.qscale[w] = zero ? 0.f : __uint_as_float(uint32_t(E - 25) << 23);
+  }
+  __syncthreads();
+
+  // A operands of the QK product for k-step s: lane (g, j) holds rows g and
+  // g+8 (head g & 3, digits g >> 2 and (g >> 2) + 2) at the dims
+  // 32j + 8s + {0,2,4,6} (a0, a1) and 32j + 8s + {1,3,5,7} (a2, a3), the same
+  // dims the key operand of that lane carries.
+  uint32_t qa[4][4];
+  const int hh = g & 3;
+  {
+    const int dr0 = g >> 2, dr1 = (g >> 2) + 2;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint2 r0 = *reinterpret_cast<const uint2*>(&sm.qd[dr0][hh][32 * j + 8 * s]);
+      const uint2 r1 = *reinterpret_cast<const uint2*>(&sm.qd[dr1][hh][32 * j + 8 * s]);
+      qa[s][0] = __byte_perm(r0.x, r0.y, 0x6420);
+      qa[s][1] = __byte_perm(r1.x, r1.y, 0x6420);
+      qa[s][2] = __byte_perm(r0.x, r0.y, 0x7531);
+      qa[s][3] = __byte_perm(r1.x, r1.y, 0x7531);
+    }
+  }
+  const float qs = sm.qscale[hh];
+  // Digit weights of the two rows this lane holds: rows g (digit g>>2) and
+  // g+8 (digit (g>>2)+2; digit 3 is the zero row).
+  const float wl = g < 4 ? 1.f : 256.f;
+  const float wh = g < 4 ? 65536.f : 0.f;
+
+  // ---- token range of this CTA and the warp's tiles ----
+  const int64_t t_begin = int64_t(split) * a.chunk;
+  const int64_t t_end = min(a.tokens, t_begin + a.chunk);
+  const int ntiles = t_begin < t_end ? int((t_end - t_begin + kAttnTile - 1) / kAttnTile) : 0;
+  const int nw = ntiles > w ? (ntiles - w + kAttnWarps - 1) / kAttnWarps : 0;
+
+  const uint8_t* kc = a.k_codes + row0 * kAttnKRow;
+  const uint8_t* vc = a.v_codes + row0 * kAttnKRow;
+  const float* ksc = a.k_scales + row0;
+  const float* vsc = a.v_scales + row0;
+
+  // Copy pattern of one tile (per array, 16 tokens x 4 chunks of 16 bytes):
+  // lane covers token lane/4 and 8 + lane/4, chunk lane%4; the scale copy
+  // takes one float per lane (K scales in lanes 0-15, V scales in 16-31).
+  const int ctok = lane >> 2, cpart = lane & 3;
+  const uint32_t s_ring = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.u.stage[w][0][0]));
+  const uint32_t d_k = ctok * kAttnKRow + cpart * 16;
+  const uint32_t d_v = kAttnStV + ctok * kAttnVRow + cpart * 16;
+  const uint32_t d_s = kAttnStS + 4 * lane;
+  const int64_t lane_tok = t_begin + int64_t(w) * kAttnTile + ctok;  // token of the first chunk, tile 0
+  const uint8_t* g_k = kc + lane_tok * kAttnKRow + cpart * 16;
+  const uint8_t* g_v = vc + lane_tok * kAttnKRow + cpart * 16;
+  const float* g_s = (lane < 16 ? ksc : vsc) + t_begin + int64_t(w) * kAttnTile + (lane & 15);
+  constexpr int64_t kStepTok = int64_t(kAttnWarps) * kAttnTile;  // tokens between a warp's tiles
+
+  auto issue = [&](int k) {
+    const uint32_t st = s_ring + uint32_t(k % STAGES) * kAttnStageBytes;
+    const int64_t adv = int64_t(k) * kStepTok;
+    const int64_t t0 = t_begin + int64_t(w + kAttnWarps * k) * kAttnTile;
+    if (t0 + kAttnTile <= t_end) {
+      cp_async16(st + d_k, g_k + adv * kAttnKRow);
+      cp_async16(st + d_k + 8 * kAttnKRow, g_k + (adv + 8) * kAttnKRow);
+      cp_async16(st + d_v, g_v + adv * kAttnKRow);
+      cp_async16(st + d_v + 8 * kAttnVRow, g_v + (adv + 8) * kAttnKRow);
+      cp_async4(st + d_s, g_s + adv);
+    } else {  // ragged last tile: rows past t_end are zero-filled, never read
+      // (their source address is replaced by the first row of the head).
+      const bool v0 = t0 + ctok < t_end, v1 = t0 + ctok + 8 < t_end;
+      const bool vs = t0 + (lane & 15) < t_end;
+      const float* s0 = lane < 16 ? ksc : vsc;
+      cp_async16_zfill(st + d_k, v0 ? g_k + adv * kAttnKRow : kc, v0);
+      cp_async16_zfill(st + d_k + 8 * kAttnKRow, v1 ? g_k + (adv + 8) * kAttnKRow : kc, v1);
+      cp_async16_zfill(st + d_v, v0 ? g_v + adv * kAttnKRow : vc, v0);
+      cp_async16_zfill(st + d_v + 8 * kAttnVRow, v1 ? g_v + (adv + 8) * kAttnKRow : vc, v1);
+      cp_async4_zfill(st + d_s, vs ? g_s + adv : s0, vs);
+    }
+  };
+
+  float o[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+
+#pragma unroll
+  for (int k = 0; k < STAGES - 1; ++k) {
+    if (k < nw) issue(k);
+    cp_async_commit();
+  }
+
+  for (int k = 0; k < nw; ++k) {
+    if (k + STAGES - 1 < nw) issue(k + STAGES - 1);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
+    __syncwarp();
+
+    const uint8_t* st = sm.u.stage[w][k % STAGES];
+    const int64_t t0 = t_begin + int64_t(w + kAttnWarps * k) * kAttnTile;
+
+    // --- scores: S^T[head x digit, token] = Qdigits . (16 * kcode) ---
+    int c0[4] = {0, 0, 0, 0}, c1[4] = {0, 0, 0, 0};
+    {
+      const uint4 k0 = *reinterpret_cast<const uint4*>(st + g * kAttnKRow + 16 * j);
+      const uint4 k1 = *reinterpret_cast<const uint4*>(st + (g + 8) * kAttnKRow + 16 * j);
+      const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
+      const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        uint32_t e, od;
+        int4x8_to_s8x16(kw0[s], e, od);
+        mma_s8_16832(c0, qa[s], e, od);
+        int4x8_to_s8x16(kw1[s], e, od);
+        mma_s8_16832(c1, qa[s], e, od);
+      }
+    }
+    const float* sc = reinterpret_cast<const float*>(st + kAttnStS);
+    const float2 ks01 = *reinterpret_cast<const float2*>(sc + 2 * j);
+    const float2 ks89 = *reinterpret_cast<const float2*>(sc + 8 + 2 * j);
+    const float2 vs01 = *reinterpret_cast<const float2*>(sc + 16 + 2 * j);
+    const float2 vs89 = *reinterpret_cast<const float2*>(sc + 24 + 2 * j);
+
+    // Tokens of this lane: 2j, 2j+1 (columns of the first n8 tile) and
+    // 2j+8, 2j+9 (second tile); the same tokens it feeds to the PV product.
+    float sv[4];
+    sv[0] = fmaf(float(c0[2]), wh, float(c0[0]) * wl);
+    sv[1] = fmaf(float(c0[3]), wh, float(c0[1]) * wl);
+    sv[2] = fmaf(float(c1[2]), wh, float(c1[0]) * wl);
+    sv[3] = fmaf(float(c1[3]), wh, float(c1[1]) * wl);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], 16);
+    const float ksv[4] = {ks01.x, ks01.y, ks89.x, ks89.y};
+    const int toff[4] = {2 * j, 2 * j + 1, 2 * j + 8, 2 * j + 9};
+    float mt = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sv[i] = (t0 + toff[i] < t_end) ? sv[i] * (qs * ksv[i]) : -INFINITY;
+      mt = fmaxf(mt, sv[i]);
+    }
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+
+    // --- online softmax (base 2); the running max is raised only when the
+    // tile max exceeds it by more than kAttnSlack, so p stays <= 2^8 ---
+    const bool need = mt > m_run + kAttnSlack;
+    if (__any_sync(0xffffffffu, need)) {
+      const float alpha = need ? exp2f(m_run - mt) : 1.f;
+      if (need) m_run = mt;
+      l_run *= alpha;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        mul2(o[i][0], o[i][1], alpha);
+        mul2(o[i][2], o[i][3], alpha);
+      }
+    }
+    float p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = exp2f(sv[i] - m_run);
+    l_run += (p[0] + p[1]) + (p[2] + p[3]);
+    const float vsv[4] = {vs01.x, vs01.y, vs89.x, vs89.y};
+
+    // --- A operand of PV: rows (head, part), part 0/1/2 = hi/mid/lo of
+    // p * vscale, part 3 zero.  Lanes g < 4 hold parts 0 and 2, g >= 4 part 1.
+    uint32_t pa[4];
+    {
+      uint32_t h01, m01, l01, h89, m89, l89;
+      split3_bf16(p[0] * vsv[0], p[1] * vsv[1], h01, m01, l01);
+      split3_bf16(p[2] * vsv[2], p[3] * vsv[3], h89, m89, l89);
+      const bool low = g < 4;
+      pa[0] = low ? h01 : m01;
+      pa[1] = low ? l01 : 0u;
+      pa[2] = low ? h89 : m89;
+      pa[3] = low ? l89 : 0u;
+    }
+
+    // --- PV: O[(head, part), dim] += P . V; lane (g, j) feeds the value
+    // codes of dims 16g + i (n8 tile i) for tokens 2j, 2j+1 / 2j+8, 2j+9 ---
+    {
+      const uint8_t* svp = st + kAttnStV + 8 * g;
+      const uint2 va = *reinterpret_cast<const uint2*>(svp + (2 * j) * kAttnVRow);
+      const uint2 vb = *reinterpret_cast<const uint2*>(svp + (2 * j + 1) * kAttnVRow);
+      const uint2 vcx = *reinterpret_cast<const uint2*>(svp + (2 * j + 8) * kAttnVRow);
+      const uint2 vd = *reinterpret_cast<const uint2*>(svp + (2 * j + 9) * kAttnVRow);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t sel = (h & 1) ? 0x7632u : 0x5410u;
+        const uint32_t xab = __byte_perm(h < 2 ? va.x : va.y, h < 2 ? vb.x : vb.y, sel);
+        const uint32_t xcd = __byte_perm(h < 2 ? vcx.x : vcx.y, h < 2 ? vd.x : vd.y, sel);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          mma_bf16_16816(o[4 * h + e], pa, int4x2_to_bf16x2(xab >> (4 * e)), int4x2_to_bf16x2(xcd >> (4 * e)));
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+  // ---- merge the warp's parts and store it for the CTA merge ----
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  float oa[16], ob[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    oa[i] = o[i][0] + o[i][2];
+    ob[i] = o[i][1] + o[i][3];
+    oa[i] += __shfl_xor_sync(0xffffffffu, oa[i], 16);
+    ob[i] += __shfl_xor_sync(0xffffffffu, ob[i], 16);
+  }
+  __syncthreads();  // every warp is done with its ring: the merge area may reuse it
+  // Lane (g < 4, j) holds head g at dims 32j + i (oa) and 32j + 16 + i (ob).
+  // The merge area and the workspace keep a head's 128 values in the order
+  // idx = 8 * (dim & 15) + 4 * ((dim >> 4) & 1) + (dim >> 5), a permutation of
+  // the index bits, under which H_128 is unchanged.
+  if (g < 4) {
+    float* cb = sm.u.comb[w][g];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      cb[8 * i + j] = oa[i];
+      cb[8 * i + 4 + j] = ob[i];
+    }
+    if (j == 0) {
+      sm.m[w][g] = m_run;
+      sm.l[w][g] = l_run;
+    }
+  }
+  __syncthreads();
+
+  // ---- CTA merge: thread (head w, lane) owns idx 4*lane .. 4*lane+3 ----
+  const int64_t slot = (int64_t(grp) * a.splits + split) * kAttnHeads + w;
+  {
+    float M = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kAttnWarps; ++u) M = fmaxf(M, sm.m[u][w]);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kAttnWarps; ++u) {
+      const float mu = sm.m[u][w];
+      const float f = mu == -INFINITY ? 0.f : exp2f(mu - M);
+      L = fmaf(f, sm.l[u][w], L);
+      const float4 v = *reinterpret_cast<const float4*>(&sm.u.comb[u][w][4 * lane]);
+      acc.x = fmaf(f, v.x, acc.x);
+      acc.y = fmaf(f, v.y, acc.y);
+      acc.z = fmaf(f, v.z, acc.z);
+      acc.w = fmaf(f, v.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(a.part_o + slot * kAttnDim + 4 * lane) = acc;
+    if (lane == 0) *reinterpret_cast<float2*>(a.part_ml + slot * 2) = make_float2(M, L);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.last = atomicAdd(a.counters + grp, 1u) == unsigned(a.splits - 1);
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+
+  // ---- last CTA of the group: merge all splits, undo the rotation ----
+  if (w < hn) {
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < a.splits; ++sp) {
+      const int64_t sl = (int64_t(grp) * a.splits + sp) * kAttnHeads + w;
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + sl * 2));
+      if (ml.x == -INFINITY) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + sl * kAttnDim + 4 * lane));
+      const float Mn = fmaxf(M, ml.x);
+      const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      const float fn = exp2f(ml.x - Mn);
+      L = L * fo + ml.y * fn;
+      acc.x = acc.x * fo + v.x * fn;
+      acc.y = acc.y * fo + v.y * fn;
+      acc.z = acc.z * fo + v.z * fn;
+      acc.w = acc.w * fo + v.w * fn;
+      M = Mn;
+    }
+    const float inv = a.inv_sqrt_dim / L;
+    float y[4] = {acc.x, acc.y, acc.z, acc.w};
+    // H_128 on the permuted index: bits 0-1 in registers, bits 2-6 on lanes.
+    bfly(y[0], y[1]);
+    bfly(y[2], y[3]);
+    bfly(y[0], y[2]);
+    bfly(y[1], y[3]);
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float ov = __shfl_xor_sync(0xffffffffu, y[i], m);
+        y[i] = upper ? ov - y[i] : y[i] + ov;
+      }
+    }
+    const int64_t orow = (int64_t(bidx) * a.nqh + head0 + w) * kAttnDim;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      // idx = 4*lane + r  ->  dim = 32 r + 16 (lane & 1) + (lane >> 1)
+      const int dim = 32 * r + 16 * (lane & 1) + (lane >> 1);
+      float v = y[r] * inv;
+      if (a.signs && a.signs[dim] < 0) v = -v;
+      if (a.out_f32)
+        static_cast<float*>(a.out)[orow + dim] = v;
+      else
+        static_cast<uint16_t*>(a.out)[orow + dim] = uint16_t(pack_bf16x2(v, 0.f) & 0xffffu);
+    }
+  }
+  if (tid == 0) a.counters[grp] = 0u;  // ready for the next call
+}
+
+}  // namespace hadq

@@ -22,3 +22,11 @@ const void* full4096_kernel_ptr(int bits, bool signs, int logG);
 const void* generic_kernel_ptr(int direction, int bits);
 
 }  // namespace hadq
+
+namespace hadq {
+
+// Decode attention over the rotated INT4 KV cache (head dim 128, one scale
+// per cached row), 128 threads per CTA.
+const void* kv_decode_attn_kernel_ptr();
+
+}  // namespace hadq

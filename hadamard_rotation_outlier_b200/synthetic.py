@@ -229,3 +229,71 @@ def random_signs(dim: int, seed: int) -> np.ndarray:
     """Seeded +-1 int8 sign vector of length ``dim``."""
     rng = np.random.default_rng(np.random.SeedSequence([seed, 0x5161, dim]))
     return (rng.integers(0, 2, size=dim) * 2 - 1).astype(np.int8)
+
+
+# ------------------------------------------------------------------ decode
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """One decode step of attention over a rotated INT4 KV cache.
+
+    ``batch`` sequences, each with ``n_q_heads`` query heads (one new token)
+    and ``n_kv_heads`` cached heads of ``tokens`` rows at head dim ``dim``.
+    """
+    name: str
+    description: str
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    tokens: int
+    dim: int = 128
+    with_signs: bool = False
+
+    def attn_bytes(self, out_bytes_per_elem: int = 2) -> int:
+        """bf16 query in + K and V codes + K and V row scales in + output,
+        each byte moved once."""
+        rows = self.batch * self.n_kv_heads * self.tokens
+        q = self.batch * self.n_q_heads * self.dim
+        return 2 * q + 2 * rows * (self.dim // 2) + 2 * rows * 4 + out_bytes_per_elem * q
+
+
+DECODE_WORKLOADS = {
+    "d1_decode_q32_kv8_t131072_d128_int4": DecodeWorkload(
+        name="d1_decode_q32_kv8_t131072_d128_int4",
+        description="one decode step: 32 query heads, 8 KV heads (4 per group), the "
+                    "131072-token INT4 cache of K and V [8,131072,128]",
+        batch=1, n_q_heads=32, n_kv_heads=8, tokens=131072),
+}
+
+
+def decode_query(batch: int, n_q_heads: int, dim: int, seed: int, outlier_dims: int = 2,
+                 outlier_scale: float = 50.0) -> np.ndarray:
+    """Seeded query rows, bf16 bits [batch, n_q_heads, dim]: N(0,1) with
+    ``outlier_dims`` seeded columns per head scaled by ``outlier_scale``."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x0E7A, batch, n_q_heads, dim]))
+    v = rng.standard_normal((batch, n_q_heads, dim), dtype=np.float32)
+    for h in range(n_q_heads):
+        cols = rng.choice(dim, size=outlier_dims, replace=False)
+        v[:, h, cols] *= np.float32(outlier_scale)
+    return f32_to_bf16_bits(v)
+
+
+def random_int4_cache(batch: int, n_kv_heads: int, stride: int, dim: int, seed: int,
+                      scale_range=(0.25, 0.75)):
+    """Seeded packed INT4 cache rows and positive float32 row scales.
+
+    Each code is an independent draw of binomial(14, 1/2) - 7 (values -7..7,
+    standard deviation 1.87), taken as the number of set bits among 14 random
+    bits minus 7, and stored as 4-bit two's complement with element 2j in the
+    low nibble of byte j.  Returns ``(codes uint8 [batch, n_kv_heads, stride,
+    dim/2], scales float32 [batch, n_kv_heads, stride])``.
+    """
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0xCAC4, batch, n_kv_heads, stride, dim]))
+    shape = (batch, n_kv_heads, stride, dim // 2)
+    ones = np.array([bin(v).count("1") - 7 for v in range(1 << 14)], dtype=np.int8)
+    lo = ones[rng.integers(0, 1 << 14, size=shape, dtype=np.uint16)]
+    hi = ones[rng.integers(0, 1 << 14, size=shape, dtype=np.uint16)]
+    codes = ((lo.view(np.uint8) & 0xF) | ((hi.view(np.uint8) & 0xF) << 4)).astype(np.uint8)
+    scales = rng.uniform(scale_range[0], scale_range[1],
+                         size=(batch, n_kv_heads, stride)).astype(np.float32)
+    return codes, scales

@@ -57,7 +57,7 @@ typedef struct CUstream_st *hadq_stream_t;
 typedef enum {
   HADQ_OK = 0,
   HADQ_ERR_INVALID_ARG = 1,  /* out-of-range size, NULL pointer, bad enum     */
-  HADQ_ERR_UNSUPPORTED = 2,  /* valid maths, no kernel for it (not used now)  */
+  HADQ_ERR_UNSUPPORTED = 2,  /* valid maths, no kernel for it                 */
   HADQ_ERR_MISALIGNED = 3,   /* pointer not aligned to its element size       */
   HADQ_ERR_CUDA = 4          /* the CUDA runtime reported an error            */
 } hadq_status;
@@ -121,6 +121,65 @@ hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int6
                                     int32_t dim, int32_t block, const int8_t *signs,
                                     int32_t bits, int32_t group, void *out,
                                     hadq_out_dtype out_dtype, hadq_stream_t stream);
+
+/*
+ * hadq_kv_decode_attention -- one decode step of attention over a KV cache
+ * stored in the rotated basis as INT4 codes.
+ *
+ * The cache rows are what hadq_rotate_quantize writes for dim 128, block 128
+ * (or -1), group 128 (or -1), bits 4 and the same signs: K_rot = (K * s) H and
+ * V_rot = (V * s) H, quantised per row.  Because H is orthogonal,
+ * (q H)(K H)^T = q K^T ("Hartmann rotation, lightweight QAT, streaming
+ * attention", section 1), so the scores come from the rotated query against
+ * the dequantised rotated keys, and the output is rotated back once ("QuaRot
+ * hands-on", sections 2.2 and 2.3: the 4-bit KV cache is dequantised when read,
+ * the output transformed back):
+ *
+ *   q_rot  = (q * s) H
+ *   p      = softmax_t( softmax_scale * q_rot . kcode_t * kscale_t )
+ *   out    = ((sum_t p_t * vcode_t * vscale_t) H) * s
+ *
+ *   q            device, bfloat16 [batch, n_q_heads, dim], 8-byte aligned.
+ *   k_codes,     device, uint8 [batch, n_kv_heads, token_stride, dim/2] packed
+ *   v_codes      INT4 (element 2j in the low nibble of byte j), 16-byte
+ *                aligned.  Only the first `tokens` rows of each head are read.
+ *   k_scales,    device, float32 [batch, n_kv_heads, token_stride], 4-byte
+ *   v_scales     aligned: the per-row scales of the codes.
+ *   batch        >= 0 (0 = empty call).
+ *   n_q_heads    >= 1, a multiple of n_kv_heads; query head h reads KV head
+ *                h / (n_q_heads / n_kv_heads) (grouped-query attention).
+ *   tokens       cached tokens attended over, 1 <= tokens <= token_stride.
+ *   dim, block,  the cache's rotate+quantise parameters; the kernel supports
+ *   bits, group  dim 128, block 128 or -1, bits 4, group 128 or -1 and returns
+ *                HADQ_ERR_UNSUPPORTED for any other valid combination.
+ *   signs        device int8 [dim] (4-byte aligned) or NULL, as for the cache.
+ *   softmax_scale  > 0 and finite (usually 1/sqrt(dim)).
+ *   out          device output [batch, n_q_heads, dim]: bfloat16 (8-byte
+ *                aligned) or float32 (16-byte aligned).
+ *   workspace    device scratch of at least hadq_kv_decode_workspace_size()
+ *                bytes, 256-byte aligned, owned by the caller.  It must be
+ *                zero-filled before its first use; every call leaves it ready
+ *                for the next one.  Calls sharing a workspace must be ordered
+ *                (same stream, or synchronised).
+ * Queries whose scaled rotated entries are all below 2^-100 in magnitude are
+ * treated as zero (uniform weights).  No other rounding beyond float32.
+ */
+hadq_status hadq_kv_decode_attention(const void *q, const void *k_codes, const float *k_scales,
+                                     const void *v_codes, const float *v_scales, int32_t batch,
+                                     int32_t n_q_heads, int32_t n_kv_heads, int64_t tokens,
+                                     int64_t token_stride, int32_t dim, int32_t block,
+                                     const int8_t *signs, int32_t bits, int32_t group,
+                                     float softmax_scale, void *out, hadq_out_dtype out_dtype,
+                                     void *workspace, size_t workspace_bytes,
+                                     hadq_stream_t stream);
+
+/*
+ * hadq_kv_decode_workspace_size -- host-only: bytes of workspace that
+ * hadq_kv_decode_attention needs for these sizes on any device (an upper bound
+ * that does not depend on the GPU).  Writes *bytes; validates like the call.
+ */
+hadq_status hadq_kv_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                          int64_t tokens, size_t *bytes);
 
 /*
  * hadq_plan -- host-only: validate the sizes of a call and report the kernel

@@ -53,6 +53,7 @@ __all__ = [
     "quant_error",
     "half_boundary_distance",
     "dequant_rotated",
+    "kv_decode_scores",
     "kv_decode_attention",
 ]
 
@@ -292,6 +293,35 @@ def dequant_rotated(codes: np.ndarray, scales: np.ndarray, dim: int, bits: int =
     return (q.reshape(lead + (dim // G, G)) * s[..., None]).reshape(lead + (dim,))
 
 
+def kv_decode_scores(q_bits: np.ndarray, k_codes: np.ndarray, k_scales: np.ndarray, dim: int,
+                     block: int = -1, signs=None, bits: int = 4, group: int = -1,
+                     softmax_scale: float | None = None) -> np.ndarray:
+    """Attention scores of one decode query per head against a rotated,
+    quantised key cache: softmax_scale * q_rot . k_hat_t, float64
+    [batch, n_q_heads, tokens].
+
+    [Hartmann rotation] §1: Q_rot K_rot^T = Q K^T, so the rotated query
+    against the dequantised rotated keys gives the scores of the un-rotated
+    ones.  Query head h reads KV head h // (n_q_heads / n_kv_heads).
+    """
+    q = bf16_bits_to_f64(q_bits)
+    nb, nqh, d = q.shape
+    assert d == dim
+    kr = dequant_rotated(k_codes, k_scales, dim, bits, group)   # [b, hk, T, d]
+    nkh = kr.shape[1]
+    if nqh % nkh:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    g = nqh // nkh
+    if softmax_scale is None:
+        softmax_scale = 1.0 / np.sqrt(dim)
+    qr = rotate(q, block=block, signs=signs)
+    s = np.empty((nb, nqh, kr.shape[2]))
+    for b in range(nb):
+        for h in range(nqh):
+            s[b, h] = softmax_scale * (kr[b, h // g] @ qr[b, h])
+    return s
+
+
 def kv_decode_attention(q_bits: np.ndarray, k_codes: np.ndarray, k_scales: np.ndarray,
                         v_codes: np.ndarray, v_scales: np.ndarray, dim: int, block: int = -1,
                         signs=None, bits: int = 4, group: int = -1,
@@ -301,9 +331,8 @@ def kv_decode_attention(q_bits: np.ndarray, k_codes: np.ndarray, k_scales: np.nd
 
     * [QuaRot hands-on] §2.2: K and V are rotated online and stored in 4 bits,
       then dequantised when they are read for attention.
-    * [Hartmann rotation] §1: Q_rot K_rot^T = Q K^T, so the scores come from
-      the rotated query against the rotated keys, without undoing the
-      rotation of K.
+    * Scores from :func:`kv_decode_scores` (rotated query against rotated
+      keys, [Hartmann rotation] §1), softmax over the cached tokens.
     * P V_rot = (P V) H: the output is computed in the rotated basis and
       transformed back once ([QuaRot hands-on] §2.3), with H and the signs
       of :func:`inverse_rotate`.
@@ -313,26 +342,16 @@ def kv_decode_attention(q_bits: np.ndarray, k_codes: np.ndarray, k_scales: np.nd
     n_kv_heads, tokens, dim/G].  Query head h reads KV head h // (n_q_heads /
     n_kv_heads).  Returns float64 [batch, n_q_heads, dim].
     """
-    q = bf16_bits_to_f64(q_bits)
-    nb, nqh, d = q.shape
-    assert d == dim
-    kr = dequant_rotated(k_codes, k_scales, dim, bits, group)   # [b, hk, T, d]
-    vr = dequant_rotated(v_codes, v_scales, dim, bits, group)
-    nkh = kr.shape[1]
-    if nqh % nkh:
-        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
-    g = nqh // nkh
-    if softmax_scale is None:
-        softmax_scale = 1.0 / np.sqrt(dim)
-    qr = rotate(q, block=block, signs=signs)
+    s = kv_decode_scores(q_bits, k_codes, k_scales, dim, block, signs, bits, group, softmax_scale)
+    vr = dequant_rotated(v_codes, v_scales, dim, bits, group)   # [b, hk, T, d]
+    nb, nqh, _ = s.shape
+    g = nqh // vr.shape[1]
     out = np.empty((nb, nqh, dim))
     for b in range(nb):
         for h in range(nqh):
-            kv = h // g
-            s = softmax_scale * (kr[b, kv] @ qr[b, h])
-            p = np.exp(s - s.max())
+            p = np.exp(s[b, h] - s[b, h].max())
             p /= p.sum()
-            out[b, h] = p @ vr[b, kv]
+            out[b, h] = p @ vr[b, h // g]
     return inverse_rotate(out, block=block, signs=signs)
 
 

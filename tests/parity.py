@@ -14,6 +14,13 @@
   (round to nearest, ties to even), where the value's float32 error allowed
   above (1e-5 of max(|o|, row RMS)) is added to that ulp: a value near zero
   may carry an absolute float32 error several bf16 ulps wide.
+* Decode attention: the rule for float32 values above plus the conditioning
+  of softmax on float32 scores.  A score s held in float32 (log2 units, after
+  a few roundings) is off by at most 16 u |s| (u = 2^-24); a weight then moves
+  by p_t ln2 (ds_t - sum_t' p_t' ds_t'), so output element d moves by at most
+  2 ln2 * 16 u * (sum_t p_t |s_t|) * max_t |v_td - o_d|.  That term is added
+  to the allowance of each output element (v: dequantised values in the
+  original basis).
 """
 
 from __future__ import annotations
@@ -125,3 +132,48 @@ def check_bf16(g_bits: np.ndarray, o: np.ndarray, what: str) -> int:
                              f"first at {i}: gpu {g[i]!r} oracle {o[i]!r}")
     d = np.abs(_ordered(g_bits) - _ordered(ref))
     return int(d.max()) if d.size else 0
+
+
+ATTN_SCORE_ULPS = 16
+U32 = 2.0 ** -24
+
+
+def attention_allowance(o: np.ndarray, scores: np.ndarray, values: np.ndarray, group: int) -> np.ndarray:
+    """Per-element allowance of the decode-attention output (see module note).
+
+    ``o`` [b, h, d] oracle output; ``scores`` [b, h, T] oracle scores (natural
+    units); ``values`` [b, kvh, T, d] dequantised values in the original
+    basis; query head h reads KV head h // group.
+    """
+    s2 = scores * np.log2(np.e)
+    p = np.exp(scores - scores.max(axis=-1, keepdims=True))
+    p /= p.sum(axis=-1, keepdims=True)
+    sbar = np.sum(p * np.abs(s2), axis=-1)                        # [b, h]
+    nb, nh, d = o.shape
+    spread = np.empty_like(o)
+    for b in range(nb):
+        for h in range(nh):
+            spread[b, h] = np.max(np.abs(values[b, h // group] - o[b, h]), axis=0)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True))
+    return (REL_TOL * np.maximum(np.abs(o), rms)
+            + 2 * np.log(2.0) * ATTN_SCORE_ULPS * U32 * sbar[..., None] * spread)
+
+
+def check_attention(g: np.ndarray, o: np.ndarray, allowance: np.ndarray, what: str,
+                    bf16: bool = False) -> float:
+    """Compare a decode-attention output (float32 values or bf16 bits) with
+    the oracle under :func:`attention_allowance`; bf16 adds one bf16 ulp.
+    Returns the largest error as a fraction of the allowance."""
+    o = np.asarray(o, dtype=np.float64)
+    if bf16:
+        gv = decode_bf16(np.asarray(g, dtype=np.uint16).reshape(o.shape))
+        allowance = allowance + bf16_ulp(o)
+    else:
+        gv = np.asarray(g, dtype=np.float64).reshape(o.shape)
+    err = np.abs(gv - o)
+    bad = err > allowance
+    if np.any(bad):
+        i = tuple(np.argwhere(bad)[0])
+        raise AssertionError(f"{what}: {int(bad.sum())} values off; first at {i}: gpu {gv[i]!r} "
+                             f"oracle {o[i]!r} allowance {allowance[i]:.3e}")
+    return float(np.max(err / allowance)) if err.size else 0.0

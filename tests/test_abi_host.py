@@ -138,3 +138,72 @@ def test_last_error_is_cleared_by_a_good_call(lib):
     assert B.hadq_last_error()
     lib.hadq_rotate_quantize(None, 0, 128, 64, None, 8, -1, None, None, None, None)
     assert B.hadq_last_error() == ""
+
+
+# ------------------------------------------------------ decode attention
+
+def test_decode_workspace_size(lib):
+    # counters (256-byte block), (m, l) per split and head, O per split and head
+    n = B.hadq_kv_decode_workspace_size(1, 32, 8, 131072)
+    groups, splits = 8, 256
+    assert n == 256 + groups * splits * 4 * 2 * 4 + groups * splits * 4 * 128 * 4
+    small = B.hadq_kv_decode_workspace_size(2, 8, 8, 10)   # one split per group
+    assert small == 256 + 16 * 4 * 2 * 4 + 16 * 4 * 128 * 4
+    assert B.hadq_kv_decode_workspace_size(0, 8, 8, 10) == 0
+
+
+@pytest.mark.parametrize("args,msg", [
+    ((-1, 8, 8, 10), "batch"),
+    ((1, 0, 8, 10), "n_q_heads"),
+    ((1, 6, 4, 10), "multiple"),
+    ((1, 8, 8, 0), "tokens"),
+])
+def test_decode_workspace_size_rejects(lib, args, msg):
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_kv_decode_workspace_size(*args)
+    assert e.value.status == B.HADQ_ERR_INVALID_ARG and msg in str(e.value)
+
+
+def _attn(lib, q=0x10000, kc=0x10000, ks=0x10000, vc=0x10000, vs=0x10000, batch=1, nqh=4, nkv=1,
+          tokens=16, stride=16, dim=128, block=128, signs=None, bits=4, group=128, scale=0.1,
+          out=0x10000, dtype=B.HADQ_OUT_BF16, ws=0x10000, ws_bytes=1 << 20):
+    vp = ctypes.c_void_p
+    p = lambda v: None if v is None else vp(v)
+    return lib.hadq_kv_decode_attention(p(q), p(kc), p(ks), p(vc), p(vs), batch, nqh, nkv, tokens, stride,
+                                        dim, block, p(signs), bits, group, scale, p(out), dtype, p(ws),
+                                        ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(stride=8), B.HADQ_ERR_INVALID_ARG, "token_stride"),
+    (dict(tokens=0), B.HADQ_ERR_INVALID_ARG, "tokens"),
+    (dict(nqh=6, nkv=4), B.HADQ_ERR_INVALID_ARG, "multiple"),
+    (dict(scale=0.0), B.HADQ_ERR_INVALID_ARG, "softmax_scale"),
+    (dict(scale=float("inf")), B.HADQ_ERR_INVALID_ARG, "softmax_scale"),
+    (dict(dtype=5), B.HADQ_ERR_INVALID_ARG, "out_dtype"),
+    (dict(dim=64, block=64, group=64), B.HADQ_ERR_UNSUPPORTED, "dim 128"),
+    (dict(bits=8), B.HADQ_ERR_UNSUPPORTED, "bits 4"),
+    (dict(group=32), B.HADQ_ERR_UNSUPPORTED, "group 128"),
+    (dict(block=64), B.HADQ_ERR_UNSUPPORTED, "block 128"),
+    (dict(block=48), B.HADQ_ERR_INVALID_ARG, "power of two"),
+    (dict(ws=None), B.HADQ_ERR_INVALID_ARG, "NULL"),
+    (dict(q=0x10004), B.HADQ_ERR_MISALIGNED, "q must"),
+    (dict(kc=0x10008), B.HADQ_ERR_MISALIGNED, "codes"),
+    (dict(vs=0x10002), B.HADQ_ERR_MISALIGNED, "scales"),
+    (dict(signs=0x10002), B.HADQ_ERR_MISALIGNED, "signs"),
+    (dict(out=0x10008, dtype=B.HADQ_OUT_F32), B.HADQ_ERR_MISALIGNED, "out"),
+    (dict(ws=0x10010), B.HADQ_ERR_MISALIGNED, "workspace"),
+    (dict(ws_bytes=100), B.HADQ_ERR_INVALID_ARG, "workspace of 100 bytes"),
+])
+def test_decode_attention_rejects_before_launch(lib, kw, status, msg):
+    n0 = B.hadq_launch_count()
+    st = _attn(lib, **kw)
+    assert st == status, (st, B.hadq_last_error())
+    assert msg in B.hadq_last_error()
+    assert B.hadq_launch_count() == n0
+
+
+def test_decode_attention_empty_batch_is_a_noop(lib):
+    n0 = B.hadq_launch_count()
+    assert _attn(lib, batch=0, q=None, kc=None, ks=None, vc=None, vs=None, out=None, ws=None) == B.HADQ_OK
+    assert B.hadq_launch_count() == n0

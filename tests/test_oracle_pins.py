@@ -464,3 +464,19 @@ def test_decode_attention_rejects_bad_head_ratio():
     qbits = np.zeros((1, 3, 64), np.uint16)
     with pytest.raises(ValueError):
         O.kv_decode_attention(qbits, kc, ks, kc, ks, 64, -1, None, 8, 64)
+
+
+def test_decode_scores_equal_unrotated_dot_products():
+    # The scores alone: rotated query against rotated keys = q . k / sqrt(d)
+    # with the keys un-rotated through scipy's H.
+    rng = np.random.default_rng(12)
+    nb, nqh, nkv, T, dim = 1, 6, 3, 11, 64
+    signs = S.random_signs(dim, 12)
+    qk, kc, ks = _random_kv_codes(rng, nb, nkv, T, dim, 4, 32)
+    qbits = S.f32_to_bf16_bits(rng.normal(size=(nb, nqh, dim)).astype(np.float32))
+    got = O.kv_decode_scores(qbits, kc, ks, dim, 32, signs, 4, 32, softmax_scale=0.3)
+    deq = (qk.reshape(nb, nkv, T, 2, 32) * ks.astype(np.float64)[..., None]).reshape(nb, nkv, T, dim)
+    K = _scipy_unrotate(deq, dim, 32, signs)
+    x = O.bf16_bits_to_f64(qbits)
+    for h in range(nqh):
+        np.testing.assert_allclose(got[0, h], 0.3 * K[0, h // 2] @ x[0, h], rtol=1e-12, atol=1e-12)
