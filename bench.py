@@ -5,7 +5,10 @@
 
 One step is one pass of the hot path over the workload's whole batch: one
 rotate+quantise launch over every input row (plus, for the KV-cache workload,
-one dequantise+inverse launch to bf16).  Inputs are resident in HBM before the
+one dequantise+inverse launch to bf16).  The decode workload
+(``--workload d1_decode_q32_kv8_t131072_d128_int4``) instead times one decode
+step of attention over the rotated INT4 KV cache: one launch that reads every
+cached K/V code and scale once.  Inputs are resident in HBM before the
 timed region.  Between timed steps a 256 MiB buffer is written to flush the
 126 MB L2; that write sits outside the CUDA events that time each step.  The
 default workload is the Q/K rotation (2 x [1, 32, 8192, 128] bf16, full
@@ -252,6 +255,163 @@ def aggregate_gbs(world: int, bytes_per_step: int, steps: int, total_ms: float) 
     return world * bytes_per_step * steps / (total_ms * 1e-3) / 1e9
 
 
+DECODE_METRIC = ("decode attention over the rotated INT4 KV cache, GB/s (bf16 query + K/V codes + "
+                 "K/V scales in, bf16 out), % of B200 HBM peak")
+
+
+def decode_oracle_rate(dw, target_s: float, seed: int = 71):
+    """Time the oracle's decode attention on a bounded token sample of ``dw``
+    (one KV head and its query heads); returns (GB/s, info)."""
+    import oracle as O
+    from hadamard_rotation_outlier_b200 import synthetic as S
+
+    g = dw.n_q_heads // dw.n_kv_heads
+    q = S.decode_query(1, g, dw.dim, seed)
+
+    def run(tokens):
+        kc, ks = S.random_int4_cache(1, 1, tokens, dw.dim, seed + 1)
+        vc, vs = S.random_int4_cache(1, 1, tokens, dw.dim, seed + 2)
+        t = time.perf_counter()
+        O.kv_decode_attention(q, kc, ks, vc, vs, dw.dim, 128, None, 4, 128)
+        return time.perf_counter() - t
+
+    n = 4096
+    dt = run(n)
+    while dt < 0.2 * target_s and n < dw.tokens:
+        n = min(dw.tokens, int(n * min(8.0, max(2.0, 0.5 * target_s / max(dt, 1e-3)))))
+        dt = run(n)
+    nbytes = 2 * g * dw.dim + 2 * n * (dw.dim // 2) + 2 * n * 4 + 2 * g * dw.dim
+    info = {"tokens": n, "q_heads": g, "seconds": round(dt, 3), "bytes": int(nbytes)}
+    return nbytes / dt / 1e9, info
+
+
+def run_decode(args):
+    """One decode step of attention per timed step (see the module note)."""
+    import torch
+    from hadamard_rotation_outlier_b200 import binding as B
+    from hadamard_rotation_outlier_b200 import synthetic as S
+    from hadamard_rotation_outlier_b200.build import build
+
+    dw = S.DECODE_WORKLOADS[args.workload]
+    world, rank, local = _dist_setup(args)
+    if rank == 0:
+        build()
+    _barrier(world)
+    B.load_library()
+    warmup = max(3, args.warmup)
+    steps = max(1, args.steps)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    seed = 71 + rank
+    kc, ks = S.random_int4_cache(dw.batch, dw.n_kv_heads, dw.tokens, dw.dim, seed)
+    vc, vs = S.random_int4_cache(dw.batch, dw.n_kv_heads, dw.tokens, dw.dim, seed + 1000)
+    qbits = S.decode_query(dw.batch, dw.n_q_heads, dw.dim, seed)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    k_codes, k_scales, v_codes, v_scales = to_dev(kc), to_dev(ks), to_dev(vc), to_dev(vs)
+    q = to_dev(qbits.view(np.int16)).view(torch.bfloat16)
+    out = torch.empty((dw.batch, dw.n_q_heads, dw.dim), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(B.hadq_kv_decode_workspace_size(dw.batch, dw.n_q_heads, dw.n_kv_heads, dw.tokens),
+                     dtype=torch.uint8, device=dev)
+    flusher = L2Flush(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qt, o, s):
+        B.hadq_kv_decode_attention(qt, k_codes, k_scales, v_codes, v_scales, tokens=dw.tokens, block=128,
+                                   bits=4, group=128, out=o, workspace=ws, stream=s)
+
+    for _ in range(warmup):
+        flusher()
+        step(q, out, stream)
+    torch.cuda.synchronize(dev)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    done = torch.cuda.Event()
+    clocks = ClockSampler(dev.index)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = B.hadq_launch_count()
+    torch.cuda._sleep(hold_cycles(steps))
+    for i in range(steps):
+        flusher()
+        starts[i].record(stream)
+        step(q, out, stream)
+        ends[i].record(stream)
+    done.record(stream)
+    clocks.poll_until(done)
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    launches = B.hadq_launch_count() - n0
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = _max_over_ranks(world, sum(step_ms))
+
+    # ---- end to end: the new query from pinned host memory, the output back ----
+    h_q = torch.from_numpy(qbits.view(np.int16)).pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    q_dev = torch.empty_like(q)
+
+    def e2e_step():
+        q_dev.view(torch.int16).copy_(h_q, non_blocking=True)
+        step(q_dev, out, stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        flusher()
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_ms = 0.0
+    for _ in range(args.e2e_steps):
+        flusher()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms += a.elapsed_time(b)
+    e_ms = _max_over_ranks(world, e_ms)
+
+    if rank != 0:
+        return None
+    nbytes = dw.attn_bytes()
+    value = aggregate_gbs(world, nbytes, steps, total_ms)
+    avg_ms = sum(step_ms) / steps
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (avg_ms * 1e-3) / 1e9
+    out_line = {
+        "metric": DECODE_METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": round(total_ms / steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": dw.name, "description": dw.description, "batch": dw.batch,
+            "n_q_heads": dw.n_q_heads, "n_kv_heads": dw.n_kv_heads, "tokens": dw.tokens, "dim": dw.dim,
+            "bytes_per_step": nbytes,
+            "cache": "seeded INT4 codes binomial(14,1/2)-7, row scales uniform [0.25, 0.75]",
+            "l2": "flushed between steps outside the timed events: 256 MiB written, then 256 MiB read",
+            "parallelism": f"dp{world} (independent sequences, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "kv_decode_attn_kernel", "achieved": round(achieved, 1),
+            "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)", "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(dw.name),
+            "algorithmic_bytes_per_launch": nbytes, "avg_launch_ms": round(avg_ms, 5),
+        },
+        "e2e": {"value": round(world * nbytes * args.e2e_steps / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(q.numel() * 2), "d2h_bytes_per_step": int(out.numel() * 2),
+                "steps": args.e2e_steps, "ms_per_step": round(e_ms / args.e2e_steps, 4),
+                "note": "the KV cache is decode state resident in HBM; each step uploads the new query "
+                        "and downloads the attention output"},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        rate, info = decode_oracle_rate(dw, args.cpu_seconds)
+        out_line["cpu_baseline"] = {
+            "value": round(rate, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{info['q_heads']} query heads over {info['tokens']} cached tokens of one KV head "
+                      f"through the float64 oracle in {info['seconds']} s"}
+    return out_line
+
+
 def run_ours(args):
     import torch
     from hadamard_rotation_outlier_b200 import binding as B
@@ -447,6 +607,8 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return None
+    if args.workload in S.DECODE_WORKLOADS:
+        return run_reference_decode(args, S.DECODE_WORKLOADS[args.workload], world)
     wl = S.WORKLOADS[args.workload]
     steps = max(1, args.steps if args.steps <= 5 else 3)
     target = max(1.0, args.cpu_seconds / 2)
@@ -477,9 +639,41 @@ def run_reference(args):
     }
 
 
+def run_reference_decode(args, dw, world):
+    steps = max(1, args.steps if args.steps <= 5 else 3)
+    target = max(1.0, args.cpu_seconds / 2)
+    rates, infos = [], []
+    for _ in range(steps):
+        r, info = decode_oracle_rate(dw, target)
+        rates.append(r)
+        infos.append(info)
+    total_bytes = sum(i["bytes"] for i in infos)
+    total_s = sum(i["seconds"] for i in infos)
+    value = total_bytes / total_s / 1e9
+    sample = (f"{steps} steps, each {infos[0]['q_heads']} query heads over {infos[0]['tokens']} cached "
+              f"tokens of one KV head through the float64 oracle")
+    return {
+        "impl": "reference", "metric": DECODE_METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": round(total_s / steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": dw.name, "batch": dw.batch, "n_q_heads": dw.n_q_heads,
+                   "n_kv_heads": dw.n_kv_heads, "tokens": dw.tokens, "dim": dw.dim},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
-    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        out = run_reference(args)
+    else:
+        from hadamard_rotation_outlier_b200 import synthetic as S
+        out = run_decode(args) if args.workload in S.DECODE_WORKLOADS else run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)
     if args.impl == "ours" and int(os.environ.get("WORLD_SIZE", "1")) > 1:

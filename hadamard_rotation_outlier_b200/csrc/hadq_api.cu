@@ -591,6 +591,8 @@ hadq_status hadq_kv_decode_attention(const void* q, const void* k_codes, const f
   a.qmul = (float)(double(softmax_scale) * 1.4426950408889634 / std::sqrt(double(hadq::kAttnDim)));
   a.inv_sqrt_dim = (float)(1.0 / std::sqrt(double(hadq::kAttnDim)));
   a.out_f32 = f32 ? 1 : 0;
+  a.vmask = 0x000F000Fu;
+  a.vmagic = 0x43084308u;
   void* args[] = {&a};
   cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(splits), unsigned(as.groups)), dim3(hadq::kAttnThreads),
                                    args, 0, reinterpret_cast<cudaStream_t>(stream));

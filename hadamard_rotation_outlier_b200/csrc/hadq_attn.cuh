@@ -72,6 +72,7 @@ struct AttnArgs {
   float qmul;                // softmax_scale * log2(e) / sqrt(128)
   float inv_sqrt_dim;        // 1 / sqrt(128)
   int out_f32;
+  uint32_t vmask, vmagic;    // 0x000F000F and 0x43084308 (see int4x2_to_bf16x2)
 };
 
 template <int STAGES>
@@ -121,12 +122,23 @@ __device__ __forceinline__ void cp_async4_zfill(uint32_t smem, const void* gmem,
 
 // Two INT4 codes (nibbles at bits 0-3 and 16-19 of x) -> bf16x2 holding the
 // codes exactly: the nibble with its sign bit flipped is c + 8; placed in the
-// mantissa of 128.0 it reads 136 + c, and subtracting 136 leaves c.
-__device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t x) {
-  const uint32_t t = (x & 0x000F000Fu) ^ 0x43084308u;
-  uint32_t r;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(0x43084308u));
+// mantissa of 128.0 it reads 136 + c, and subtracting 136 leaves c.  The mask
+// (0x000F000F) and the bit pattern of 136.0 twice (0x43084308) arrive as
+// kernel arguments, so that one three-input logic operation does the masking,
+// the flip and the exponent at once.
+__device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t x, uint32_t mask, uint32_t magic) {
+  uint32_t t, r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t) : "r"(x), "r"(mask), "r"(magic));  // (x & mask) ^ magic
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(t), "r"(magic));
   return r;
+}
+
+// 2^x for the softmax weights (the ISA approximation; results below 2^-126,
+// i.e. weights below 2^-126 of the running maximum, flush to zero).
+__device__ __forceinline__ float exp2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // bf16x2 of (lo, hi), round to nearest even.
@@ -261,15 +273,19 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     }
   }
   const float qs = sm.qscale[hh];
+  const uint32_t vmask = a.vmask, vmagic = a.vmagic;
   // Digit weights of the two rows this lane holds: rows g (digit g>>2) and
   // g+8 (digit (g>>2)+2; digit 3 is the zero row).
   const float wl = g < 4 ? 1.f : 256.f;
   const float wh = g < 4 ? 65536.f : 0.f;
+  const bool low = g < 4;
+  const int own = low ? 2 * j : 2 * j + 8;  // first of the two tokens this lane finishes
 
   // ---- token range of this CTA and the warp's tiles ----
   const int64_t t_begin = int64_t(split) * a.chunk;
   const int64_t t_end = min(a.tokens, t_begin + a.chunk);
-  const int ntiles = t_begin < t_end ? int((t_end - t_begin + kAttnTile - 1) / kAttnTile) : 0;
+  const int n_tok = t_begin < t_end ? int(t_end - t_begin) : 0;  // tokens of this CTA (< 2^31)
+  const int ntiles = (n_tok + kAttnTile - 1) / kAttnTile;
   const int nw = ntiles > w ? (ntiles - w + kAttnWarps - 1) / kAttnWarps : 0;
 
   const uint8_t* kc = a.k_codes + row0 * kAttnKRow;
@@ -294,8 +310,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   auto issue = [&](int k) {
     const uint32_t st = s_ring + uint32_t(k % STAGES) * kAttnStageBytes;
     const int64_t adv = int64_t(k) * kStepTok;
-    const int64_t t0 = t_begin + int64_t(w + kAttnWarps * k) * kAttnTile;
-    if (t0 + kAttnTile <= t_end) {
+    const int r0 = (w + kAttnWarps * k) * kAttnTile;  // first token of the tile, from t_begin
+    if (r0 + kAttnTile <= n_tok) {
       cp_async16(st + d_k, g_k + adv * kAttnKRow);
       cp_async16(st + d_k + 8 * kAttnKRow, g_k + (adv + 8) * kAttnKRow);
       cp_async16(st + d_v, g_v + adv * kAttnKRow);
@@ -303,8 +319,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
       cp_async4(st + d_s, g_s + adv);
     } else {  // ragged last tile: rows past t_end are zero-filled, never read
       // (their source address is replaced by the first row of the head).
-      const bool v0 = t0 + ctok < t_end, v1 = t0 + ctok + 8 < t_end;
-      const bool vs = t0 + (lane & 15) < t_end;
+      const bool v0 = r0 + ctok < n_tok, v1 = r0 + ctok + 8 < n_tok;
+      const bool vs = r0 + (lane & 15) < n_tok;
       const float* s0 = lane < 16 ? ksc : vsc;
       cp_async16_zfill(st + d_k, v0 ? g_k + adv * kAttnKRow : kc, v0);
       cp_async16_zfill(st + d_k + 8 * kAttnKRow, v1 ? g_k + (adv + 8) * kAttnKRow : kc, v1);
@@ -332,7 +348,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     __syncwarp();
 
     const uint8_t* st = sm.u.stage[w][k % STAGES];
-    const int64_t t0 = t_begin + int64_t(w + kAttnWarps * k) * kAttnTile;
+    const int r0 = (w + kAttnWarps * k) * kAttnTile;
 
     // --- scores: S^T[head x digit, token] = Qdigits . (16 * kcode) ---
     int c0[4] = {0, 0, 0, 0}, c1[4] = {0, 0, 0, 0};
@@ -350,38 +366,36 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
         mma_s8_16832(c1, qa[s], e, od);
       }
     }
+    // Scores.  Every lane holds digit partials of tokens 2j, 2j+1, 2j+8 and
+    // 2j+9 for head g & 3; the lane pair (g, g ^ 4) shares that head, and the
+    // low lane (g < 4) finishes tokens 2j, 2j+1 while the high lane finishes
+    // 2j+8, 2j+9 (`own`), each adding the partner's partials.
+    const float pl0 = fmaf(float(c0[2]), wh, float(c0[0]) * wl);
+    const float pl1 = fmaf(float(c0[3]), wh, float(c0[1]) * wl);
+    const float pl2 = fmaf(float(c1[2]), wh, float(c1[0]) * wl);
+    const float pl3 = fmaf(float(c1[3]), wh, float(c1[1]) * wl);
+    const float x0 = __shfl_xor_sync(0xffffffffu, low ? pl2 : pl0, 16);
+    const float x1 = __shfl_xor_sync(0xffffffffu, low ? pl3 : pl1, 16);
     const float* sc = reinterpret_cast<const float*>(st + kAttnStS);
-    const float2 ks01 = *reinterpret_cast<const float2*>(sc + 2 * j);
-    const float2 ks89 = *reinterpret_cast<const float2*>(sc + 8 + 2 * j);
-    const float2 vs01 = *reinterpret_cast<const float2*>(sc + 16 + 2 * j);
-    const float2 vs89 = *reinterpret_cast<const float2*>(sc + 24 + 2 * j);
-
-    // Tokens of this lane: 2j, 2j+1 (columns of the first n8 tile) and
-    // 2j+8, 2j+9 (second tile); the same tokens it feeds to the PV product.
-    float sv[4];
-    sv[0] = fmaf(float(c0[2]), wh, float(c0[0]) * wl);
-    sv[1] = fmaf(float(c0[3]), wh, float(c0[1]) * wl);
-    sv[2] = fmaf(float(c1[2]), wh, float(c1[0]) * wl);
-    sv[3] = fmaf(float(c1[3]), wh, float(c1[1]) * wl);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], 16);
-    const float ksv[4] = {ks01.x, ks01.y, ks89.x, ks89.y};
-    const int toff[4] = {2 * j, 2 * j + 1, 2 * j + 8, 2 * j + 9};
-    float mt = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      sv[i] = (t0 + toff[i] < t_end) ? sv[i] * (qs * ksv[i]) : -INFINITY;
-      mt = fmaxf(mt, sv[i]);
+    const float2 ksp = *reinterpret_cast<const float2*>(sc + own);
+    const float2 vsp = *reinterpret_cast<const float2*>(sc + kAttnTile + own);
+    float sv0 = ((low ? pl0 : pl2) + x0) * (qs * ksp.x);
+    float sv1 = ((low ? pl1 : pl3) + x1) * (qs * ksp.y);
+    if (r0 + kAttnTile > n_tok) {  // ragged last tile (warp-uniform): mask the missing tokens
+      if (r0 + own >= n_tok) sv0 = -INFINITY;
+      if (r0 + own + 1 >= n_tok) sv1 = -INFINITY;
     }
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+    float mtile = fmaxf(sv0, sv1);
+    mtile = fmaxf(mtile, __shfl_xor_sync(0xffffffffu, mtile, 1));
+    mtile = fmaxf(mtile, __shfl_xor_sync(0xffffffffu, mtile, 2));
+    mtile = fmaxf(mtile, __shfl_xor_sync(0xffffffffu, mtile, 16));
 
     // --- online softmax (base 2); the running max is raised only when the
     // tile max exceeds it by more than kAttnSlack, so p stays <= 2^8 ---
-    const bool need = mt > m_run + kAttnSlack;
+    const bool need = mtile > m_run + kAttnSlack;
     if (__any_sync(0xffffffffu, need)) {
-      const float alpha = need ? exp2f(m_run - mt) : 1.f;
-      if (need) m_run = mt;
+      const float alpha = need ? exp2f(m_run - mtile) : 1.f;
+      if (need) m_run = mtile;
       l_run *= alpha;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -389,24 +403,23 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
         mul2(o[i][2], o[i][3], alpha);
       }
     }
-    float p[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = exp2f(sv[i] - m_run);
-    l_run += (p[0] + p[1]) + (p[2] + p[3]);
-    const float vsv[4] = {vs01.x, vs01.y, vs89.x, vs89.y};
+    const float p0 = exp2_ftz(sv0 - m_run);
+    const float p1 = exp2_ftz(sv1 - m_run);
+    l_run += p0 + p1;
 
     // --- A operand of PV: rows (head, part), part 0/1/2 = hi/mid/lo of
-    // p * vscale, part 3 zero.  Lanes g < 4 hold parts 0 and 2, g >= 4 part 1.
+    // p * vscale, part 3 zero.  Lanes g < 4 hold parts 0 and 2, g >= 4 part 1;
+    // each lane cut its own two tokens and takes the partner's parts it needs.
     uint32_t pa[4];
     {
-      uint32_t h01, m01, l01, h89, m89, l89;
-      split3_bf16(p[0] * vsv[0], p[1] * vsv[1], h01, m01, l01);
-      split3_bf16(p[2] * vsv[2], p[3] * vsv[3], h89, m89, l89);
-      const bool low = g < 4;
-      pa[0] = low ? h01 : m01;
-      pa[1] = low ? l01 : 0u;
-      pa[2] = low ? h89 : m89;
-      pa[3] = low ? l89 : 0u;
+      uint32_t hi, mid, lo;
+      split3_bf16(p0 * vsp.x, p1 * vsp.y, hi, mid, lo);
+      const uint32_t r1 = __shfl_xor_sync(0xffffffffu, low ? mid : hi, 16);
+      const uint32_t r2 = __shfl_xor_sync(0xffffffffu, lo, 16);
+      pa[0] = low ? hi : r1;   // row g, tokens 2j, 2j+1
+      pa[1] = low ? lo : 0u;   // row g + 8, tokens 2j, 2j+1
+      pa[2] = low ? r1 : mid;  // row g, tokens 2j+8, 2j+9
+      pa[3] = low ? r2 : 0u;   // row g + 8, tokens 2j+8, 2j+9
     }
 
     // --- PV: O[(head, part), dim] += P . V; lane (g, j) feeds the value
@@ -424,7 +437,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
         const uint32_t xcd = __byte_perm(h < 2 ? vcx.x : vcx.y, h < 2 ? vd.x : vd.y, sel);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          mma_bf16_16816(o[4 * h + e], pa, int4x2_to_bf16x2(xab >> (4 * e)), int4x2_to_bf16x2(xcd >> (4 * e)));
+          mma_bf16_16816(o[4 * h + e], pa, int4x2_to_bf16x2(xab >> (4 * e), vmask, vmagic),
+                         int4x2_to_bf16x2(xcd >> (4 * e), vmask, vmagic));
       }
     }
     __syncwarp();
@@ -434,6 +448,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   // ---- merge the warp's parts and store it for the CTA merge ----
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
   float oa[16], ob[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -491,23 +506,54 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   __threadfence();
 
   // ---- last CTA of the group: merge all splits, undo the rotation ----
+  // Pass 1: every thread fetches (m, l) pairs at once; each warp then reduces
+  // its head's maximum M and sum L and keeps the weights 2^(m - M) in shared
+  // memory.  Pass 2: independent loads of the partial outputs, weighted.
+  float2* ml_s = reinterpret_cast<float2*>(&sm.u.stage[0][0][0]);           // [splits][4]
+  float* f_s = reinterpret_cast<float*>(ml_s + kAttnMaxSplits * kAttnHeads);  // [4][splits]
+  const float2* pml = reinterpret_cast<const float2*>(a.part_ml) + int64_t(grp) * a.splits * kAttnHeads;
+  for (int i = tid; i < a.splits * kAttnHeads; i += kAttnThreads) ml_s[i] = __ldcg(pml + i);
+  __syncthreads();
   if (w < hn) {
-    float M = -INFINITY, L = 0.f;
+    float M = -INFINITY;
+    for (int sp = lane; sp < a.splits; sp += 32) M = fmaxf(M, ml_s[sp * kAttnHeads + w].x);
+#pragma unroll
+    for (int m = 16; m; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    float L = 0.f;
+    for (int sp = lane; sp < a.splits; sp += 32) {
+      const float2 ml = ml_s[sp * kAttnHeads + w];
+      const float f = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+      f_s[w * kAttnMaxSplits + sp] = f;
+      L = fmaf(f, ml.y, L);
+    }
+#pragma unroll
+    for (int m = 16; m; m >>= 1) L += __shfl_xor_sync(0xffffffffu, L, m);
+    __syncwarp();
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + (int64_t(grp) * a.splits * kAttnHeads + w) *
+                                                                      kAttnDim) + lane;
+    const float* fw = f_s + w * kAttnMaxSplits;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp = 0; sp < a.splits; ++sp) {
-      const int64_t sl = (int64_t(grp) * a.splits + sp) * kAttnHeads + w;
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml + sl * 2));
-      if (ml.x == -INFINITY) continue;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + sl * kAttnDim + 4 * lane));
-      const float Mn = fmaxf(M, ml.x);
-      const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn);
-      const float fn = exp2f(ml.x - Mn);
-      L = L * fo + ml.y * fn;
-      acc.x = acc.x * fo + v.x * fn;
-      acc.y = acc.y * fo + v.y * fn;
-      acc.z = acc.z * fo + v.z * fn;
-      acc.w = acc.w * fo + v.w * fn;
-      M = Mn;
+    int sp = 0;
+    for (; sp + 8 <= a.splits; sp += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(po + int64_t(sp + u) * kAttnHeads * (kAttnDim / 4));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float f = fw[sp + u];
+        acc.x = fmaf(f, v[u].x, acc.x);
+        acc.y = fmaf(f, v[u].y, acc.y);
+        acc.z = fmaf(f, v[u].z, acc.z);
+        acc.w = fmaf(f, v[u].w, acc.w);
+      }
+    }
+    for (; sp < a.splits; ++sp) {
+      const float4 v = __ldcg(po + int64_t(sp) * kAttnHeads * (kAttnDim / 4));
+      const float f = fw[sp];
+      acc.x = fmaf(f, v.x, acc.x);
+      acc.y = fmaf(f, v.y, acc.y);
+      acc.z = fmaf(f, v.z, acc.z);
+      acc.w = fmaf(f, v.w, acc.w);
     }
     const float inv = a.inv_sqrt_dim / L;
     float y[4] = {acc.x, acc.y, acc.z, acc.w};
