@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     HadqError,
     hadq_dequant_rotate_inv,
     hadq_kv_decode_attention,
+    hadq_kv_decode_attention_noalloc,
     hadq_kv_decode_workspace_size,
     hadq_last_error,
     hadq_launch_count,

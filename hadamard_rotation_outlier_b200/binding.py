@@ -23,7 +23,7 @@ PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 
 MAX_DIM = 32768
 
 EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_kv_decode_attention",
-            "hadq_kv_decode_workspace_size", "hadq_plan", "hadq_status_str", "hadq_last_error",
+            "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_status_str", "hadq_last_error",
             "hadq_launch_count", "hadq_version")
 
 
@@ -57,6 +57,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                              c_i32, c_i32, vp, c_i32, c_i32, ctypes.c_float, vp,
                                              ctypes.c_int, vp, ctypes.c_size_t, vp]
     lib.hadq_kv_decode_attention.restype = ctypes.c_int
+    lib.hadq_kv_decode_attention_noalloc.argtypes = [vp, vp, vp, vp, vp, c_i32, c_i32, c_i32, c_i64, c_i64,
+                                                     c_i32, c_i32, vp, c_i32, c_i32, ctypes.c_float, vp,
+                                                     ctypes.c_int, vp]
+    lib.hadq_kv_decode_attention_noalloc.restype = ctypes.c_int
     lib.hadq_kv_decode_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i64,
                                                   ctypes.POINTER(ctypes.c_size_t)]
     lib.hadq_kv_decode_workspace_size.restype = ctypes.c_int
@@ -272,4 +276,41 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
                                         _ptr(v_scales), batch, nqh, nkv, tokens, stride, dim, block,
                                         _ptr(signs), bits, group, float(softmax_scale), _ptr(out), code,
                                         _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def hadq_kv_decode_attention_noalloc(q: torch.Tensor, k_codes: torch.Tensor, k_scales: torch.Tensor,
+                                     v_codes: torch.Tensor, v_scales: torch.Tensor, out: torch.Tensor,
+                                     tokens: int | None = None, block: int = -1,
+                                     signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                                     softmax_scale: float | None = None, stream=None) -> torch.Tensor:
+    """:func:`hadq_kv_decode_attention` on the library's static scratch.
+
+    Nothing is allocated: ``out`` (bf16 or fp32 ``[batch, n_q_heads, dim]``)
+    is required and the partials use the scratch the library holds.
+    """
+    lib = load_library()
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("q must be a contiguous bf16 CUDA tensor [batch, n_q_heads, dim]")
+    batch, nqh, dim = q.shape
+    dev = q.device
+    if k_codes.dim() != 4 or v_codes.shape != k_codes.shape or k_codes.shape[0] != batch:
+        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim/2] alike")
+    nkv, stride = k_codes.shape[1], k_codes.shape[2]
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, dev)
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float32, dev, batch * nkv * stride)
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bfloat16 or float32")
+    _need(out, "out", out.dtype, dev, batch * nqh * dim)
+    if softmax_scale is None:
+        softmax_scale = 1.0 / float(dim) ** 0.5
+    code = HADQ_OUT_F32 if out.dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_kv_decode_attention_noalloc(
+        _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), batch, nqh, nkv,
+        stride if tokens is None else tokens, stride, dim, block, _ptr(signs), bits, group,
+        float(softmax_scale), _ptr(out), code, _stream(stream)))
     return out

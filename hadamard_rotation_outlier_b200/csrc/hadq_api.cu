@@ -358,6 +358,103 @@ size_t attn_ws_bytes(int64_t groups, int splits, size_t* off_ml, size_t* off_o) 
   return c + ml + o;
 }
 
+hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales, const void* v_codes,
+                      const float* v_scales, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                      int64_t tokens, int64_t token_stride, int32_t dim, int32_t block, const int8_t* signs,
+                      int32_t bits, int32_t group, float softmax_scale, void* out, hadq_out_dtype out_dtype,
+                      void* workspace, size_t workspace_bytes, bool static_scratch, hadq_stream_t stream) {
+  AttnShape as;
+  hadq_status st = attn_check(batch, n_q_heads, n_kv_heads, tokens, &as);
+  if (st != HADQ_OK) return st;
+  if (token_stride < tokens)
+    return fail(HADQ_ERR_INVALID_ARG, "token_stride %lld is below tokens %lld", (long long)token_stride,
+                (long long)tokens);
+  Shape s;
+  st = check_sizes(int64_t(batch) * n_q_heads, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(HADQ_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
+    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
+  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || s.G != hadq::kAttnDim || bits != 4)
+    return fail(HADQ_ERR_UNSUPPORTED,
+                "decode attention supports dim 128, block 128, group 128, bits 4 (got %d, %d, %d, %d)", dim,
+                s.B, s.G, bits);
+  if (batch == 0) return HADQ_OK;
+  if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || (!workspace && !static_scratch))
+    return fail(HADQ_ERR_INVALID_ARG, "q, codes, scales, out and workspace must not be NULL");
+  const bool f32 = out_dtype == HADQ_OUT_F32;
+  if (!aligned(q, 8)) return fail(HADQ_ERR_MISALIGNED, "q must be 8-byte aligned");
+  if (!aligned(k_codes, 16) || !aligned(v_codes, 16))
+    return fail(HADQ_ERR_MISALIGNED, "k_codes and v_codes must be 16-byte aligned");
+  if (!aligned(k_scales, 4) || !aligned(v_scales, 4))
+    return fail(HADQ_ERR_MISALIGNED, "k_scales and v_scales must be 4-byte aligned");
+  if (signs && !aligned(signs, 4)) return fail(HADQ_ERR_MISALIGNED, "signs must be 4-byte aligned");
+  if (!aligned(out, f32 ? 16 : 8))
+    return fail(HADQ_ERR_MISALIGNED, "out must be %d-byte aligned", f32 ? 16 : 8);
+  if (!static_scratch && !aligned(workspace, 256))
+    return fail(HADQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+
+  const void* fn = hadq::kv_decode_attn_kernel_ptr();
+  // One wave of CTAs: split the tokens of each head group so that all CTAs
+  // are resident at once (a CTA beyond the wave would run alone afterwards);
+  // at least 64 tokens (a tile per warp) per split.
+  const int64_t wave = int64_t(resident(fn, hadq::kAttnThreads, 0)) * sm_count();
+  int64_t splits = wave / as.groups;
+  if (splits > as.max_splits) splits = as.max_splits;
+  if (splits < 1) splits = 1;
+  int64_t chunk = (tokens + splits - 1) / splits;
+  chunk = (chunk + hadq::kAttnTile - 1) / hadq::kAttnTile * hadq::kAttnTile;
+  splits = (tokens + chunk - 1) / chunk;
+  size_t off_ml = 0, off_o = 0;
+  const size_t need = attn_ws_bytes(as.groups, int(splits), &off_ml, &off_o);
+  if (static_scratch) {
+    if (need > workspace_bytes)
+      return fail(HADQ_ERR_UNSUPPORTED, "these sizes need %zu bytes of scratch, above the %zu bytes the library holds",
+                  need, workspace_bytes);
+    workspace = hadq::attn_static_scratch();
+    if (!workspace) return fail(HADQ_ERR_CUDA, "cannot resolve the library's static scratch on this device");
+  } else if (workspace_bytes < need) {
+    return fail(HADQ_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu bytes needed", workspace_bytes,
+                need);
+  }
+
+  hadq::AttnArgs a{};
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_codes = static_cast<const uint8_t*>(k_codes);
+  a.k_scales = k_scales;
+  a.v_codes = static_cast<const uint8_t*>(v_codes);
+  a.v_scales = v_scales;
+  a.signs = signs;
+  a.out = out;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.counters = reinterpret_cast<unsigned*>(ws);
+  a.part_ml = reinterpret_cast<float*>(ws + off_ml);
+  a.part_o = reinterpret_cast<float*>(ws + off_o);
+  a.tokens = tokens;
+  a.stride = token_stride;
+  a.chunk = chunk;
+  a.nqh = n_q_heads;
+  a.nkv = n_kv_heads;
+  a.g = n_q_heads / n_kv_heads;
+  a.hgroups = as.hgroups;
+  a.splits = int(splits);
+  a.qmul = (float)(double(softmax_scale) * 1.4426950408889634 / std::sqrt(double(hadq::kAttnDim)));
+  a.inv_sqrt_dim = (float)(1.0 / std::sqrt(double(hadq::kAttnDim)));
+  a.out_f32 = f32 ? 1 : 0;
+  a.vmask = 0x000F000Fu;
+  a.vmagic = 0x43084308u;
+  void* args[] = {&a};
+  cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(splits), unsigned(as.groups)), dim3(hadq::kAttnThreads),
+                                   args, 0, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "decode attention launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("decode attention kernel");
+}
+
 }  // namespace
 
 extern "C" {
@@ -520,88 +617,22 @@ hadq_status hadq_kv_decode_attention(const void* q, const void* k_codes, const f
                                      float softmax_scale, void* out, hadq_out_dtype out_dtype,
                                      void* workspace, size_t workspace_bytes, hadq_stream_t stream) {
   g_last_error.clear();
-  AttnShape as;
-  hadq_status st = attn_check(batch, n_q_heads, n_kv_heads, tokens, &as);
-  if (st != HADQ_OK) return st;
-  if (token_stride < tokens)
-    return fail(HADQ_ERR_INVALID_ARG, "token_stride %lld is below tokens %lld", (long long)token_stride,
-                (long long)tokens);
-  Shape s;
-  st = check_sizes(int64_t(batch) * n_q_heads, dim, block, bits, group, &s);
-  if (st != HADQ_OK) return st;
-  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
-    return fail(HADQ_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
-  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
-    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
-  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || s.G != hadq::kAttnDim || bits != 4)
-    return fail(HADQ_ERR_UNSUPPORTED,
-                "decode attention supports dim 128, block 128, group 128, bits 4 (got %d, %d, %d, %d)", dim,
-                s.B, s.G, bits);
-  if (batch == 0) return HADQ_OK;
-  if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || !workspace)
-    return fail(HADQ_ERR_INVALID_ARG, "q, codes, scales, out and workspace must not be NULL");
-  const bool f32 = out_dtype == HADQ_OUT_F32;
-  if (!aligned(q, 8)) return fail(HADQ_ERR_MISALIGNED, "q must be 8-byte aligned");
-  if (!aligned(k_codes, 16) || !aligned(v_codes, 16))
-    return fail(HADQ_ERR_MISALIGNED, "k_codes and v_codes must be 16-byte aligned");
-  if (!aligned(k_scales, 4) || !aligned(v_scales, 4))
-    return fail(HADQ_ERR_MISALIGNED, "k_scales and v_scales must be 4-byte aligned");
-  if (signs && !aligned(signs, 4)) return fail(HADQ_ERR_MISALIGNED, "signs must be 4-byte aligned");
-  if (!aligned(out, f32 ? 16 : 8))
-    return fail(HADQ_ERR_MISALIGNED, "out must be %d-byte aligned", f32 ? 16 : 8);
-  if (!aligned(workspace, 256)) return fail(HADQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  return attn_call(q, k_codes, k_scales, v_codes, v_scales, batch, n_q_heads, n_kv_heads, tokens, token_stride,
+                   dim, block, signs, bits, group, softmax_scale, out, out_dtype, workspace, workspace_bytes,
+                   false, stream);
+}
 
-  const void* fn = hadq::kv_decode_attn_kernel_ptr();
-  // One wave of CTAs: split the tokens of each head group so that all CTAs
-  // are resident at once (a CTA beyond the wave would run alone afterwards);
-  // at least 64 tokens (a tile per warp) per split.
-  const int64_t wave = int64_t(resident(fn, hadq::kAttnThreads, 0)) * sm_count();
-  int64_t splits = wave / as.groups;
-  if (splits > as.max_splits) splits = as.max_splits;
-  if (splits < 1) splits = 1;
-  int64_t chunk = (tokens + splits - 1) / splits;
-  chunk = (chunk + hadq::kAttnTile - 1) / hadq::kAttnTile * hadq::kAttnTile;
-  splits = (tokens + chunk - 1) / chunk;
-  size_t off_ml = 0, off_o = 0;
-  const size_t need = attn_ws_bytes(as.groups, int(splits), &off_ml, &off_o);
-  if (workspace_bytes < need)
-    return fail(HADQ_ERR_INVALID_ARG, "workspace of %zu bytes is below the %zu bytes needed", workspace_bytes,
-                need);
-
-  hadq::AttnArgs a{};
-  a.q = static_cast<const uint16_t*>(q);
-  a.k_codes = static_cast<const uint8_t*>(k_codes);
-  a.k_scales = k_scales;
-  a.v_codes = static_cast<const uint8_t*>(v_codes);
-  a.v_scales = v_scales;
-  a.signs = signs;
-  a.out = out;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.counters = reinterpret_cast<unsigned*>(ws);
-  a.part_ml = reinterpret_cast<float*>(ws + off_ml);
-  a.part_o = reinterpret_cast<float*>(ws + off_o);
-  a.tokens = tokens;
-  a.stride = token_stride;
-  a.chunk = chunk;
-  a.nqh = n_q_heads;
-  a.nkv = n_kv_heads;
-  a.g = n_q_heads / n_kv_heads;
-  a.hgroups = as.hgroups;
-  a.splits = int(splits);
-  a.qmul = (float)(double(softmax_scale) * 1.4426950408889634 / std::sqrt(double(hadq::kAttnDim)));
-  a.inv_sqrt_dim = (float)(1.0 / std::sqrt(double(hadq::kAttnDim)));
-  a.out_f32 = f32 ? 1 : 0;
-  a.vmask = 0x000F000Fu;
-  a.vmagic = 0x43084308u;
-  void* args[] = {&a};
-  cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(splits), unsigned(as.groups)), dim3(hadq::kAttnThreads),
-                                   args, 0, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return fail(HADQ_ERR_CUDA, "decode attention launch failed: %s", cudaGetErrorString(e));
-  }
-  return after_launch("decode attention kernel");
+hadq_status hadq_kv_decode_attention_noalloc(const void* q, const void* k_codes, const float* k_scales,
+                                             const void* v_codes, const float* v_scales, int32_t batch,
+                                             int32_t n_q_heads, int32_t n_kv_heads, int64_t tokens,
+                                             int64_t token_stride, int32_t dim, int32_t block,
+                                             const int8_t* signs, int32_t bits, int32_t group,
+                                             float softmax_scale, void* out, hadq_out_dtype out_dtype,
+                                             hadq_stream_t stream) {
+  g_last_error.clear();
+  return attn_call(q, k_codes, k_scales, v_codes, v_scales, batch, n_q_heads, n_kv_heads, tokens, token_stride,
+                   dim, block, signs, bits, group, softmax_scale, out, out_dtype, nullptr,
+                   hadq::kAttnStaticScratchBytes, true, stream);
 }
 
 const char* hadq_status_str(hadq_status st) {

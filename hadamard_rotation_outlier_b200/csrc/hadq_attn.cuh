@@ -54,6 +54,7 @@ constexpr int kAttnStS = kAttnStV + kAttnTile * kAttnVRow;      // 2304: 16 K sc
 constexpr int kAttnStageBytes = kAttnStS + 2 * kAttnTile * 4;   // 2432
 constexpr int kAttnCombPitch = kAttnDim + 4;                    // floats per head in the CTA merge
 constexpr int kAttnMaxSplits = 256;
+constexpr size_t kAttnStaticScratchBytes = size_t(16) << 20;  // scratch of the allocation-free entry
 constexpr float kAttnSlack = 8.0f;  // log2 units the running max may trail the true max
 
 struct AttnArgs {

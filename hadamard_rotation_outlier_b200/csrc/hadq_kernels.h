@@ -28,5 +28,8 @@ namespace hadq {
 // Decode attention over the rotated INT4 KV cache (head dim 128, one scale
 // per cached row), 128 threads per CTA.
 const void* kv_decode_attn_kernel_ptr();
+// Device address (current device) of the library's static attention scratch
+// of kAttnStaticScratchBytes, or NULL if the runtime cannot resolve it.
+void* attn_static_scratch();
 
 }  // namespace hadq

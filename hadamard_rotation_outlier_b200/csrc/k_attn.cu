@@ -6,4 +6,18 @@ namespace hadq {
 
 const void* kv_decode_attn_kernel_ptr() { return reinterpret_cast<const void*>(&kv_decode_attn_kernel<kAttnStages>); }
 
+// Scratch of the allocation-free entry point: a static device array, zero
+// when the module loads (so its arrival counters start at zero); every call
+// leaves the counters at zero again.
+__device__ __align__(256) unsigned char g_attn_scratch[kAttnStaticScratchBytes];
+
+void* attn_static_scratch() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return p;
+}
+
 }  // namespace hadq

@@ -182,6 +182,29 @@ hadq_status hadq_kv_decode_workspace_size(int32_t batch, int32_t n_q_heads, int3
                                           int64_t tokens, size_t *bytes);
 
 /*
+ * hadq_kv_decode_attention_noalloc -- hadq_kv_decode_attention without a
+ * caller workspace: the split partials and arrival counters live in a 16 MiB
+ * scratch array that the library holds as a static device variable (256-byte
+ * aligned, zero when the library loads, left at zero by every call).  Nothing
+ * is allocated per call.
+ *
+ *   Arguments, layouts and results as for hadq_kv_decode_attention.
+ *   Sizes whose partials exceed the scratch return HADQ_ERR_UNSUPPORTED
+ *   (use hadq_kv_decode_attention with a workspace then).
+ *   All calls in a process share the one scratch per device, so calls that
+ *   could overlap on the GPU (different streams, no synchronisation) must not
+ *   both use this entry point.
+ */
+hadq_status hadq_kv_decode_attention_noalloc(const void *q, const void *k_codes,
+                                             const float *k_scales, const void *v_codes,
+                                             const float *v_scales, int32_t batch,
+                                             int32_t n_q_heads, int32_t n_kv_heads,
+                                             int64_t tokens, int64_t token_stride, int32_t dim,
+                                             int32_t block, const int8_t *signs, int32_t bits,
+                                             int32_t group, float softmax_scale, void *out,
+                                             hadq_out_dtype out_dtype, hadq_stream_t stream);
+
+/*
  * hadq_plan -- host-only: validate the sizes of a call and report the kernel
  * family it would use.  direction 0 = rotate_quantize, 1 = dequant_rotate_inv.
  * `aligned16` says whether every pointer of the call is 16-byte aligned.

@@ -207,3 +207,19 @@ def test_decode_attention_empty_batch_is_a_noop(lib):
     n0 = B.hadq_launch_count()
     assert _attn(lib, batch=0, q=None, kc=None, ks=None, vc=None, vs=None, out=None, ws=None) == B.HADQ_OK
     assert B.hadq_launch_count() == n0
+
+
+def test_noalloc_entry_validates_before_launch(lib):
+    vp = ctypes.c_void_p
+    f = vp(0x10000)
+    n0 = B.hadq_launch_count()
+    call = lambda q, tokens, dim, block, group, bits: lib.hadq_kv_decode_attention_noalloc(
+        q, f, f, f, f, 1, 4, 1, tokens, 16, dim, block, None, bits, group, 0.1, f, B.HADQ_OUT_BF16, None)
+    assert call(f, 0, 128, 128, 128, 4) == B.HADQ_ERR_INVALID_ARG
+    assert call(f, 16, 64, 64, 64, 4) == B.HADQ_ERR_UNSUPPORTED
+    assert call(None, 16, 128, 128, 128, 4) == B.HADQ_ERR_INVALID_ARG
+    assert call(vp(0x10002), 16, 128, 128, 128, 4) == B.HADQ_ERR_MISALIGNED
+    assert B.hadq_launch_count() == n0
+    # batch 0 is an empty call with no pointers at all
+    assert lib.hadq_kv_decode_attention_noalloc(None, None, None, None, None, 0, 4, 1, 16, 16, 128, 128, None,
+                                                4, 128, 0.1, None, B.HADQ_OUT_BF16, None) == B.HADQ_OK
