@@ -72,27 +72,39 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# Device sources each kernel family is built from; a recorded DRAM traffic
+# figure stays valid while these files hash the same.
+KERNEL_SOURCES = {
+    "quant": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_blocked.cuh", "hadq_full4096.cuh",
+              "hadq_generic.cuh", "k_blocked.cu", "k_chunk.cu", "k_chunk_dq4.cu", "k_chunk_dq8.cu",
+              "k_full4096.cu", "k_generic.cu"],
+    "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
+}
+
+
+def kernel_source_hash(family: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "hadamard_rotation_outlier_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[family]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the quantise kernel from a committed ncu summary.
+def recorded_traffic(workload: str, family: str):
+    """DRAM bytes per launch of the workload's timed kernel from a committed ncu
+    summary.
 
     ``profiles/dram_traffic.txt`` holds lines ``workload source_hash bytes``;
-    the figure is used only while the kernel sources still hash the same.
+    the figure is used only while the kernel family's sources still hash the
+    same (see ``KERNEL_SOURCES``).
     """
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    h = kernel_source_hash()
+    h = kernel_source_hash(family)
     for ln in lines:
         parts = ln.split()
         if len(parts) == 3 and not ln.startswith("#") and parts[0] == workload and parts[1] == h:
@@ -392,7 +404,7 @@ def run_decode(args):
         "roofline": {
             "bound": "hbm", "kernel": "kv_decode_attn_kernel", "achieved": round(achieved, 1),
             "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)", "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(dw.name),
+            "frac": round(achieved / peak, 4), "traffic": recorded_traffic(dw.name, "attn"),
             "algorithmic_bytes_per_launch": nbytes, "avg_launch_ms": round(avg_ms, 5),
         },
         "e2e": {"value": round(world * nbytes * args.e2e_steps / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
@@ -481,7 +493,7 @@ def run_ours(args):
     q_bytes = wl.quant_bytes()
     q_ms = sum(quant_ms) / len(quant_ms)
     achieved = q_bytes / (q_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(wl.name)
+    traffic = recorded_traffic(wl.name, "quant")
     out = {
         "metric": METRIC,
         "value": round(value, 2),
