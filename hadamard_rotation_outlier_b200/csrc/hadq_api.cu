@@ -334,6 +334,8 @@ hadq_status attn_check(int32_t batch, int32_t nqh, int32_t nkv, int64_t tokens, 
   if (nqh % nkv)
     return fail(HADQ_ERR_INVALID_ARG, "n_q_heads %d is not a multiple of n_kv_heads %d", nqh, nkv);
   if (tokens < 1) return fail(HADQ_ERR_INVALID_ARG, "tokens must be >= 1 (got %lld)", (long long)tokens);
+  if (tokens > (int64_t(1) << 30))
+    return fail(HADQ_ERR_UNSUPPORTED, "tokens must be at most 2^30 (got %lld)", (long long)tokens);
   const int g = nqh / nkv;
   s->hgroups = (g + hadq::kAttnHeads - 1) / hadq::kAttnHeads;
   s->groups = int64_t(batch) * nkv * s->hgroups;
