@@ -148,7 +148,8 @@ hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int6
  *   batch        >= 0 (0 = empty call).
  *   n_q_heads    >= 1, a multiple of n_kv_heads; query head h reads KV head
  *                h / (n_q_heads / n_kv_heads) (grouped-query attention).
- *   tokens       cached tokens attended over, 1 <= tokens <= token_stride.
+ *   tokens       cached tokens attended over, 1 <= tokens <= token_stride,
+ *                at most 2^30 (HADQ_ERR_UNSUPPORTED beyond).
  *   dim, block,  the cache's rotate+quantise parameters; the kernel supports
  *   bits, group  dim 128, block 128 or -1, bits 4, group 128 or -1 and returns
  *                HADQ_ERR_UNSUPPORTED for any other valid combination.
