@@ -15,6 +15,8 @@ Page names used in citations:
 * [Outlier nemesis] -- "旋转量化：大模型低比特量化中的离群值克星", yfxerp.com.
 * [msModelSlim QuaRot] -- "QuaRot：基于旋转的离群值抑制算法说明",
   msmodelslim.readthedocs.io.
+* [HyQuant] -- "HyQuant:面向 LLM 注意力的混合精度量化" (HyQuant: mixed-precision
+  quantisation for LLM attention), ai-feeds.com.
 
 Readings taken where the pages are silent or ambiguous (each is also listed
 in the design notes of the repository):
@@ -52,6 +54,8 @@ __all__ = [
     "dequant_rotate_inv",
     "quant_error",
     "half_boundary_distance",
+    "rotate_quantize_keep",
+    "dequant_rotate_inv_keep",
     "dequant_rotated",
     "kv_decode_scores",
     "kv_decode_attention",
@@ -277,6 +281,61 @@ def dequant_rotate_inv(codes: np.ndarray, scales: np.ndarray, dim: int, block: i
     s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
     yhat = (q.reshape(q.shape[0], dim // G, G) * s[..., None]).reshape(q.shape)
     return inverse_rotate(yhat, block=block, signs=signs, method=method)
+
+
+def _kept_tokens(keep_slot, n_keep: int):
+    """(token, slot) pairs of the kept tokens: entries in [0, n_keep)."""
+    ks = np.asarray(keep_slot).astype(np.int64)
+    return [(t, int(v)) for t, v in enumerate(ks) if 0 <= v < n_keep]
+
+
+def rotate_quantize_keep(x_bits: np.ndarray, heads: int, tokens: int, keep_slot, n_keep: int,
+                         block: int = -1, signs=None, bits: int = 4, group: int = -1,
+                         method: str = "dense") -> dict:
+    """HyQuant-style mixed-precision KV quantisation of [heads * tokens, dim] rows.
+
+    [HyQuant] method, key modules: a small set of tokens (vertical-line
+    tokens, which carry most of the attention mass, and a local window) stays
+    in full precision and every other token is stored in low bit; the decode
+    stage applies that split to the KV cache.  [Hartmann rotation] §3 (the
+    first, "sink", tokens always matter) gives the other usual member of the
+    kept set.  Which tokens are kept is an input here.  Row
+    h * tokens + t belongs to head h and token t.  Token t is kept when
+    ``keep_slot[t]`` lies in [0, n_keep): its rows are copied unchanged into
+    ``kept[h, keep_slot[t]]`` (bf16 bits) and get codes 0 and scale 0.  Every
+    other row is rotated and quantised exactly as :func:`rotate_quantize`.
+    """
+    r = rotate_quantize(x_bits, block=block, signs=signs, bits=bits, group=group, method=method)
+    x = np.asarray(x_bits, dtype=np.uint16).reshape(heads * tokens, -1)
+    dim = x.shape[1]
+    codes, scales, q = r["codes"].copy(), r["scales"].copy(), r["q"].copy()
+    kept = np.zeros((heads, n_keep, dim), dtype=np.uint16)
+    keep_row = np.zeros(heads * tokens, dtype=bool)
+    for t, slot in _kept_tokens(keep_slot, n_keep):
+        for h in range(heads):
+            row = h * tokens + t
+            kept[h, slot] = x[row]
+            codes[row] = 0
+            scales[row] = 0.0
+            q[row] = 0
+            keep_row[row] = True
+    return {"codes": codes, "q": q, "scales": scales, "kept": kept, "keep_row": keep_row,
+            "rotated": r["rotated"], "pre_round": r["pre_round"], "scale64": r["scale64"]}
+
+
+def dequant_rotate_inv_keep(codes: np.ndarray, scales: np.ndarray, kept: np.ndarray, keep_slot,
+                            n_keep: int, heads: int, tokens: int, dim: int, block: int = -1,
+                            signs=None, bits: int = 4, group: int = -1,
+                            method: str = "dense") -> np.ndarray:
+    """Reads a mixed-precision cache back: kept tokens return their bf16 rows
+    exactly, every other row is dequantised and rotated back as
+    :func:`dequant_rotate_inv`.  Returns float64 [heads * tokens, dim]."""
+    out = dequant_rotate_inv(codes, scales, dim, block=block, signs=signs, bits=bits, group=group,
+                             method=method)
+    for t, slot in _kept_tokens(keep_slot, n_keep):
+        for h in range(heads):
+            out[h * tokens + t] = bf16_bits_to_f64(kept[h, slot])
+    return out
 
 
 def dequant_rotated(codes: np.ndarray, scales: np.ndarray, dim: int, bits: int = 4,

@@ -480,3 +480,70 @@ def test_decode_scores_equal_unrotated_dot_products():
     x = O.bf16_bits_to_f64(qbits)
     for h in range(nqh):
         np.testing.assert_allclose(got[0, h], 0.3 * K[0, h // 2] @ x[0, h], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------ mixed-precision (kept tokens) KV
+
+def _keep_case(heads=3, tokens=11, dim=64, seed=21):
+    x = S.random_bf16(heads * tokens, dim, seed, outlier_cols=[5], outlier_scale=30.0)
+    slots = np.full(tokens, -1, np.int32)
+    for rank, t in enumerate((0, 4, 9, 10)):        # a sink, a vertical line, a 2-token window
+        slots[t] = rank
+    return x, slots, 4
+
+
+def test_keep_nothing_equals_plain_quantisation():
+    x, _, _ = _keep_case()
+    slots = np.full(11, -1, np.int32)
+    r = O.rotate_quantize_keep(x, 3, 11, slots, 0, block=32, bits=4, group=16)
+    p = O.rotate_quantize(x, block=32, bits=4, group=16)
+    np.testing.assert_array_equal(r["codes"], p["codes"])
+    np.testing.assert_array_equal(r["scales"], p["scales"])
+    assert r["kept"].shape == (3, 0, 64)
+
+
+def test_kept_rows_are_copied_bit_exactly_and_zeroed():
+    x, slots, n_keep = _keep_case()
+    r = O.rotate_quantize_keep(x, 3, 11, slots, n_keep, block=-1, bits=4, group=-1)
+    p = O.rotate_quantize(x, block=-1, bits=4, group=-1)
+    for h in range(3):
+        for t in range(11):
+            row = h * 11 + t
+            if slots[t] >= 0:
+                np.testing.assert_array_equal(r["kept"][h, slots[t]], x[row])
+                assert not r["codes"][row].any() and r["scales"][row].item() == 0.0
+            else:
+                np.testing.assert_array_equal(r["codes"][row], p["codes"][row])
+                assert r["scales"][row].item() == p["scales"][row].item()
+    assert r["keep_row"].sum() == 3 * n_keep
+
+
+def test_slots_outside_the_range_mean_quantise():
+    x, slots, _ = _keep_case()
+    bad = slots.copy()
+    bad[4] = 4                       # n_keep = 4: out of range
+    bad[9] = -7
+    r = O.rotate_quantize_keep(x, 3, 11, bad, 4, bits=8)
+    p = O.rotate_quantize(x, bits=8)
+    for h in range(3):
+        for t in (4, 9):
+            np.testing.assert_array_equal(r["codes"][h * 11 + t], p["codes"][h * 11 + t])
+    assert not r["kept"][:, 1].any() and not r["kept"][:, 2].any()   # slots 1, 2 unused
+
+
+def test_mixed_cache_reads_back_kept_rows_exactly():
+    x, slots, n_keep = _keep_case()
+    signs = S.random_signs(64, 3)
+    r = O.rotate_quantize_keep(x, 3, 11, slots, n_keep, block=64, signs=signs, bits=4, group=32)
+    back = O.dequant_rotate_inv_keep(r["codes"], r["scales"], r["kept"], slots, n_keep, 3, 11, 64, block=64,
+                                     signs=signs, bits=4, group=32)
+    plain = O.dequant_rotate_inv(r["codes"], r["scales"], 64, block=64, signs=signs, bits=4, group=32)
+    xf = O.bf16_bits_to_f64(x)
+    for h in range(3):
+        for t in range(11):
+            row = h * 11 + t
+            want = xf[row] if slots[t] >= 0 else plain[row]
+            np.testing.assert_array_equal(back[row], want)
+    # the quantised rows still reconstruct within the INT4 error bound
+    q = ~r["keep_row"]
+    assert np.max(np.abs(back[q] - xf[q])) < 0.5 * np.max(r["scales"]) * 8
