@@ -554,9 +554,12 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
     h_codes = torch.empty(st.codes.shape, dtype=st.codes.dtype, pin_memory=True)
     h_scales = torch.empty(st.scales.shape, dtype=torch.float32, pin_memory=True)
     h_out = torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) if wl.dequant else None
+    h_kept = torch.empty(st.kept.shape, dtype=st.kept.dtype, pin_memory=True) if wl.keep else None
     streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
     rows = st.rows
     per = -(-rows // nchunks)
+    if wl.keep:  # kept-token calls take whole heads
+        per = -(-wl.heads // nchunks) * wl.tokens
     from hadamard_rotation_outlier_b200 import binding as B
 
     def one_step():
@@ -571,14 +574,29 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
             s.wait_event(ev0)
             with torch.cuda.stream(s):
                 st.x[r0:r1].copy_(st.x_host[r0:r1], non_blocking=True)
-                B.hadq_rotate_quantize(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
-                                       group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],
-                                       stream=s)
-                if wl.dequant:
-                    B.hadq_dequant_rotate_inv(st.codes[r0:r1], st.scales[r0:r1], wl.dim, block=wl.block,
-                                              signs=st.signs, bits=wl.bits, group=wl.group,
-                                              out=st.out[r0:r1], stream=s)
+                if wl.keep:
+                    h0, h1, t = r0 // wl.tokens, r1 // wl.tokens, wl.tokens
+                    B.hadq_rotate_quantize_keep(st.x[r0:r1].view(h1 - h0, t, wl.dim), st.keep_slot, wl.n_keep,
+                                                block=wl.block, signs=st.signs, bits=wl.bits, group=wl.group,
+                                                codes=st.codes[r0:r1].view(h1 - h0, t, -1),
+                                                scales=st.scales[r0:r1].view(h1 - h0, t, -1),
+                                                kept=st.kept[h0:h1], stream=s)
+                    B.hadq_dequant_rotate_inv_keep(st.codes[r0:r1].view(h1 - h0, t, -1),
+                                                   st.scales[r0:r1].view(h1 - h0, t, -1), st.kept[h0:h1],
+                                                   st.keep_slot, wl.n_keep, wl.dim, block=wl.block,
+                                                   signs=st.signs, bits=wl.bits, group=wl.group,
+                                                   out=st.out[r0:r1].view(h1 - h0, t, wl.dim), stream=s)
                     h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
+                    h_kept[h0:h1].copy_(st.kept[h0:h1], non_blocking=True)
+                else:
+                    B.hadq_rotate_quantize(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
+                                           group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],
+                                           stream=s)
+                    if wl.dequant:
+                        B.hadq_dequant_rotate_inv(st.codes[r0:r1], st.scales[r0:r1], wl.dim, block=wl.block,
+                                                  signs=st.signs, bits=wl.bits, group=wl.group,
+                                                  out=st.out[r0:r1], stream=s)
+                        h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
                 h_codes[r0:r1].copy_(st.codes[r0:r1], non_blocking=True)
                 h_scales[r0:r1].copy_(st.scales[r0:r1], non_blocking=True)
             e = torch.cuda.Event()
@@ -605,6 +623,8 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
     d2h = h_codes.numel() * h_codes.element_size() + h_scales.numel() * 4
     if h_out is not None:
         d2h += h_out.numel() * 2
+    if h_kept is not None:
+        d2h += h_kept.numel() * 2
     return {"value": round(world * st.bytes_per_step * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4), "chunks": nchunks}

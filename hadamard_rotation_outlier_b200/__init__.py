@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     MAX_DIM,
     HadqError,
     hadq_dequant_rotate_inv,
+    hadq_dequant_rotate_inv_keep,
     hadq_kv_decode_attention,
     hadq_kv_decode_attention_noalloc,
     hadq_kv_decode_workspace_size,
@@ -22,6 +23,8 @@ from .binding import (  # noqa: F401
     hadq_launch_count,
     hadq_plan,
     hadq_rotate_quantize,
+    hadq_rotate_quantize_keep,
+    hyquant_keep_slots,
     hadq_status_str,
     hadq_version,
     load_library,

@@ -22,7 +22,8 @@ HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
 PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
 MAX_DIM = 32768
 
-EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_kv_decode_attention",
+EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_keep",
+            "hadq_dequant_rotate_inv_keep", "hadq_kv_decode_attention",
             "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_status_str", "hadq_last_error",
             "hadq_launch_count", "hadq_version")
 
@@ -53,6 +54,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_dequant_rotate_inv.argtypes = [vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
                                             ctypes.c_int, vp]
     lib.hadq_dequant_rotate_inv.restype = ctypes.c_int
+    lib.hadq_rotate_quantize_keep.argtypes = [vp, c_i64, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, c_i32,
+                                              vp, vp, vp, vp]
+    lib.hadq_rotate_quantize_keep.restype = ctypes.c_int
+    lib.hadq_dequant_rotate_inv_keep.argtypes = [vp, vp, vp, vp, c_i32, c_i64, c_i64, c_i32, c_i32, vp, c_i32,
+                                                 c_i32, vp, ctypes.c_int, vp]
+    lib.hadq_dequant_rotate_inv_keep.restype = ctypes.c_int
     lib.hadq_kv_decode_attention.argtypes = [vp, vp, vp, vp, vp, c_i32, c_i32, c_i32, c_i64, c_i64,
                                              c_i32, c_i32, vp, c_i32, c_i32, ctypes.c_float, vp,
                                              ctypes.c_int, vp, ctypes.c_size_t, vp]
@@ -313,4 +320,99 @@ def hadq_kv_decode_attention_noalloc(q: torch.Tensor, k_codes: torch.Tensor, k_s
         _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), batch, nqh, nkv,
         stride if tokens is None else tokens, stride, dim, block, _ptr(signs), bits, group,
         float(softmax_scale), _ptr(out), code, _stream(stream)))
+    return out
+
+
+def hyquant_keep_slots(tokens: int, n_sink: int = 0, window: int = 0, vertical=()):
+    """Host helper: the keep table of a HyQuant-style token set.
+
+    Kept tokens are the first ``n_sink`` tokens, the last ``window`` tokens and
+    the ``vertical`` token indices; each gets its rank among the kept tokens
+    (ascending token order) as its slot.  Returns ``(keep_slot int32
+    [tokens] with -1 for quantised tokens, n_keep)``.
+    """
+    import numpy as np
+    kept = set(range(min(n_sink, tokens))) | set(range(max(0, tokens - window), tokens))
+    for t in vertical:
+        if not 0 <= int(t) < tokens:
+            raise ValueError(f"vertical token {t} outside [0, {tokens})")
+        kept.add(int(t))
+    slots = np.full(tokens, -1, dtype=np.int32)
+    for rank, t in enumerate(sorted(kept)):
+        slots[t] = rank
+    return slots, len(kept)
+
+
+def hadq_rotate_quantize_keep(x: torch.Tensor, keep_slot: torch.Tensor, n_keep: int, block: int = -1,
+                              signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                              kept: torch.Tensor | None = None, stream=None):
+    """Mixed-precision rotate+quantise of a bf16 ``[heads, tokens, dim]`` tensor.
+
+    ``keep_slot``: int32 CUDA tensor ``[tokens]``; token t is kept when
+    ``keep_slot[t]`` is in ``[0, n_keep)``.  Returns ``(codes, scales, kept)``
+    with ``kept`` bf16 ``[heads, n_keep, dim]``; kept rows get codes 0 and
+    scale 0.
+    """
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor [heads, tokens, dim]")
+    heads, tokens, dim = x.shape
+    dev = x.device
+    _need(keep_slot, "keep_slot", torch.int32, dev, tokens)
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(0, heads * tokens, dim, block, bits, group, 0, 1, None))
+    cdim = dim if bits == 8 else dim // 2
+    cdt = torch.int8 if bits == 8 else torch.uint8
+    if codes is None:
+        codes = torch.empty((heads, tokens, cdim), dtype=cdt, device=dev)
+    else:
+        _need(codes, "codes", cdt, dev, heads * tokens * cdim)
+    if scales is None:
+        scales = torch.empty((heads, tokens, dim // G), dtype=torch.float32, device=dev)
+    else:
+        _need(scales, "scales", torch.float32, dev, heads * tokens * (dim // G))
+    if kept is None:
+        kept = torch.empty((heads, n_keep, dim), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(kept, "kept", torch.bfloat16, dev, heads * n_keep * dim)
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    _check(lib.hadq_rotate_quantize_keep(_ptr(x), heads, tokens, dim, block, _ptr(signs), bits, group,
+                                         _ptr(keep_slot), n_keep, _ptr(codes), _ptr(scales),
+                                         _ptr(kept) if n_keep else None, _stream(stream)))
+    return codes, scales, kept
+
+
+def hadq_dequant_rotate_inv_keep(codes: torch.Tensor, scales: torch.Tensor, kept: torch.Tensor,
+                                 keep_slot: torch.Tensor, n_keep: int, dim: int, block: int = -1,
+                                 signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                                 out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                                 stream=None) -> torch.Tensor:
+    """Reads a mixed-precision cache back to ``[heads, tokens, dim]`` bf16 or
+    fp32: kept tokens return their stored bf16 rows exactly."""
+    lib = load_library()
+    if codes.dim() != 3 or not codes.is_cuda or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous CUDA tensor [heads, tokens, dim or dim/2]")
+    heads, tokens, _ = codes.shape
+    dev = codes.device
+    _need(keep_slot, "keep_slot", torch.int32, dev, tokens)
+    _need(kept, "kept", torch.bfloat16, dev, heads * n_keep * dim)
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(1, heads * tokens, dim, block, bits, group, 0, 1, None))
+    _need(scales, "scales", torch.float32, dev, heads * tokens * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        out = torch.empty((heads, tokens, dim), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev, heads * tokens * dim)
+    code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_dequant_rotate_inv_keep(_ptr(codes), _ptr(scales), _ptr(kept) if n_keep else None,
+                                            _ptr(keep_slot), n_keep, heads, tokens, dim, block, _ptr(signs),
+                                            bits, group, _ptr(out), code, _stream(stream)))
     return out

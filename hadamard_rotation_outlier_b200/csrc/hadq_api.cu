@@ -4,6 +4,7 @@
 // family, launches one kernel on the caller's stream and returns.  Nothing here allocates device memory and
 // nothing synchronises.
 #include <cmath>
+#include <cstdint>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -194,7 +195,11 @@ hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, b
 
 // ----------------------------------------------------------------- chunk
 
-hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool f32, cudaStream_t stream) {
+// `ka` carries the kept-token table when `keep`; the plain kernels read only
+// its ChunkArgs base (the first bytes of the struct).
+hadq_status launch_chunk_args(int direction, const Shape& s, hadq::ChunkKeepArgs ka, bool keep, bool f32,
+                              cudaStream_t stream) {
+  hadq::ChunkArgs& a = ka;
   a.cpr = s.dim / hadq::kCK;
   a.nchunks = s.rows * a.cpr;
   a.G = s.G;
@@ -205,8 +210,13 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   // that does not divide 32; the dequantiser needs no group reduction.
   const int team = (direction == 1 || (32 % a.gpc) == 0) ? 32 : hadq::kCT;
   a.slab_chunks = team == 32 ? 32 : (hadq::kCT / a.gpc) * a.gpc;  // a slab never splits a group
-  const void* fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK, team)
-                                  : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
+  const void* fn;
+  if (keep)  // kept tokens: groups of >= 128 columns on warp teams (checked by the caller)
+    fn = direction == 0 ? hadq::keep_chunk_kernel_ptr(s.bits, s.B, s.has_signs)
+                        : hadq::keep_dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, f32);
+  else
+    fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK, team)
+                        : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, direction == 0 && team != 32);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
@@ -218,7 +228,7 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   const int64_t teams = team == 32 ? hadq::kCT / 32 : 1;
   const int64_t want = ((a.nchunks + a.slab_chunks - 1) / a.slab_chunks + teams - 1) / teams;  // CTAs for one slab per team
   const unsigned grid = (unsigned)(want < cap ? want : cap);
-  void* args[] = {&a};
+  void* args[] = {&ka};
   e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -226,6 +236,12 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
     return fail(HADQ_ERR_CUDA, "chunk kernel launch failed: %s", cudaGetErrorString(e));
   }
   return after_launch("chunk kernel");
+}
+
+hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool f32, cudaStream_t stream) {
+  hadq::ChunkKeepArgs ka{};
+  static_cast<hadq::ChunkArgs&>(ka) = a;
+  return launch_chunk_args(direction, s, ka, false, f32, stream);
 }
 
 hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
@@ -635,6 +651,96 @@ hadq_status hadq_kv_decode_attention_noalloc(const void* q, const void* k_codes,
   return attn_call(q, k_codes, k_scales, v_codes, v_scales, batch, n_q_heads, n_kv_heads, tokens, token_stride,
                    dim, block, signs, bits, group, softmax_scale, out, out_dtype, nullptr,
                    hadq::kAttnStaticScratchBytes, true, stream);
+}
+
+// Mixed-precision (kept-token) variants: the chunk kernels with a keep table.
+static hadq_status keep_check(const Shape& s, int64_t heads, int64_t tokens, const int32_t* keep_slot,
+                              int32_t n_keep, const void* kept, bool a16) {
+  if (heads < 0 || tokens < 0)
+    return fail(HADQ_ERR_INVALID_ARG, "heads and tokens must be >= 0 (got %lld, %lld)", (long long)heads,
+                (long long)tokens);
+  if (n_keep < 0) return fail(HADQ_ERR_INVALID_ARG, "n_keep must be >= 0 (got %d)", n_keep);
+  if (s.rows == 0) return HADQ_OK;
+  if (!keep_slot) return fail(HADQ_ERR_INVALID_ARG, "keep_slot must not be NULL");
+  if (n_keep > 0 && !kept) return fail(HADQ_ERR_INVALID_ARG, "kept must not be NULL when n_keep > 0");
+  if (!aligned(keep_slot, 4)) return fail(HADQ_ERR_MISALIGNED, "keep_slot must be 4-byte aligned");
+  if (kept && !aligned(kept, 16)) return fail(HADQ_ERR_MISALIGNED, "kept must be 16-byte aligned");
+  const int gpc = s.G >= hadq::kCK ? s.G / hadq::kCK : 0;
+  if (!a16 || !chunk_ok(0, s) || s.G % hadq::kCK != 0 || 32 % gpc != 0 ||
+      s.rows * (s.dim / hadq::kCK) >= (int64_t(1) << 31))
+    return fail(HADQ_ERR_UNSUPPORTED,
+                "kept tokens need the chunk kernels with wide groups: dim a multiple of 128, block 8..128, "
+                "group 128 x (1, 2, 4, .., 32) columns, fewer than 2^31 chunks of 128, 16-byte-aligned buffers");
+  return HADQ_OK;
+}
+
+hadq_status hadq_rotate_quantize_keep(const void* x, int64_t heads, int64_t tokens, int32_t dim, int32_t block,
+                                      const int8_t* signs, int32_t bits, int32_t group, const int32_t* keep_slot,
+                                      int32_t n_keep, void* codes, float* scales, void* kept,
+                                      hadq_stream_t stream) {
+  g_last_error.clear();
+  if (heads < 0 || tokens < 0 || (tokens > 0 && heads > INT64_MAX / tokens))
+    return fail(HADQ_ERR_INVALID_ARG, "heads and tokens must be >= 0 (got %lld, %lld)", (long long)heads,
+                (long long)tokens);
+  Shape s;
+  hadq_status st = check_sizes(heads * tokens, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  s.has_signs = signs != nullptr;
+  if (s.rows > 0 && (!x || !codes || !scales))
+    return fail(HADQ_ERR_INVALID_ARG, "x, codes and scales must not be NULL");
+  if (s.rows > 0 && !aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  const bool a16 = aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16));
+  st = keep_check(s, heads, tokens, keep_slot, n_keep, kept, a16);
+  if (st != HADQ_OK || s.rows == 0) return st;
+  const double qmax = double((1 << (bits - 1)) - 1);
+  hadq::ChunkKeepArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.signs = signs;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.scale_mul = (float)(1.0 / (std::sqrt(double(s.B)) * qmax));
+  a.rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  a.keep_slot = keep_slot;
+  a.kept = static_cast<uint16_t*>(kept);
+  a.keep_tokens = tokens;
+  a.n_keep = n_keep;
+  return launch_chunk_args(0, s, a, true, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hadq_status hadq_dequant_rotate_inv_keep(const void* codes, const float* scales, const void* kept,
+                                         const int32_t* keep_slot, int32_t n_keep, int64_t heads, int64_t tokens,
+                                         int32_t dim, int32_t block, const int8_t* signs, int32_t bits,
+                                         int32_t group, void* out, hadq_out_dtype out_dtype,
+                                         hadq_stream_t stream) {
+  g_last_error.clear();
+  if (heads < 0 || tokens < 0 || (tokens > 0 && heads > INT64_MAX / tokens))
+    return fail(HADQ_ERR_INVALID_ARG, "heads and tokens must be >= 0 (got %lld, %lld)", (long long)heads,
+                (long long)tokens);
+  Shape s;
+  hadq_status st = check_sizes(heads * tokens, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
+    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
+  s.has_signs = signs != nullptr;
+  if (s.rows > 0 && (!codes || !scales || !out))
+    return fail(HADQ_ERR_INVALID_ARG, "codes, scales and out must not be NULL");
+  if (s.rows > 0 && !aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  const bool a16 = aligned(codes, 16) && aligned(out, 16) && (!signs || aligned(signs, 16));
+  st = keep_check(s, heads, tokens, keep_slot, n_keep, kept, a16);
+  if (st != HADQ_OK || s.rows == 0) return st;
+  const bool f32 = out_dtype == HADQ_OUT_F32;
+  hadq::ChunkKeepArgs a{};
+  a.codes_in = static_cast<const uint8_t*>(codes);
+  a.scales_in = scales;
+  a.signs = signs;
+  a.rot = f32 ? static_cast<float*>(out) : nullptr;
+  a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+  a.rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  a.keep_slot = keep_slot;
+  a.kept = static_cast<uint16_t*>(const_cast<void*>(kept));
+  a.keep_tokens = tokens;
+  a.n_keep = n_keep;
+  return launch_chunk_args(1, s, a, true, f32, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* hadq_status_str(hadq_status st) {

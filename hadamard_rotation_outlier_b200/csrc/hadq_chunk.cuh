@@ -25,6 +25,8 @@
 // one shared-memory max per slab (CTA team); a slab always holds whole groups.
 #pragma once
 
+#include <type_traits>
+
 #include "hadq_common.cuh"
 
 namespace hadq {
@@ -52,6 +54,36 @@ struct ChunkArgs {
   float scale_mul;
   float rsqrt_b;
 };
+
+// Arguments of the kept-token (mixed-precision) variants.  Rows are
+// [heads, keep_tokens]; token t is kept when keep_slot[t] is in [0, n_keep),
+// and its rows live as bf16 in kept[head][keep_slot[t]][dim].  The plain
+// kernels take the ChunkArgs base alone.
+struct ChunkKeepArgs : ChunkArgs {
+  const int32_t* keep_slot;
+  uint16_t* kept;
+  int64_t keep_tokens;
+  int n_keep;
+};
+template <bool KEEP>
+using ChunkArgsT = typename std::conditional<KEEP, ChunkKeepArgs, ChunkArgs>::type;
+
+// Keep-table entry of the token of chunk `ch` (kept-token calls have fewer
+// than 2^31 chunks).  Loaded one slab ahead of its use.
+__device__ __forceinline__ int kept_slot_of(const ChunkKeepArgs& a, int64_t ch) {
+  const uint32_t row = static_cast<uint32_t>(ch) / static_cast<uint32_t>(a.cpr);
+  return __ldg(a.keep_slot + row % static_cast<uint32_t>(a.keep_tokens));
+}
+
+// Element offset into `kept` of chunk `ch` whose token has keep-table entry
+// `s`, or -1 when the token is not kept.
+__device__ __forceinline__ int64_t kept_offset(const ChunkKeepArgs& a, int64_t ch, int s) {
+  if (s < 0 || s >= a.n_keep) return -1;
+  const uint32_t c32 = static_cast<uint32_t>(ch);
+  const uint32_t row = c32 / static_cast<uint32_t>(a.cpr);
+  const uint32_t head = row / static_cast<uint32_t>(a.keep_tokens);
+  return (int64_t(head) * a.n_keep + s) * a.dim + int64_t(c32 - row * uint32_t(a.cpr)) * kCK;
+}
 
 // Shared-memory layout shared by host and device:
 //   [two stages of kCT slots][sign table, sign bits (SIGNS)][group max (CTA teams)]
@@ -171,8 +203,10 @@ __device__ __forceinline__ void chunk_codes(const float (&v)[kCK], const float (
 // Forward: bf16 -> signs -> H_B (B = 2^LOG_B, 8..128) -> group max -> codes.
 // WIDE_G: the scale group covers whole chunks (G >= 128); otherwise 8 <= G < 128.
 // TEAM: 32 (warp teams; groups of at most 32 chunks, gpc dividing 32) or 128.
-template <int LOG_B, int BITS, bool SIGNS, bool WIDE_G, int TEAM>
-__global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
+// KEEP: rows of kept tokens (ChunkArgs.keep_slot) are copied out as bf16 and
+// get codes 0 and scale 0.
+template <int LOG_B, int BITS, bool SIGNS, bool WIDE_G, int TEAM, bool KEEP = false>
+__global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgsT<KEEP> a) {
   using T = Team<TEAM>;
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
@@ -204,19 +238,27 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
   uint8_t* st1 = T::stage(smem, 1);
 
   int64_t slab = T::first();
-  if (slab < nslabs)
+  int kslot_next = -1;  // KEEP: keep-table entry of this thread's chunk in the next slab
+  if (slab < nslabs) {
     chunk_load<16, TEAM>(xsrc + slab * a.slab_chunks * 256, slab_count(slab * a.slab_chunks, a.nchunks, a.slab_chunks), st0, tt);
+    if constexpr (KEEP)
+      if (slab * a.slab_chunks + tt < a.nchunks) kslot_next = kept_slot_of(a, slab * a.slab_chunks + tt);
+  }
   cp_async_commit();
   for (int it = 0; slab < nslabs; ++it, slab += T::stride()) {
     uint8_t* cur = (it & 1) ? st1 : st0;
     const int64_t c = slab * a.slab_chunks;
+    const int kslot = kslot_next;
     cp_async_wait<0>();
     T::sync();  // slab data visible; the other stage is free again
     {
       const int64_t nx = slab + T::stride();
-      if (nx < nslabs)
+      if (nx < nslabs) {
         chunk_load<16, TEAM>(xsrc + nx * a.slab_chunks * 256, slab_count(nx * a.slab_chunks, a.nchunks, a.slab_chunks),
                              (it & 1) ? st0 : st1, tt);
+        if constexpr (KEEP)
+          kslot_next = nx * a.slab_chunks + tt < a.nchunks ? kept_slot_of(a, nx * a.slab_chunks + tt) : -1;
+      }
       cp_async_commit();
     }
     const int nch = slab_count(c, a.nchunks, a.slab_chunks);
@@ -228,6 +270,17 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
       if (colc >= a.cpr) colc -= a.cpr;
     }
     uint8_t* mine = cur + tt * kCPad;
+    // kept row: its bf16 chunk is copied out unchanged; codes and scales are 0
+    bool kept_row = false;
+    if constexpr (KEEP) {
+      const int64_t kofs = active ? kept_offset(a, ch, kslot) : -1;
+      kept_row = kofs >= 0;
+      if (kept_row) {  // rare: a rolled loop keeps registers free
+        uint4* dst = reinterpret_cast<uint4*>(a.kept + kofs);
+#pragma unroll 1
+        for (int p = 0; p < 16; ++p) dst[p] = *reinterpret_cast<const uint4*>(mine + 16 * p);
+      }
+    }
 
     float v[kCK];
     float pm[16];
@@ -300,12 +353,13 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
     if (active) {
       // scale index = (flat element index of the group's first element) / G
       if constexpr (WIDE_G) {
-        if (glead) a.scales[multi ? slab * groups_per_slab + gslot : ch] = gmax * a.scale_mul;
+        if (glead) a.scales[multi ? slab * groups_per_slab + gslot : ch] = kept_row ? 0.0f : gmax * a.scale_mul;
       } else {
         const int lg = a.log_g;
 #pragma unroll
         for (int p = 0; p < 16; ++p)
-          if (((8 * p) & (G - 1)) == 0) a.scales[((ch * kCK) >> lg) + ((8 * p) >> lg)] = pm[p] * a.scale_mul;
+          if (((8 * p) & (G - 1)) == 0)
+            a.scales[((ch * kCK) >> lg) + ((8 * p) >> lg)] = kept_row ? 0.0f : pm[p] * a.scale_mul;
       }
       if (a.rot) {
         float4* dst = reinterpret_cast<float4*>(a.rot + ch * kCK);
@@ -340,7 +394,12 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
           }
         }
       }
-      chunk_codes<BITS>(v, inv, mine);
+      if (kept_row) {
+#pragma unroll
+        for (int p = 0; p < CB / 16; ++p) *reinterpret_cast<uint4*>(mine + 16 * p) = make_uint4(0, 0, 0, 0);
+      } else {
+        chunk_codes<BITS>(v, inv, mine);
+      }
     }
     T::sync();
     chunk_store<CB / 16, TEAM>(cur, nch, a.codes + c * CB, tt);
@@ -356,8 +415,9 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_kernel(ChunkArgs a) {
 // scale / sqrt(B).  Otherwise (G < B) the codes are scaled first.  With one
 // scale per chunk (G >= 128) the scale of the next slab is loaded one slab
 // ahead.
-template <int LOG_B, int BITS, bool SIGNS, bool SCALE_FIRST, bool OUT_F32>
-__global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
+// KEEP: rows of kept tokens return the bf16 values stored in ChunkArgs.kept.
+template <int LOG_B, int BITS, bool SIGNS, bool SCALE_FIRST, bool OUT_F32, bool KEEP = false>
+__global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgsT<KEEP> a) {
   using T = Team<32>;
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per chunk
   extern __shared__ __align__(16) uint8_t smem[];
@@ -380,16 +440,20 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
 
   int64_t slab = T::first();
   float sc_next = 0.0f;
+  int kslot_next = -1;  // KEEP: keep-table entry of this thread's chunk in the next slab
   if (slab < nslabs) {
     const int64_t c0 = slab * a.slab_chunks;
     chunk_load<CB / 16, 32>(a.codes_in + c0 * CB, slab_count(c0, a.nchunks, a.slab_chunks), st0, tt);
     if (one_scale && c0 + tt < a.nchunks) sc_next = chunk_scale(c0 + tt);
+    if constexpr (KEEP)
+      if (c0 + tt < a.nchunks) kslot_next = kept_slot_of(a, c0 + tt);
   }
   cp_async_commit();
   for (int it = 0; slab < nslabs; ++it, slab += T::stride()) {
     uint8_t* cur = (it & 1) ? st1 : st0;
     const int64_t c = slab * a.slab_chunks;
     const float sc_cur = sc_next;
+    const int kslot = kslot_next;
     cp_async_wait<0>();
     T::sync();
     {
@@ -398,6 +462,7 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
         const int64_t cn = nx * a.slab_chunks;
         chunk_load<CB / 16, 32>(a.codes_in + cn * CB, slab_count(cn, a.nchunks, a.slab_chunks), (it & 1) ? st0 : st1, tt);
         if (one_scale && cn + tt < a.nchunks) sc_next = chunk_scale(cn + tt);
+        if constexpr (KEEP) kslot_next = cn + tt < a.nchunks ? kept_slot_of(a, cn + tt) : -1;
       }
       cp_async_commit();
     }
@@ -520,6 +585,26 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_kernel(ChunkArgs a) {
             o[3] ^= m4.w;
           }
           *reinterpret_cast<uint4*>(mine + 16 * p) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      // kept row: the stored bf16 values replace the reconstruction
+      if constexpr (KEEP) {
+        const int64_t kofs = kept_offset(a, ch, kslot);
+        if (kofs >= 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.kept + kofs);
+#pragma unroll 1
+          for (int p = 0; p < 16; ++p) {
+            const uint4 r = __ldg(src + p);
+            if constexpr (OUT_F32) {
+              float* dst = a.rot + ch * kCK + 8 * p;
+              reinterpret_cast<float4*>(dst)[0] =
+                  make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+              reinterpret_cast<float4*>(dst)[1] =
+                  make_float4(bf16lo(r.z), bf16hi(r.z), bf16lo(r.w), bf16hi(r.w));
+            } else {
+              *reinterpret_cast<uint4*>(mine + 16 * p) = r;
+            }
+          }
         }
       }
     }

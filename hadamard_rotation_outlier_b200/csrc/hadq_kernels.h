@@ -16,6 +16,9 @@ const void* dq_chunk_kernel_ptr_4(int B, bool signs, bool scale_first, bool f32)
 inline const void* dq_chunk_kernel_ptr(int bits, int B, bool signs, bool scale_first, bool f32) {
   return bits == 8 ? dq_chunk_kernel_ptr_8(B, signs, scale_first, f32) : dq_chunk_kernel_ptr_4(B, signs, scale_first, f32);
 }
+// Kept-token variants (groups of >= 128 columns, warp teams).
+const void* keep_chunk_kernel_ptr(int bits, int B, bool signs);
+const void* keep_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
 // 4096-column blocks, one scale per block, one block per warp.
 const void* wide4096_kernel_ptr(int bits, bool signs);
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);

@@ -53,6 +53,15 @@ class WorkloadStep:
         self.scales = torch.empty((self.rows, dim // G), dtype=torch.float32, device=self.device)
         self.out = (torch.empty((self.rows, dim), dtype=torch.bfloat16, device=self.device)
                     if wl.dequant else None)
+        self.keep_slot = self.kept = None
+        if wl.keep:
+            n_sink, window, n_vertical = wl.keep
+            vert = S.vertical_tokens(wl.tokens, n_vertical, seed, n_sink, window)
+            slots, n_keep = B.hyquant_keep_slots(wl.tokens, n_sink, window, vert)
+            assert n_keep == wl.n_keep
+            self.keep_slot_host = slots
+            self.keep_slot = torch.from_numpy(slots).to(self.device)
+            self.kept = torch.empty((wl.heads, n_keep, dim), dtype=torch.bfloat16, device=self.device)
 
     @property
     def launches_per_step(self) -> int:
@@ -68,16 +77,30 @@ class WorkloadStep:
 
     def quantize(self, stream=None, rotated_out=None):
         wl = self.wl
+        if wl.keep:
+            h, t = wl.heads, wl.tokens
+            B.hadq_rotate_quantize_keep(self.x.view(h, t, wl.dim), self.keep_slot, wl.n_keep, block=wl.block,
+                                        signs=self.signs, bits=wl.bits, group=wl.group,
+                                        codes=self.codes.view(h, t, -1), scales=self.scales.view(h, t, -1),
+                                        kept=self.kept, stream=stream)
+            return
         B.hadq_rotate_quantize(self.x, block=wl.block, signs=self.signs, bits=wl.bits, group=wl.group,
                                codes=self.codes, scales=self.scales, rotated_out=rotated_out,
                                stream=stream)
 
     def dequantize(self, stream=None, out=None, out_dtype=torch.bfloat16):
         wl = self.wl
+        out = self.out if out is None else out
+        if wl.keep:
+            h, t = wl.heads, wl.tokens
+            return B.hadq_dequant_rotate_inv_keep(self.codes.view(h, t, -1), self.scales.view(h, t, -1),
+                                                  self.kept, self.keep_slot, wl.n_keep, wl.dim, block=wl.block,
+                                                  signs=self.signs, bits=wl.bits, group=wl.group,
+                                                  out=out.view(h, t, wl.dim), out_dtype=out_dtype,
+                                                  stream=stream)
         return B.hadq_dequant_rotate_inv(self.codes, self.scales, wl.dim, block=wl.block,
                                          signs=self.signs, bits=wl.bits, group=wl.group,
-                                         out=self.out if out is None else out, out_dtype=out_dtype,
-                                         stream=stream)
+                                         out=out, out_dtype=out_dtype, stream=stream)
 
     def step(self, stream=None):
         self.quantize(stream)

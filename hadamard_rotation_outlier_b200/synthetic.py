@@ -65,6 +65,10 @@ class Workload:
     dist: str           # "normal" or "student_t3"
     tensors: tuple
     dequant: bool = False
+    # kept tokens (mixed precision): (n_sink, window, n_vertical) or None.
+    # Rows are then [heads, tokens] over all tensors stacked (every tensor
+    # has the same tokens per head), and a token's rows are kept in all heads.
+    keep: tuple | None = None
 
     @property
     def rows(self) -> int:
@@ -77,17 +81,40 @@ class Workload:
     def scales_per_row(self) -> int:
         return self.dim // (self.dim if self.group == -1 else self.group)
 
+    @property
+    def heads(self) -> int:
+        return sum(t.heads for t in self.tensors)
+
+    @property
+    def tokens(self) -> int:
+        return self.tensors[0].rows // self.tensors[0].heads
+
+    @property
+    def n_keep(self) -> int:
+        if not self.keep:
+            return 0
+        n_sink, window, n_vertical = self.keep
+        return n_sink + window + n_vertical
+
     def quant_bytes(self) -> int:
-        """bf16 in + codes out + fp32 scales out, each byte moved once."""
+        """bf16 in + codes out + fp32 scales out, each byte moved once (plus,
+        with kept tokens, the int32 keep table in and the kept bf16 rows out)."""
         n = self.elements
         codes = n if self.bits == 8 else n // 2
-        return 2 * n + codes + 4 * self.rows * self.scales_per_row()
+        b = 2 * n + codes + 4 * self.rows * self.scales_per_row()
+        if self.keep:
+            b += 4 * self.tokens + 2 * self.heads * self.n_keep * self.dim
+        return b
 
     def dequant_bytes(self, out_bytes_per_elem: int = 2) -> int:
-        """codes + fp32 scales in + reconstructed values out."""
+        """codes + fp32 scales in + reconstructed values out (plus the keep
+        table and the kept bf16 rows in)."""
         n = self.elements
         codes = n if self.bits == 8 else n // 2
-        return codes + 4 * self.rows * self.scales_per_row() + out_bytes_per_elem * n
+        b = codes + 4 * self.rows * self.scales_per_row() + out_bytes_per_elem * n
+        if self.keep:
+            b += 4 * self.tokens + 2 * self.heads * self.n_keep * self.dim
+        return b
 
     def with_rows(self, rows_per_tensor: int) -> "Workload":
         """The same recipe with fewer rows per tensor (for oracle-sized tests).
@@ -129,6 +156,15 @@ WORKLOADS = {
         tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
                  Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
         dequant=True),
+    "c4k_kv_h8_t131072_d128_int4_g128_keep196": Workload(
+        name="c4k_kv_h8_t131072_d128_int4_g128_keep196",
+        description="the KV-cache workload with HyQuant-style mixed precision: 4 sink tokens, 64 "
+                    "seeded vertical-line tokens and a 128-token window stay bf16, the rest INT4; "
+                    "then read back (kept rows exact, the rest dequantised + inverse)",
+        dim=128, block=128, group=128, bits=4, with_signs=False, dist="normal",
+        tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
+                 Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
+        dequant=True, keep=(4, 128, 64)),
     "c5_tok32768_w11008_b128_signs_int4_g128": Workload(
         name="c5_tok32768_w11008_b128_signs_int4_g128",
         description="32768 tokens x 11008 (86 blocks of 128), Student-t(3); seeded signs, "
@@ -297,3 +333,11 @@ def random_int4_cache(batch: int, n_kv_heads: int, stride: int, dim: int, seed: 
     scales = rng.uniform(scale_range[0], scale_range[1],
                          size=(batch, n_kv_heads, stride)).astype(np.float32)
     return codes, scales
+
+
+def vertical_tokens(tokens: int, n: int, seed: int, skip_head: int = 0, skip_tail: int = 0) -> np.ndarray:
+    """Seeded distinct token indices standing in for vertical-line tokens,
+    drawn from [skip_head, tokens - skip_tail) and sorted."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x7E47, tokens, n]))
+    lo, hi = skip_head, tokens - skip_tail
+    return np.sort(rng.choice(np.arange(lo, hi), size=min(n, max(0, hi - lo)), replace=False))

@@ -123,6 +123,50 @@ hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int6
                                     hadq_out_dtype out_dtype, hadq_stream_t stream);
 
 /*
+ * hadq_rotate_quantize_keep -- mixed-precision KV quantisation: a few tokens
+ * stay in bf16, every other row is rotated and quantised as by
+ * hadq_rotate_quantize ("HyQuant: mixed-precision quantisation for LLM
+ * attention", method, key modules: vertical-line tokens and a local window
+ * stay in full precision, the rest goes to low bit; the decode stage applies
+ * the same split to the KV cache).
+ *
+ *   x          device bf16 [heads, tokens, dim]: row h * tokens + t.
+ *   keep_slot  device int32 [tokens]: token t is kept when keep_slot[t] lies
+ *              in [0, n_keep); any other value means "quantise".  Kept tokens
+ *              should have distinct slots (two tokens on one slot leave
+ *              either row there).  Which tokens to keep (sinks, vertical
+ *              lines, a window) is the caller's choice.
+ *   kept       device bf16 [heads, n_keep, dim] output, 16-byte aligned:
+ *              kept[h][keep_slot[t]] = x[h][t], bit for bit.  May be NULL
+ *              when n_keep == 0.
+ *   codes,     as for hadq_rotate_quantize; the rows of kept tokens get codes 0
+ *   scales     and scale 0.
+ *   Other arguments as for hadq_rotate_quantize.  Kernel coverage: dim a
+ *   multiple of 128 (at most 16384 when a group is wider than 128), block
+ *   8..128, group = 128 x (1, 2, 4, .., 32) columns (-1 for a row of that
+ *   width), fewer than 2^31 chunks of 128 columns, x, codes and signs
+ *   16-byte aligned; other valid combinations return HADQ_ERR_UNSUPPORTED.
+ */
+hadq_status hadq_rotate_quantize_keep(const void *x, int64_t heads, int64_t tokens, int32_t dim,
+                                      int32_t block, const int8_t *signs, int32_t bits,
+                                      int32_t group, const int32_t *keep_slot, int32_t n_keep,
+                                      void *codes, float *scales, void *kept,
+                                      hadq_stream_t stream);
+
+/*
+ * hadq_dequant_rotate_inv_keep -- reads a mixed-precision cache back: rows of
+ * kept tokens return their bf16 values from `kept` exactly (widened for
+ * float32 output), every other row is dequantised and rotated back as by
+ * hadq_dequant_rotate_inv.  Arguments as for hadq_rotate_quantize_keep and
+ * hadq_dequant_rotate_inv (out 16-byte aligned, same kernel coverage).
+ */
+hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales, const void *kept,
+                                         const int32_t *keep_slot, int32_t n_keep, int64_t heads,
+                                         int64_t tokens, int32_t dim, int32_t block,
+                                         const int8_t *signs, int32_t bits, int32_t group,
+                                         void *out, hadq_out_dtype out_dtype, hadq_stream_t stream);
+
+/*
  * hadq_kv_decode_attention -- one decode step of attention over a KV cache
  * stored in the rotated basis as INT4 codes.
  *

@@ -223,3 +223,52 @@ def test_noalloc_entry_validates_before_launch(lib):
     # batch 0 is an empty call with no pointers at all
     assert lib.hadq_kv_decode_attention_noalloc(None, None, None, None, None, 0, 4, 1, 16, 16, 128, 128, None,
                                                 4, 128, 0.1, None, B.HADQ_OUT_BF16, None) == B.HADQ_OK
+
+
+# ------------------------------------------------------------ kept tokens
+
+def _keep(lib, x=0x10000, heads=2, tokens=16, dim=128, block=128, signs=None, bits=4, group=128, slot=0x10000,
+          n_keep=2, codes=0x10000, scales=0x10000, kept=0x10000):
+    vp = ctypes.c_void_p
+    p = lambda v: None if v is None else vp(v)
+    return lib.hadq_rotate_quantize_keep(p(x), heads, tokens, dim, block, p(signs), bits, group, p(slot), n_keep,
+                                         p(codes), p(scales), p(kept), None)
+
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(slot=None), B.HADQ_ERR_INVALID_ARG, "keep_slot"),
+    (dict(kept=None), B.HADQ_ERR_INVALID_ARG, "kept"),
+    (dict(n_keep=-1), B.HADQ_ERR_INVALID_ARG, "n_keep"),
+    (dict(heads=-1), B.HADQ_ERR_INVALID_ARG, "heads"),
+    (dict(slot=0x10002), B.HADQ_ERR_MISALIGNED, "keep_slot"),
+    (dict(kept=0x10008), B.HADQ_ERR_MISALIGNED, "kept"),
+    (dict(group=32), B.HADQ_ERR_UNSUPPORTED, "wide groups"),
+    (dict(dim=96, block=32, group=96), B.HADQ_ERR_UNSUPPORTED, "wide groups"),
+    (dict(dim=128 * 48, block=128, group=128 * 48), B.HADQ_ERR_UNSUPPORTED, "wide groups"),
+    (dict(block=256, dim=256, group=256), B.HADQ_ERR_UNSUPPORTED, "wide groups"),
+    (dict(x=0x10008), B.HADQ_ERR_UNSUPPORTED, "16-byte"),
+    (dict(bits=5), B.HADQ_ERR_INVALID_ARG, "bits"),
+])
+def test_keep_entry_rejects_before_launch(lib, kw, status, msg):
+    n0 = B.hadq_launch_count()
+    assert _keep(lib, **kw) == status, B.hadq_last_error()
+    assert msg in B.hadq_last_error()
+    assert B.hadq_launch_count() == n0
+
+
+def test_keep_entries_empty_calls(lib):
+    n0 = B.hadq_launch_count()
+    assert _keep(lib, heads=0, x=None, slot=None, codes=None, scales=None, kept=None) == B.HADQ_OK
+    assert lib.hadq_dequant_rotate_inv_keep(None, None, None, None, 0, 3, 0, 128, 128, None, 4, 128, None,
+                                            B.HADQ_OUT_BF16, None) == B.HADQ_OK
+    assert B.hadq_launch_count() == n0
+
+
+def test_hyquant_keep_slots():
+    slots, n = B.hyquant_keep_slots(12, n_sink=2, window=3, vertical=[7, 1])
+    assert n == 6
+    assert slots.tolist() == [0, 1, -1, -1, -1, -1, -1, 2, -1, 3, 4, 5]
+    slots, n = B.hyquant_keep_slots(5, n_sink=9, window=9)
+    assert n == 5 and slots.tolist() == [0, 1, 2, 3, 4]
+    with pytest.raises(ValueError):
+        B.hyquant_keep_slots(5, vertical=[5])

@@ -41,6 +41,17 @@ def test_workload_byte_counts():
     assert wl["c4_kv_h8_t131072_d128_int4_g128"].quant_bytes() == 679_477_248
     assert wl["c4_kv_h8_t131072_d128_int4_g128"].dequant_bytes(2) == 679_477_248
     assert wl["c5_tok32768_w11008_b128_signs_int4_g128"].quant_bytes() == 913_047_552
+    # the mixed-precision variant adds the int32 keep table and 196 kept bf16 rows per head (16 heads)
+    k = wl["c4k_kv_h8_t131072_d128_int4_g128_keep196"]
+    assert (k.heads, k.tokens, k.n_keep) == (16, 131072, 196)
+    assert k.quant_bytes() == 679_477_248 + 4 * 131072 + 2 * 16 * 196 * 128
+    assert k.dequant_bytes(2) == k.quant_bytes()
+
+
+def test_vertical_tokens_seeded_and_in_range():
+    a = S.vertical_tokens(1000, 20, 3, 4, 100)
+    np.testing.assert_array_equal(a, S.vertical_tokens(1000, 20, 3, 4, 100))
+    assert len(set(a)) == 20 and a.min() >= 4 and a.max() < 900 and np.all(np.diff(a) > 0)
 
 
 def test_signs_are_pm1():

@@ -53,7 +53,11 @@ def test_full_workload_sampled_parity(name):
         lo = (codes & 0xF).to(torch.int16)
         hi = (codes >> 4).to(torch.int16)
         assert not torch.any(lo == 8) and not torch.any(hi == 8), "INT4 code -8 never produced"
-    assert torch.all(st.scales > 0), "these workloads have no all-zero group"
+    if wl.keep:  # rows of kept tokens have scale 0; every other row has none all-zero
+        quantised = torch.from_numpy(st.keep_slot_host < 0).to("cuda").repeat(wl.heads)
+        assert torch.all(st.scales[quantised] > 0) and not st.scales[~quantised].any()
+    else:
+        assert torch.all(st.scales > 0), "these workloads have no all-zero group"
     assert torch.isfinite(st.scales).all()
 
     rng = np.random.default_rng(zlib.crc32(name.encode()))
@@ -64,6 +68,25 @@ def test_full_workload_sampled_parity(name):
     x = np.stack([S.tensor_rows(wl, ti, r, r + 1)[0] for ti, r, _ in samples])
     np.testing.assert_array_equal(bf16_tensor_to_bits(st.x.index_select(0, idx)), x)
     signs = S.signs(wl)
+    if wl.keep:
+        # rows of kept tokens: codes 0, scale 0, the bf16 row in `kept` and in
+        # the read-back; the sampled rows of the other tokens follow below
+        rows = np.array([s[2] for s in samples])
+        heads_of, tok_of = rows // wl.tokens, rows % wl.tokens
+        slot = st.keep_slot_host[tok_of]
+        kept_s = slot >= 0
+        for extra in (0, wl.tokens - 1):     # a sink and a window token of every head
+            assert st.keep_slot_host[extra] >= 0
+        kept_rows = np.array([h * wl.tokens + t for h in range(wl.heads) for t in (0, wl.tokens - 1)])
+        kidx = torch.from_numpy(kept_rows).to("cuda")
+        kx = bf16_tensor_to_bits(st.x.index_select(0, kidx))
+        assert not codes.index_select(0, kidx).any() and not st.scales.index_select(0, kidx).any()
+        kb = bf16_tensor_to_bits(st.kept).reshape(wl.heads, wl.n_keep, dim)
+        np.testing.assert_array_equal(kb[kept_rows // wl.tokens, st.keep_slot_host[kept_rows % wl.tokens]], kx)
+        np.testing.assert_array_equal(bf16_tensor_to_bits(st.out.index_select(0, kidx)), kx)
+        keep_q = ~kept_s
+        x, g_codes, g_scales, idx = x[keep_q], g_codes[keep_q], g_scales[keep_q], idx[torch.from_numpy(keep_q).to("cuda")]
+        assert len(x) > 20
     ref = O.rotate_quantize(x, block=wl.block, signs=signs, bits=bits, group=wl.group)
     check_scales(g_scales, ref["scales"])
     check_codes(gpu_codes_to_int(g_codes, bits, dim), ref["q"], ref["pre_round"])
