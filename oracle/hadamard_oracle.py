@@ -54,6 +54,11 @@ __all__ = [
     "dequant_rotate_inv",
     "quant_error",
     "half_boundary_distance",
+    "quantize_asym",
+    "pack_uint4",
+    "unpack_uint4",
+    "rotate_quantize_asym",
+    "dequant_rotate_inv_asym",
     "rotate_quantize_keep",
     "dequant_rotate_inv_keep",
     "dequant_rotated",
@@ -280,6 +285,93 @@ def dequant_rotate_inv(codes: np.ndarray, scales: np.ndarray, dim: int, block: i
     G = _group_size(dim, group)
     s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
     yhat = (q.reshape(q.shape[0], dim // G, G) * s[..., None]).reshape(q.shape)
+    return inverse_rotate(yhat, block=block, signs=signs, method=method)
+
+
+def quantize_asym(y: np.ndarray, bits: int, group: int = -1):
+    """Asymmetric (zero-point) quantisation of the last axis, per group of G columns.
+
+    [Hartmann rotation] §2, the FakeQuantize forward: x_int = round(x / scale)
+    + zero_point, clamped to [0, 2^b - 1]; dequantised as (x_int - zero_point)
+    * scale.  The page takes scale and zero point as given (learned); here
+    they come from the group's range, which always holds 0 (reading):
+    lo = min(0, min y), hi = max(0, max y), scale = (hi - lo) / (2^b - 1),
+    zero_point = clamp(round(-lo / scale), 0, 2^b - 1).  Rounding is half to
+    even.  A group of zeros gets scale 0, zero point 0 and codes 0.
+
+    Returns ``(q, scale64, scale32, zp, v, zv)``: unsigned integer codes
+    (int64), the float64 scale, that scale rounded to float32 (stored), the
+    zero points (int64), the pre-round values v = y / scale64 and
+    zv = -lo / scale64.
+    """
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    y = np.asarray(y, dtype=np.float64)
+    dim = y.shape[-1]
+    G = _group_size(dim, group)
+    qmax = float(2 ** bits - 1)
+    yg = y.reshape(y.shape[:-1] + (dim // G, G))
+    lo = np.minimum(yg.min(axis=-1), 0.0)
+    hi = np.maximum(yg.max(axis=-1), 0.0)
+    scale64 = (hi - lo) / qmax
+    nz = scale64 > 0
+    safe = np.where(nz, scale64, 1.0)
+    zv = np.where(nz, -lo / safe, 0.0)
+    zp = np.clip(np.round(zv), 0, qmax).astype(np.int64)
+    v = np.where(nz[..., None], yg / safe[..., None], 0.0)
+    q = np.clip(np.round(v) + zp[..., None], 0, qmax).astype(np.int64)
+    q = np.where(nz[..., None], q, 0)
+    return (q.reshape(y.shape), scale64, scale64.astype(np.float32), zp, v.reshape(y.shape), zv)
+
+
+def pack_uint4(q: np.ndarray) -> np.ndarray:
+    """Two unsigned 4-bit codes (0..15) per byte; element 2j in the low nibble."""
+    q = np.asarray(q, dtype=np.int64)
+    if q.shape[-1] % 2:
+        raise ValueError("INT4 packing needs an even number of columns")
+    return ((q[..., 0::2] & 0xF) | ((q[..., 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def unpack_uint4(packed: np.ndarray) -> np.ndarray:
+    """Inverse of :func:`pack_uint4` (values 0..15, int64)."""
+    p = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = (p >> 4) & 0xF
+    return out
+
+
+def rotate_quantize_asym(x_bits: np.ndarray, block: int = -1, signs=None, bits: int = 4,
+                         group: int = -1, method: str = "dense") -> dict:
+    """The forward step with the asymmetric quantiser: decode bf16 -> signs ->
+    block Hadamard (as :func:`rotate_quantize`) -> :func:`quantize_asym` ->
+    unsigned codes (uint8 per element for INT8, two per byte for INT4).
+
+    Returns ``codes``, ``q``, ``scales`` (float32 [rows, dim/G]),
+    ``zero_points`` (uint8 [rows, dim/G]), ``scale64``, ``rotated``,
+    ``pre_round`` (y / scale64) and ``zp_pre_round`` (-lo / scale64).
+    """
+    x = bf16_bits_to_f64(x_bits)
+    y = rotate(x, block=block, signs=signs, method=method)
+    q, scale64, scale32, zp, v, zv = quantize_asym(y, bits, group)
+    codes = q.astype(np.uint8) if bits == 8 else pack_uint4(q)
+    return {"codes": codes, "q": q, "scales": scale32, "zero_points": zp.astype(np.uint8),
+            "scale64": scale64, "rotated": y, "pre_round": v, "zp_pre_round": zv}
+
+
+def dequant_rotate_inv_asym(codes: np.ndarray, scales: np.ndarray, zero_points: np.ndarray, dim: int,
+                            block: int = -1, signs=None, bits: int = 4, group: int = -1,
+                            method: str = "dense") -> np.ndarray:
+    """x_hat = (((q - zero_point) * scale) H_B) * s with the stored float32
+    scale ([Hartmann rotation] §2: (x_int - zero_point) * scale, then the
+    inverse rotation as :func:`dequant_rotate_inv`).  Returns float64
+    [rows, dim]."""
+    q = np.asarray(codes).astype(np.int64) if bits == 8 else unpack_uint4(codes)
+    q = q.reshape(-1, dim)
+    G = _group_size(dim, group)
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
+    z = np.asarray(zero_points).astype(np.int64).reshape(q.shape[0], dim // G)
+    yhat = ((q.reshape(q.shape[0], dim // G, G) - z[..., None]) * s[..., None]).reshape(q.shape)
     return inverse_rotate(yhat, block=block, signs=signs, method=method)
 
 

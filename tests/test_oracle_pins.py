@@ -547,3 +547,70 @@ def test_mixed_cache_reads_back_kept_rows_exactly():
     # the quantised rows still reconstruct within the INT4 error bound
     q = ~r["keep_row"]
     assert np.max(np.abs(back[q] - xf[q])) < 0.5 * np.max(r["scales"]) * 8
+
+
+# ------------------------------------------------------ asymmetric (zero-point) quantiser
+
+def test_asym_hand_worked_group():
+    # y = [-1, 0, 2, 3], 4 bits: lo = -1, hi = 3, scale = 4/15, zero point
+    # round(3.75) = 4; codes round([-3.75, 0, 7.5, 11.25]) + 4 = [0, 4, 12, 15]
+    # (7.5 rounds to the even 8).
+    q, s64, _, zp, _, _ = O.quantize_asym(np.array([[-1.0, 0.0, 2.0, 3.0]]), 4, -1)
+    assert s64[0] == 4 / 15 and zp[0] == 4
+    np.testing.assert_array_equal(q[0], [0, 4, 12, 15])
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_asym_closed_forms(bits):
+    qmax = 2 ** bits - 1
+    rng = np.random.default_rng(bits)
+    pos = np.abs(rng.normal(size=(3, 16))) + 0.1
+    q, s64, _, zp, _, _ = O.quantize_asym(pos, bits, -1)
+    assert np.all(zp == 0)                                    # all positive: lo = 0
+    np.testing.assert_array_equal(q.max(axis=1), qmax)        # the maximum maps to the top code
+    q, s64, _, zp, _, _ = O.quantize_asym(-pos, bits, -1)
+    assert np.all(zp == qmax)                                 # all negative: hi = 0
+    np.testing.assert_array_equal(q.min(axis=1), 0)
+    # zeros are exact, and a zero group gets scale 0, codes 0
+    y = np.concatenate([rng.normal(size=(2, 8)), np.zeros((2, 8))], axis=1)
+    y[:, 3] = 0.0
+    q, s64, s32, zp, _, _ = O.quantize_asym(y, bits, 8)
+    assert np.all(q[:, 3] == zp[:, 0]) and np.all(s64[:, 1] == 0) and np.all(q[:, 8:] == 0)
+
+
+@pytest.mark.parametrize("bits,G", [(4, 8), (4, 16), (8, 32)])
+def test_asym_codes_are_the_nearest_grid_points(bits, G):
+    # Brute force: the code is an argmin over all 2^b codes of |(k - zp) scale - y|.
+    rng = np.random.default_rng(40 + bits + G)
+    y = rng.standard_t(3, size=(6, 64))
+    q, s64, _, zp, _, _ = O.quantize_asym(y, bits, G)
+    k = np.arange(2 ** bits)
+    yg, qg = y.reshape(6, -1, G), q.reshape(6, -1, G)
+    for r in range(6):
+        for g in range(64 // G):
+            grid = (k - zp[r, g]) * s64[r, g]
+            d = np.abs(grid[None, :] - yg[r, g][:, None])
+            best = d.min(axis=1)
+            np.testing.assert_allclose(d[np.arange(G), qg[r, g]], best, rtol=0, atol=1e-12)
+            assert np.all(np.abs((qg[r, g] - zp[r, g]) * s64[r, g] - yg[r, g]) <= s64[r, g] / 2 + 1e-12)
+
+
+def test_asym_uint4_pack_roundtrip():
+    q = np.stack([np.arange(16), np.arange(16)[::-1]])
+    b = O.pack_uint4(q)
+    np.testing.assert_array_equal(O.unpack_uint4(b), q)
+    assert b[0, 0] == 0x10 and b[0, 7] == 0xFE and b[1, 0] == 0xEF
+
+
+def test_asym_rotate_quantize_and_back():
+    x = S.random_bf16(5, 256, 8, outlier_cols=[3, 200], outlier_scale=50.0)
+    signs = S.random_signs(256, 8)
+    r = O.rotate_quantize_asym(x, block=128, signs=signs, bits=4, group=64)
+    back = O.dequant_rotate_inv_asym(r["codes"], r["scales"], r["zero_points"], 256, block=128, signs=signs,
+                                     bits=4, group=64)
+    # error bound: each rotated value is off by at most scale/2, H orthonormal
+    yerr = (r["q"].reshape(5, 4, 64) - r["zero_points"][..., None].astype(np.int64)) * \
+        r["scales"][..., None].astype(np.float64) - r["rotated"].reshape(5, 4, 64)
+    assert np.all(np.abs(yerr) <= r["scales"][..., None] / 2 * (1 + 1e-6))
+    xf = O.bf16_bits_to_f64(x)
+    assert np.linalg.norm(back - xf, axis=1).max() <= np.linalg.norm(yerr.reshape(5, 256), axis=1).max() + 1e-9
