@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     MAX_DIM,
     HadqError,
     hadq_dequant_rotate_inv,
+    hadq_dequant_rotate_inv_asym,
     hadq_dequant_rotate_inv_keep,
     hadq_kv_decode_attention,
     hadq_kv_decode_attention_noalloc,
@@ -23,6 +24,7 @@ from .binding import (  # noqa: F401
     hadq_launch_count,
     hadq_plan,
     hadq_rotate_quantize,
+    hadq_rotate_quantize_asym,
     hadq_rotate_quantize_keep,
     hyquant_keep_slots,
     hadq_status_str,

@@ -22,7 +22,8 @@ HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
 PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
 MAX_DIM = 32768
 
-EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_keep",
+EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_asym",
+            "hadq_dequant_rotate_inv_asym", "hadq_rotate_quantize_keep",
             "hadq_dequant_rotate_inv_keep", "hadq_kv_decode_attention",
             "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_status_str", "hadq_last_error",
             "hadq_launch_count", "hadq_version")
@@ -54,6 +55,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_dequant_rotate_inv.argtypes = [vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
                                             ctypes.c_int, vp]
     lib.hadq_dequant_rotate_inv.restype = ctypes.c_int
+    lib.hadq_rotate_quantize_asym.argtypes = [vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, vp, vp, vp]
+    lib.hadq_rotate_quantize_asym.restype = ctypes.c_int
+    lib.hadq_dequant_rotate_inv_asym.argtypes = [vp, vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
+                                                 ctypes.c_int, vp]
+    lib.hadq_dequant_rotate_inv_asym.restype = ctypes.c_int
     lib.hadq_rotate_quantize_keep.argtypes = [vp, c_i64, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, c_i32,
                                               vp, vp, vp, vp]
     lib.hadq_rotate_quantize_keep.restype = ctypes.c_int
@@ -415,4 +421,76 @@ def hadq_dequant_rotate_inv_keep(codes: torch.Tensor, scales: torch.Tensor, kept
     _check(lib.hadq_dequant_rotate_inv_keep(_ptr(codes), _ptr(scales), _ptr(kept) if n_keep else None,
                                             _ptr(keep_slot), n_keep, heads, tokens, dim, block, _ptr(signs),
                                             bits, group, _ptr(out), code, _stream(stream)))
+    return out
+
+
+def hadq_rotate_quantize_asym(x: torch.Tensor, block: int = -1, signs: torch.Tensor | None = None,
+                              bits: int = 4, group: int = -1, codes: torch.Tensor | None = None,
+                              scales: torch.Tensor | None = None, zero_points: torch.Tensor | None = None,
+                              stream=None):
+    """Rotate, then quantise with a zero point (unsigned codes).
+
+    Returns ``(codes, scales, zero_points)``: uint8 ``[..., dim]`` (bits 8) or
+    ``[..., dim/2]`` (bits 4), float32 ``[..., dim/G]`` and uint8 ``[..., dim/G]``.
+    """
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    dim = x.shape[-1]
+    rows = x.numel() // dim if dim else 0
+    lead = tuple(x.shape[:-1])
+    dev = x.device
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(0, rows, dim, block, bits, group, 0, 1, None))
+    cdim = dim if bits == 8 else dim // 2
+    if codes is None:
+        codes = torch.empty(lead + (cdim,), dtype=torch.uint8, device=dev)
+    else:
+        _need(codes, "codes", torch.uint8, dev, rows * cdim)
+    if scales is None:
+        scales = torch.empty(lead + (dim // G,), dtype=torch.float32, device=dev)
+    else:
+        _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    if zero_points is None:
+        zero_points = torch.empty(lead + (dim // G,), dtype=torch.uint8, device=dev)
+    else:
+        _need(zero_points, "zero_points", torch.uint8, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    _check(lib.hadq_rotate_quantize_asym(_ptr(x), rows, dim, block, _ptr(signs), bits, group, _ptr(codes),
+                                         _ptr(scales), _ptr(zero_points), _stream(stream)))
+    return codes, scales, zero_points
+
+
+def hadq_dequant_rotate_inv_asym(codes: torch.Tensor, scales: torch.Tensor, zero_points: torch.Tensor,
+                                 dim: int, block: int = -1, signs: torch.Tensor | None = None,
+                                 bits: int = 4, group: int = -1, out: torch.Tensor | None = None,
+                                 out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """(codes - zero_point) * scale, then the inverse rotation; ``[..., dim]``."""
+    lib = load_library()
+    if not codes.is_cuda or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous CUDA tensor")
+    dev = codes.device
+    per_row = dim if bits == 8 else dim // 2
+    if per_row <= 0:
+        _check(lib.hadq_plan(1, 0, dim, block, bits, group, 0, 1, None))
+    rows = codes.numel() // per_row
+    lead = tuple(codes.shape[:-1]) if codes.shape[-1] == per_row else (rows,)
+    G = _resolve(dim, block, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(1, rows, dim, block, bits, group, 0, 1, None))
+    _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    _need(zero_points, "zero_points", torch.uint8, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        out = torch.empty(lead + (dim,), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev, rows * dim)
+    code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_dequant_rotate_inv_asym(_ptr(codes), _ptr(scales), _ptr(zero_points), rows, dim, block,
+                                            _ptr(signs), bits, group, _ptr(out), code, _stream(stream)))
     return out

@@ -14,6 +14,7 @@
 #include <unordered_map>
 
 #include "../../include/hadq.h"
+#include "hadq_asym.cuh"
 #include "hadq_attn.cuh"
 #include "hadq_blocked.cuh"
 #include "hadq_chunk.cuh"
@@ -741,6 +742,101 @@ hadq_status hadq_dequant_rotate_inv_keep(const void* codes, const float* scales,
   a.keep_tokens = tokens;
   a.n_keep = n_keep;
   return launch_chunk_args(1, s, a, true, f32, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Asymmetric (zero-point) variants: the chunk pipeline with range-derived
+// scale and zero point.
+static hadq_status asym_coverage(const Shape& s, bool a16) {
+  const int gpc = s.G >= hadq::kCK ? s.G / hadq::kCK : 0;
+  if (!a16 || s.B < 8 || s.B > hadq::kCK || s.dim % hadq::kCK != 0 || s.G % hadq::kCK != 0 || 32 % gpc != 0)
+    return fail(HADQ_ERR_UNSUPPORTED,
+                "the asymmetric quantiser needs dim a multiple of 128, block 8..128, group 128 x (1, 2, 4, .., "
+                "32) columns and 16-byte-aligned x/codes/out/signs");
+  return HADQ_OK;
+}
+
+static hadq_status launch_asym(int direction, const Shape& s, hadq::ChunkAsymArgs a, bool f32, cudaStream_t stream) {
+  a.cpr = s.dim / hadq::kCK;
+  a.nchunks = s.rows * a.cpr;
+  a.slab_chunks = 32;
+  a.G = s.G;
+  a.gpc = s.G / hadq::kCK;
+  a.dim = s.dim;
+  a.log_g = -1;
+  const void* fn = direction == 0 ? hadq::asym_chunk_kernel_ptr(s.bits, s.B, s.has_signs)
+                                  : hadq::asym_dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, f32);
+  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "asymmetric kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                cudaGetErrorString(e));
+  }
+  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab per warp
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  void* args[] = {&a};
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "asymmetric kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("asymmetric kernel");
+}
+
+hadq_status hadq_rotate_quantize_asym(const void* x, int64_t rows, int32_t dim, int32_t block, const int8_t* signs,
+                                      int32_t bits, int32_t group, void* codes, float* scales,
+                                      uint8_t* zero_points, hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = check_sizes(rows, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  s.has_signs = signs != nullptr;
+  if (rows == 0) return HADQ_OK;
+  if (!x || !codes || !scales || !zero_points)
+    return fail(HADQ_ERR_INVALID_ARG, "x, codes, scales and zero_points must not be NULL");
+  if (!aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  st = asym_coverage(s, aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)));
+  if (st != HADQ_OK) return st;
+  hadq::ChunkAsymArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.signs = signs;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.zp = zero_points;
+  a.scale_mul = (float)(1.0 / (std::sqrt(double(s.B)) * double((1 << bits) - 1)));
+  a.rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  return launch_asym(0, s, a, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hadq_status hadq_dequant_rotate_inv_asym(const void* codes, const float* scales, const uint8_t* zero_points,
+                                         int64_t rows, int32_t dim, int32_t block, const int8_t* signs,
+                                         int32_t bits, int32_t group, void* out, hadq_out_dtype out_dtype,
+                                         hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = check_sizes(rows, dim, block, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
+    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
+  s.has_signs = signs != nullptr;
+  if (rows == 0) return HADQ_OK;
+  if (!codes || !scales || !zero_points || !out)
+    return fail(HADQ_ERR_INVALID_ARG, "codes, scales, zero_points and out must not be NULL");
+  if (!aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "scales must be 4-byte aligned");
+  st = asym_coverage(s, aligned(codes, 16) && aligned(out, 16) && (!signs || aligned(signs, 16)));
+  if (st != HADQ_OK) return st;
+  const bool f32 = out_dtype == HADQ_OUT_F32;
+  hadq::ChunkAsymArgs a{};
+  a.codes_in = static_cast<const uint8_t*>(codes);
+  a.scales_in = scales;
+  a.zp_in = zero_points;
+  a.signs = signs;
+  a.rot = f32 ? static_cast<float*>(out) : nullptr;
+  a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+  a.rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
+  return launch_asym(1, s, a, f32, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* hadq_status_str(hadq_status st) {

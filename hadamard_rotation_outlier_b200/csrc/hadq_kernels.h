@@ -19,6 +19,9 @@ inline const void* dq_chunk_kernel_ptr(int bits, int B, bool signs, bool scale_f
 // Kept-token variants (groups of >= 128 columns, warp teams).
 const void* keep_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* keep_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
+// Asymmetric (zero-point) variants (groups of 128 x 2^k columns, warp teams).
+const void* asym_chunk_kernel_ptr(int bits, int B, bool signs);
+const void* asym_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
 // 4096-column blocks, one scale per block, one block per warp.
 const void* wide4096_kernel_ptr(int bits, bool signs);
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);

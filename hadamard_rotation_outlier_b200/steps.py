@@ -49,8 +49,12 @@ class WorkloadStep:
         G = dim if wl.group == -1 else wl.group
         cdim = dim if wl.bits == 8 else dim // 2
         cdt = torch.int8 if wl.bits == 8 else torch.uint8
+        if wl.asym:
+            cdt = torch.uint8
         self.codes = torch.empty((self.rows, cdim), dtype=cdt, device=self.device)
         self.scales = torch.empty((self.rows, dim // G), dtype=torch.float32, device=self.device)
+        self.zero_points = (torch.empty((self.rows, dim // G), dtype=torch.uint8, device=self.device)
+                            if wl.asym else None)
         self.out = (torch.empty((self.rows, dim), dtype=torch.bfloat16, device=self.device)
                     if wl.dequant else None)
         self.keep_slot = self.kept = None
@@ -77,6 +81,11 @@ class WorkloadStep:
 
     def quantize(self, stream=None, rotated_out=None):
         wl = self.wl
+        if wl.asym:
+            B.hadq_rotate_quantize_asym(self.x, block=wl.block, signs=self.signs, bits=wl.bits, group=wl.group,
+                                        codes=self.codes, scales=self.scales, zero_points=self.zero_points,
+                                        stream=stream)
+            return
         if wl.keep:
             h, t = wl.heads, wl.tokens
             B.hadq_rotate_quantize_keep(self.x.view(h, t, wl.dim), self.keep_slot, wl.n_keep, block=wl.block,
@@ -91,6 +100,10 @@ class WorkloadStep:
     def dequantize(self, stream=None, out=None, out_dtype=torch.bfloat16):
         wl = self.wl
         out = self.out if out is None else out
+        if wl.asym:
+            return B.hadq_dequant_rotate_inv_asym(self.codes, self.scales, self.zero_points, wl.dim,
+                                                  block=wl.block, signs=self.signs, bits=wl.bits, group=wl.group,
+                                                  out=out, out_dtype=out_dtype, stream=stream)
         if wl.keep:
             h, t = wl.heads, wl.tokens
             return B.hadq_dequant_rotate_inv_keep(self.codes.view(h, t, -1), self.scales.view(h, t, -1),

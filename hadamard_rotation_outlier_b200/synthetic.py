@@ -69,6 +69,8 @@ class Workload:
     # Rows are then [heads, tokens] over all tensors stacked (every tensor
     # has the same tokens per head), and a token's rows are kept in all heads.
     keep: tuple | None = None
+    # asymmetric (zero-point) quantiser: unsigned codes + one zero point per group
+    asym: bool = False
 
     @property
     def rows(self) -> int:
@@ -104,6 +106,8 @@ class Workload:
         b = 2 * n + codes + 4 * self.rows * self.scales_per_row()
         if self.keep:
             b += 4 * self.tokens + 2 * self.heads * self.n_keep * self.dim
+        if self.asym:
+            b += self.rows * self.scales_per_row()
         return b
 
     def dequant_bytes(self, out_bytes_per_elem: int = 2) -> int:
@@ -114,6 +118,8 @@ class Workload:
         b = codes + 4 * self.rows * self.scales_per_row() + out_bytes_per_elem * n
         if self.keep:
             b += 4 * self.tokens + 2 * self.heads * self.n_keep * self.dim
+        if self.asym:
+            b += self.rows * self.scales_per_row()
         return b
 
     def with_rows(self, rows_per_tensor: int) -> "Workload":
@@ -165,6 +171,14 @@ WORKLOADS = {
         tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
                  Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
         dequant=True, keep=(4, 128, 64)),
+    "c4a_kv_h8_t131072_d128_uint4_g128_asym": Workload(
+        name="c4a_kv_h8_t131072_d128_uint4_g128_asym",
+        description="the KV-cache workload with the asymmetric quantiser: unsigned INT4 codes, one "
+                    "fp32 scale and one uint8 zero point per 128-column group; then dequant + inverse",
+        dim=128, block=128, group=128, bits=4, with_signs=False, dist="normal",
+        tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
+                 Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
+        dequant=True, asym=True),
     "c5_tok32768_w11008_b128_signs_int4_g128": Workload(
         name="c5_tok32768_w11008_b128_signs_int4_g128",
         description="32768 tokens x 11008 (86 blocks of 128), Student-t(3); seeded signs, "

@@ -123,6 +123,43 @@ hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int6
                                     hadq_out_dtype out_dtype, hadq_stream_t stream);
 
 /*
+ * hadq_rotate_quantize_asym -- rotate, then quantise with a zero point
+ * ("Hartmann rotation, lightweight QAT, streaming attention", section 2, the
+ * FakeQuantize forward: x_int = round(x / scale) + zero_point, clamped to
+ * [0, 2^b - 1]).  Scale and zero point come from each group's range, which
+ * always holds 0:
+ *   lo = min(0, min y), hi = max(0, max y), scale = (hi - lo) / (2^b - 1),
+ *   zero_point = clamp(round(-lo / scale), 0, 2^b - 1),
+ *   q = clamp(round(y / scale) + zero_point, 0, 2^b - 1),
+ * rounding half to even; an all-zero group gets scale 0, zero point 0, codes 0.
+ *
+ *   codes        device output, unsigned: bits 8 -> uint8 [rows, dim]; bits 4
+ *                -> uint8 [rows, dim/2], element 2j in the low nibble, values
+ *                0..15.
+ *   scales       device output float32 [rows, dim/G].
+ *   zero_points  device output uint8 [rows, dim/G].
+ *   Other arguments as for hadq_rotate_quantize.  Kernel coverage: dim a
+ *   multiple of 128, block 8..128, group 128 x (1, 2, 4, .., 32) columns (-1
+ *   for rows of such a width), x, codes and signs 16-byte aligned; other valid
+ *   combinations return HADQ_ERR_UNSUPPORTED.
+ */
+hadq_status hadq_rotate_quantize_asym(const void *x, int64_t rows, int32_t dim, int32_t block,
+                                      const int8_t *signs, int32_t bits, int32_t group, void *codes,
+                                      float *scales, uint8_t *zero_points, hadq_stream_t stream);
+
+/*
+ * hadq_dequant_rotate_inv_asym -- x_hat = (((q - zero_point) * scale) H_B) * s
+ * for codes, scales and zero points written by hadq_rotate_quantize_asym (same
+ * dim, block, signs, bits, group).  Output as for hadq_dequant_rotate_inv
+ * (16-byte aligned); same kernel coverage as the forward call.
+ */
+hadq_status hadq_dequant_rotate_inv_asym(const void *codes, const float *scales,
+                                         const uint8_t *zero_points, int64_t rows, int32_t dim,
+                                         int32_t block, const int8_t *signs, int32_t bits,
+                                         int32_t group, void *out, hadq_out_dtype out_dtype,
+                                         hadq_stream_t stream);
+
+/*
  * hadq_rotate_quantize_keep -- mixed-precision KV quantisation: a few tokens
  * stay in bf16, every other row is rotated and quantised as by
  * hadq_rotate_quantize ("HyQuant: mixed-precision quantisation for LLM

@@ -14,6 +14,10 @@
   (round to nearest, ties to even), where the value's float32 error allowed
   above (1e-5 of max(|o|, row RMS)) is added to that ulp: a value near zero
   may carry an absolute float32 error several bf16 ulps wide.
+* Asymmetric quantiser: scales as above; a zero point may differ from the
+  oracle's by one only where the oracle's pre-round value -lo/scale lies
+  within 1e-4 of a .5 boundary; codes are then compared, under the code rule
+  above, with round(y/scale) plus the GPU's zero point, clamped.
 * Decode attention: the rule for float32 values above plus the conditioning
   of softmax on float32 scores.  A score s held in float32 (log2 units, after
   a few roundings) is off by at most 16 u |s| (u = 2^-24); a weight then moves
@@ -72,8 +76,9 @@ def check_scales(g: np.ndarray, o: np.ndarray) -> float:
     return float(rel.max()) if rel.size else 0.0
 
 
-def check_codes(g_q: np.ndarray, o_q: np.ndarray, pre_round: np.ndarray) -> int:
-    """Returns the number of (allowed) boundary mismatches."""
+def check_codes(g_q: np.ndarray, o_q: np.ndarray, pre_round: np.ndarray, max_mismatches=None) -> int:
+    """Returns the number of (allowed) boundary mismatches.  ``max_mismatches``
+    overrides the count limit for inputs built to sit on ties."""
     g_q = np.asarray(g_q).reshape(o_q.shape)
     mism = g_q != o_q
     n = int(mism.sum())
@@ -86,7 +91,7 @@ def check_codes(g_q: np.ndarray, o_q: np.ndarray, pre_round: np.ndarray) -> int:
                                  f"at {tuple(idx)} gpu {g_q[tuple(idx)]} oracle {o_q[tuple(idx)]} "
                                  f"pre-round {pre_round[tuple(idx)]!r}")
         assert np.all(np.abs(g_q[mism] - o_q[mism]) == 1)
-    allowed = max(1.0, MISMATCH_RATE * o_q.size)
+    allowed = max(1.0, MISMATCH_RATE * o_q.size) if max_mismatches is None else max_mismatches
     assert n <= allowed, f"codes: {n} boundary mismatches > {allowed:g} allowed"
     return n
 
@@ -177,3 +182,27 @@ def check_attention(g: np.ndarray, o: np.ndarray, allowance: np.ndarray, what: s
         raise AssertionError(f"{what}: {int(bad.sum())} values off; first at {i}: gpu {gv[i]!r} "
                              f"oracle {o[i]!r} allowance {allowance[i]:.3e}")
     return float(np.max(err / allowance)) if err.size else 0.0
+
+
+def check_asym(g_q: np.ndarray, g_scales: np.ndarray, g_zp: np.ndarray, ref: dict, bits: int,
+               max_mismatches=None) -> int:
+    """Asymmetric codes, scales and zero points against ``oracle.rotate_quantize_asym``.
+
+    ``g_q``: unpacked GPU codes [rows, dim] (int); ``g_scales``, ``g_zp``
+    [rows, dim/G].  Returns the number of tolerated code mismatches.
+    """
+    o_zp = ref["zero_points"].astype(np.int64).reshape(-1)
+    gz = np.asarray(g_zp).astype(np.int64).reshape(o_zp.shape)
+    check_scales(np.asarray(g_scales).reshape(ref["scales"].shape), ref["scales"])
+    mz = gz != o_zp
+    if np.any(mz):
+        d = O.half_boundary_distance(ref["zp_pre_round"].reshape(-1)[mz])
+        assert np.all(d <= BOUNDARY) and np.all(np.abs(gz[mz] - o_zp[mz]) == 1), "zero point mismatch"
+    v = ref["pre_round"]
+    rows, dim = v.shape
+    ngroups = ref["scales"].shape[-1]
+    G = dim // ngroups
+    zp_full = np.repeat(gz.reshape(rows, ngroups), G, axis=1)
+    nz = np.repeat(ref["scale64"].reshape(rows, ngroups) > 0, G, axis=1)
+    o_q = np.where(nz, np.clip(np.round(v) + zp_full, 0, 2 ** bits - 1), 0).astype(np.int64)
+    return check_codes(np.asarray(g_q).reshape(rows, dim), o_q, v, max_mismatches)

@@ -272,3 +272,33 @@ def test_hyquant_keep_slots():
     assert n == 5 and slots.tolist() == [0, 1, 2, 3, 4]
     with pytest.raises(ValueError):
         B.hyquant_keep_slots(5, vertical=[5])
+
+
+# ------------------------------------------------------------ asymmetric quantiser
+
+@pytest.mark.parametrize("kw,status,msg", [
+    (dict(zp=None), B.HADQ_ERR_INVALID_ARG, "NULL"),
+    (dict(group=64), B.HADQ_ERR_UNSUPPORTED, "asymmetric"),
+    (dict(dim=96, block=32, group=96), B.HADQ_ERR_UNSUPPORTED, "asymmetric"),
+    (dict(block=256, dim=256, group=256), B.HADQ_ERR_UNSUPPORTED, "asymmetric"),
+    (dict(x=0x10008), B.HADQ_ERR_UNSUPPORTED, "16-byte"),
+    (dict(scales=0x10002), B.HADQ_ERR_MISALIGNED, "scales"),
+    (dict(bits=3), B.HADQ_ERR_INVALID_ARG, "bits"),
+])
+def test_asym_entry_rejects_before_launch(lib, kw, status, msg):
+    vp = ctypes.c_void_p
+    a = dict(x=0x10000, rows=4, dim=128, block=128, bits=4, group=128, codes=0x10000, scales=0x10000, zp=0x10000)
+    a.update(kw)
+    p = lambda v: None if v is None else vp(v)
+    n0 = B.hadq_launch_count()
+    st = lib.hadq_rotate_quantize_asym(p(a["x"]), a["rows"], a["dim"], a["block"], None, a["bits"], a["group"],
+                                       p(a["codes"]), p(a["scales"]), p(a["zp"]), None)
+    assert st == status, B.hadq_last_error()
+    assert msg in B.hadq_last_error()
+    assert B.hadq_launch_count() == n0
+
+
+def test_asym_empty_calls(lib):
+    assert lib.hadq_rotate_quantize_asym(None, 0, 128, 128, None, 4, 128, None, None, None, None) == B.HADQ_OK
+    assert lib.hadq_dequant_rotate_inv_asym(None, None, None, 0, 128, 128, None, 4, 128, None, B.HADQ_OUT_F32,
+                                            None) == B.HADQ_OK

@@ -17,7 +17,7 @@ import oracle as O
 from hadamard_rotation_outlier_b200 import synthetic as S
 from hadamard_rotation_outlier_b200.steps import WorkloadStep, bf16_tensor_to_bits
 
-from parity import check_bf16, check_codes, check_scales, gpu_codes_to_int
+from parity import check_asym, check_bf16, check_codes, check_scales, gpu_codes_to_int
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
@@ -47,7 +47,9 @@ def test_full_workload_sampled_parity(name):
     qmax = 2 ** (bits - 1) - 1
     codes = st.codes
     # properties over every row: code range (INT8 is stored directly; INT4 nibbles)
-    if bits == 8:
+    if wl.asym:
+        pass  # unsigned codes: every value is in range
+    elif bits == 8:
         assert int(codes.min()) >= -qmax and int(codes.max()) <= qmax
     else:
         lo = (codes & 0xF).to(torch.int16)
@@ -87,6 +89,17 @@ def test_full_workload_sampled_parity(name):
         keep_q = ~kept_s
         x, g_codes, g_scales, idx = x[keep_q], g_codes[keep_q], g_scales[keep_q], idx[torch.from_numpy(keep_q).to("cuda")]
         assert len(x) > 20
+    if wl.asym:
+        ref = O.rotate_quantize_asym(x, block=wl.block, signs=signs, bits=bits, group=wl.group)
+        g_zp = st.zero_points.index_select(0, idx).cpu().numpy()
+        gq = g_codes.astype(np.int64) if bits == 8 else O.unpack_uint4(g_codes)
+        check_asym(gq, g_scales, g_zp, ref, bits)
+        rec = O.dequant_rotate_inv_asym(g_codes, g_scales, g_zp, dim, block=wl.block, signs=signs, bits=bits,
+                                        group=wl.group)
+        check_bf16(bf16_tensor_to_bits(st.out.index_select(0, idx)), rec, "asym dequant bf16")
+        del st
+        torch.cuda.empty_cache()
+        return
     ref = O.rotate_quantize(x, block=wl.block, signs=signs, bits=bits, group=wl.group)
     check_scales(g_scales, ref["scales"])
     check_codes(gpu_codes_to_int(g_codes, bits, dim), ref["q"], ref["pre_round"])
