@@ -54,6 +54,10 @@ __all__ = [
     "dequant_rotate_inv",
     "quant_error",
     "half_boundary_distance",
+    "kron_rotate",
+    "kron_inverse_rotate",
+    "rotate_quantize_kron",
+    "dequant_rotate_inv_kron",
     "quantize_asym",
     "pack_uint4",
     "unpack_uint4",
@@ -286,6 +290,66 @@ def dequant_rotate_inv(codes: np.ndarray, scales: np.ndarray, dim: int, block: i
     s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
     yhat = (q.reshape(q.shape[0], dim // G, G) * s[..., None]).reshape(q.shape)
     return inverse_rotate(yhat, block=block, signs=signs, method=method)
+
+
+def kron_rotate(x: np.ndarray, fa: np.ndarray, b: int, signs=None) -> np.ndarray:
+    """y = (F (x) H_b) (x * s) for rows of width a * b, float64.
+
+    [msModelSlim QuaRot], online rotation: down_proj is rotated online with a
+    Kronecker-product matrix, and dimensions without a Sylvester matrix take
+    stored Hadamard matrices (FAQ: add the matrix for the dimension).  F is
+    the a x a factor as it multiplies (e.g. a stored Hadamard matrix over
+    sqrt(a)); H_b is the normalised Sylvester matrix.  With the row viewed as
+    X[a, b] (element i * b + j), y = vec(F X H_b^T).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    fa = np.asarray(fa, dtype=np.float64)
+    a = fa.shape[0]
+    if fa.shape != (a, a) or x.shape[-1] != a * b:
+        raise ValueError("row width must be a * b with F of shape (a, a)")
+    if signs is not None:
+        x = x * np.where(np.asarray(signs) < 0, -1.0, 1.0)
+    X = x.reshape(x.shape[:-1] + (a, b))
+    Y = np.einsum("pi,...ij,qj->...pq", fa, X, sylvester(b))
+    return Y.reshape(x.shape)
+
+
+def kron_inverse_rotate(y: np.ndarray, fa: np.ndarray, b: int, signs=None) -> np.ndarray:
+    """x = (F^T (x) H_b) y, then the signs: the inverse of :func:`kron_rotate`
+    for an orthogonal F (H_b is symmetric and orthogonal)."""
+    y = np.asarray(y, dtype=np.float64)
+    fa = np.asarray(fa, dtype=np.float64)
+    a = fa.shape[0]
+    Y = y.reshape(y.shape[:-1] + (a, b))
+    X = np.einsum("ip,...ij,qj->...pq", fa, Y, sylvester(b))
+    x = X.reshape(y.shape)
+    if signs is not None:
+        x = x * np.where(np.asarray(signs) < 0, -1.0, 1.0)
+    return x
+
+
+def rotate_quantize_kron(x_bits: np.ndarray, fa: np.ndarray, b: int, signs=None, bits: int = 4,
+                         group: int = -1) -> dict:
+    """The forward step with the Kronecker rotation: decode bf16 ->
+    :func:`kron_rotate` -> symmetric absmax quantisation (:func:`quantize`) ->
+    codes, as :func:`rotate_quantize`."""
+    y = kron_rotate(bf16_bits_to_f64(x_bits), fa, b, signs)
+    q, scale64, scale32, v = quantize(y, bits, group)
+    codes = q.astype(np.int8) if bits == 8 else pack_int4(q)
+    return {"codes": codes, "q": q, "scales": scale32, "scale64": scale64, "rotated": y, "pre_round": v}
+
+
+def dequant_rotate_inv_kron(codes: np.ndarray, scales: np.ndarray, fa: np.ndarray, b: int, signs=None,
+                            bits: int = 4, group: int = -1) -> np.ndarray:
+    """q * scale with the stored float32 scale, then :func:`kron_inverse_rotate`."""
+    a = np.asarray(fa).shape[0]
+    dim = a * b
+    q = np.asarray(codes).astype(np.int64) if bits == 8 else unpack_int4(codes)
+    q = q.reshape(-1, dim)
+    G = _group_size(dim, group)
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64).reshape(q.shape[0], dim // G)
+    yhat = (q.reshape(q.shape[0], dim // G, G) * s[..., None]).reshape(q.shape)
+    return kron_inverse_rotate(yhat, fa, b, signs)
 
 
 def quantize_asym(y: np.ndarray, bits: int, group: int = -1):

@@ -614,3 +614,66 @@ def test_asym_rotate_quantize_and_back():
     assert np.all(np.abs(yerr) <= r["scales"][..., None] / 2 * (1 + 1e-6))
     xf = O.bf16_bits_to_f64(x)
     assert np.linalg.norm(back - xf, axis=1).max() <= np.linalg.norm(yerr.reshape(5, 256), axis=1).max() + 1e-9
+
+
+# -------------------------------------------------------------- Kronecker rotation
+
+def _paley_hadamard(q):
+    """Paley construction I (textbook): a Hadamard matrix of order q + 1 for a
+    prime q = 3 (mod 4), from the quadratic-residue character of GF(q)."""
+    res = {(i * i) % q for i in range(1, q)}
+    chi = lambda v: 0 if v % q == 0 else (1 if v % q in res else -1)
+    Q = np.array([[chi(j - i) for j in range(q)] for i in range(q)])
+    S = np.zeros((q + 1, q + 1), dtype=np.int64)
+    S[0, 1:] = 1
+    S[1:, 0] = -1
+    S[1:, 1:] = Q
+    return S + np.eye(q + 1, dtype=np.int64)
+
+
+@pytest.mark.parametrize("q", [3, 7, 11, 19])
+def test_paley_matrix_is_hadamard(q):
+    S = _paley_hadamard(q)
+    n = q + 1
+    assert set(np.unique(S)) == {-1, 1}
+    np.testing.assert_array_equal(S @ S.T, n * np.eye(n, dtype=np.int64))
+
+
+@pytest.mark.parametrize("a,b", [(1, 64), (2, 64), (4, 32), (8, 16)])
+def test_kron_of_sylvester_factors_is_the_sylvester_block(a, b):
+    # Sylvester H_a (x) H_b = H_ab (the Kronecker recursion): the Kronecker
+    # rotation with a Sylvester factor is the block rotation of size a * b.
+    x = S.random_bf16(3, a * b, a + b)
+    xf = O.bf16_bits_to_f64(x)
+    Fa = scipy.linalg.hadamard(a) / math.sqrt(a)
+    got = O.kron_rotate(xf, Fa, b)
+    want = xf @ (scipy.linalg.hadamard(a * b) / math.sqrt(a * b)).T
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_kron_matches_the_explicit_kronecker_matrix():
+    # vec(F X H^T) = (F (x) H) vec(X), checked against numpy's kron.
+    Fa = _paley_hadamard(11) / math.sqrt(12)
+    b = 16
+    x = S.random_bf16(4, 12 * b, 9, outlier_cols=[5], outlier_scale=40.0)
+    signs = S.random_signs(12 * b, 9)
+    xf = O.bf16_bits_to_f64(x)
+    M = np.kron(Fa, scipy.linalg.hadamard(b) / math.sqrt(b))
+    np.testing.assert_allclose(O.kron_rotate(xf, Fa, b, signs), (xf * np.where(signs < 0, -1, 1)) @ M.T,
+                               rtol=0, atol=1e-12)
+    y = O.kron_rotate(xf, Fa, b, signs)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(xf, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(O.kron_inverse_rotate(y, Fa, b, signs), xf, rtol=0, atol=1e-12)
+
+
+def test_kron_quantise_and_back():
+    Fa = _paley_hadamard(19) / math.sqrt(20)
+    x = S.random_bf16(5, 20 * 32, 3, outlier_cols=[7, 300], outlier_scale=80.0)
+    r = O.rotate_quantize_kron(x, Fa, 32, bits=4, group=32)
+    p = O.quantize(r["rotated"], 4, 32)
+    np.testing.assert_array_equal(r["q"], p[0])
+    back = O.dequant_rotate_inv_kron(r["codes"], r["scales"], Fa, 32, bits=4, group=32)
+    xf = O.bf16_bits_to_f64(x)
+    err = np.linalg.norm(back - xf, axis=1)
+    bound = np.sqrt(20 * 32) * 0.5 * r["scale64"].max(axis=1)
+    assert np.all(err <= bound)
