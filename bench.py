@@ -186,13 +186,31 @@ def oracle_sample_rate(wl, target_s: float, seed: int = 42):
     signs = S.signs(wl, seed)
     t0 = wl.tensors[0]
 
+    fa = None
+    if wl.kron_a:
+        fa = (S.paley_hadamard(wl.kron_a - 1).astype(np.float32) / np.float32(np.sqrt(wl.kron_a))).astype(np.float64)
+
     def run(nrows):
         x = S.tensor_rows(wl, 0, 0, nrows, seed)
         t = time.perf_counter()
-        r = O.rotate_quantize(x, block=wl.block, signs=signs, bits=wl.bits, group=wl.group)
-        if wl.dequant:
-            O.dequant_rotate_inv(r["codes"], r["scales"], wl.dim, block=wl.block, signs=signs,
-                                 bits=wl.bits, group=wl.group)
+        if wl.kron_a:
+            O.rotate_quantize_kron(x, fa, wl.dim // wl.kron_a, signs, wl.bits, wl.group)
+        elif wl.asym:
+            r = O.rotate_quantize_asym(x, block=wl.block, signs=signs, bits=wl.bits, group=wl.group)
+            O.dequant_rotate_inv_asym(r["codes"], r["scales"], r["zero_points"], wl.dim, block=wl.block,
+                                      signs=signs, bits=wl.bits, group=wl.group)
+        elif wl.keep:  # the sample's rows as one head of consecutive tokens, first n_sink kept
+            slots = np.full(nrows, -1, np.int32)
+            slots[:min(nrows, wl.keep[0])] = np.arange(min(nrows, wl.keep[0]))
+            r = O.rotate_quantize_keep(x, 1, nrows, slots, wl.keep[0], block=wl.block, signs=signs,
+                                       bits=wl.bits, group=wl.group)
+            O.dequant_rotate_inv_keep(r["codes"], r["scales"], r["kept"], slots, wl.keep[0], 1, nrows, wl.dim,
+                                      block=wl.block, signs=signs, bits=wl.bits, group=wl.group)
+        else:
+            r = O.rotate_quantize(x, block=wl.block, signs=signs, bits=wl.bits, group=wl.group)
+            if wl.dequant:
+                O.dequant_rotate_inv(r["codes"], r["scales"], wl.dim, block=wl.block, signs=signs,
+                                     bits=wl.bits, group=wl.group)
         return time.perf_counter() - t
 
     n = min(t0.rows, max(1, (1 << 20) // wl.dim))
@@ -517,8 +535,10 @@ def run_ours(args):
             "parallelism": f"dp{world} (independent rows, no collective)",
         },
         "roofline": {
-            "bound": "hbm", "kernel": KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits,
-                                                              wl.group, wl.with_signs, True)],
+            "bound": "hbm",
+            "kernel": ("rq_kron_kernel" if wl.kron_a else "rq_chunk_asym_kernel" if wl.asym else
+                       KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group,
+                                                wl.with_signs, True)]),
             "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
             "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
             "algorithmic_bytes_per_launch": q_bytes, "avg_launch_ms": round(q_ms, 5),
@@ -555,6 +575,7 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
     h_scales = torch.empty(st.scales.shape, dtype=torch.float32, pin_memory=True)
     h_out = torch.empty(st.out.shape, dtype=st.out.dtype, pin_memory=True) if wl.dequant else None
     h_kept = torch.empty(st.kept.shape, dtype=st.kept.dtype, pin_memory=True) if wl.keep else None
+    h_zp = torch.empty(st.zero_points.shape, dtype=torch.uint8, pin_memory=True) if wl.asym else None
     streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
     rows = st.rows
     per = -(-rows // nchunks)
@@ -588,6 +609,18 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
                                                    out=st.out[r0:r1].view(h1 - h0, t, wl.dim), stream=s)
                     h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
                     h_kept[h0:h1].copy_(st.kept[h0:h1], non_blocking=True)
+                elif wl.kron_a:
+                    B.hadq_rotate_quantize_kron(st.x[r0:r1], st.fa, wl.dim // wl.kron_a, signs=st.signs,
+                                                bits=wl.bits, group=wl.group, codes=st.codes[r0:r1],
+                                                scales=st.scales[r0:r1], stream=s)
+                elif wl.asym:
+                    B.hadq_rotate_quantize_asym(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
+                                                group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],
+                                                zero_points=st.zero_points[r0:r1], stream=s)
+                    B.hadq_dequant_rotate_inv_asym(st.codes[r0:r1], st.scales[r0:r1], st.zero_points[r0:r1],
+                                                   wl.dim, block=wl.block, signs=st.signs, bits=wl.bits,
+                                                   group=wl.group, out=st.out[r0:r1], stream=s)
+                    h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
                 else:
                     B.hadq_rotate_quantize(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
                                            group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],
@@ -599,6 +632,8 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
                         h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
                 h_codes[r0:r1].copy_(st.codes[r0:r1], non_blocking=True)
                 h_scales[r0:r1].copy_(st.scales[r0:r1], non_blocking=True)
+                if h_zp is not None:
+                    h_zp[r0:r1].copy_(st.zero_points[r0:r1], non_blocking=True)
             e = torch.cuda.Event()
             e.record(s)
             tails.append(e)
@@ -625,6 +660,8 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
         d2h += h_out.numel() * 2
     if h_kept is not None:
         d2h += h_kept.numel() * 2
+    if h_zp is not None:
+        d2h += h_zp.numel()
     return {"value": round(world * st.bytes_per_step * steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 4), "chunks": nchunks}
@@ -655,7 +692,7 @@ def run_reference(args):
     total_s = sum(i["seconds"] for i in infos)
     value = total_bytes / total_s / 1e9
     sample = (f"{steps} steps, each {infos[0]['rows']} rows of {wl.name} through the float64 "
-              f"oracle (numpy, dense Sylvester product)")
+              f"oracle (numpy, dense matrix products)")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": steps, "warmup": args.warmup,

@@ -16,6 +16,7 @@ from .binding import (  # noqa: F401
     HadqError,
     hadq_dequant_rotate_inv,
     hadq_dequant_rotate_inv_asym,
+    hadq_dequant_rotate_inv_kron,
     hadq_dequant_rotate_inv_keep,
     hadq_kv_decode_attention,
     hadq_kv_decode_attention_noalloc,
@@ -25,6 +26,7 @@ from .binding import (  # noqa: F401
     hadq_plan,
     hadq_rotate_quantize,
     hadq_rotate_quantize_asym,
+    hadq_rotate_quantize_kron,
     hadq_rotate_quantize_keep,
     hyquant_keep_slots,
     hadq_status_str,

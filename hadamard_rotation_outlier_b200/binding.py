@@ -22,7 +22,8 @@ HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
 PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
 MAX_DIM = 32768
 
-EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_asym",
+EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_kron",
+            "hadq_dequant_rotate_inv_kron", "hadq_rotate_quantize_asym",
             "hadq_dequant_rotate_inv_asym", "hadq_rotate_quantize_keep",
             "hadq_dequant_rotate_inv_keep", "hadq_kv_decode_attention",
             "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_status_str", "hadq_last_error",
@@ -55,6 +56,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_dequant_rotate_inv.argtypes = [vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
                                             ctypes.c_int, vp]
     lib.hadq_dequant_rotate_inv.restype = ctypes.c_int
+    lib.hadq_rotate_quantize_kron.argtypes = [vp, c_i64, c_i32, vp, c_i32, vp, c_i32, c_i32, vp, vp, vp, vp]
+    lib.hadq_rotate_quantize_kron.restype = ctypes.c_int
+    lib.hadq_dequant_rotate_inv_kron.argtypes = [vp, vp, c_i64, c_i32, vp, c_i32, vp, c_i32, c_i32, vp,
+                                                 ctypes.c_int, vp]
+    lib.hadq_dequant_rotate_inv_kron.restype = ctypes.c_int
     lib.hadq_rotate_quantize_asym.argtypes = [vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, vp, vp, vp]
     lib.hadq_rotate_quantize_asym.restype = ctypes.c_int
     lib.hadq_dequant_rotate_inv_asym.argtypes = [vp, vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
@@ -493,4 +499,79 @@ def hadq_dequant_rotate_inv_asym(codes: torch.Tensor, scales: torch.Tensor, zero
     code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
     _check(lib.hadq_dequant_rotate_inv_asym(_ptr(codes), _ptr(scales), _ptr(zero_points), rows, dim, block,
                                             _ptr(signs), bits, group, _ptr(out), code, _stream(stream)))
+    return out
+
+
+def hadq_rotate_quantize_kron(x: torch.Tensor, fa: torch.Tensor, b: int, signs: torch.Tensor | None = None,
+                              bits: int = 4, group: int = -1, codes: torch.Tensor | None = None,
+                              scales: torch.Tensor | None = None, rotated_out: torch.Tensor | None = None,
+                              stream=None):
+    """Kronecker rotation (F (x) H_b) then quantisation of a bf16 ``[..., a * b]``
+    tensor; ``fa``: float32 CUDA ``[a, a]`` (as it multiplies).  Returns
+    ``(codes, scales)`` as :func:`hadq_rotate_quantize`."""
+    lib = load_library()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    if fa.dim() != 2 or fa.shape[0] != fa.shape[1]:
+        raise ValueError("fa must be a square [a, a] matrix")
+    a = fa.shape[0]
+    dim = x.shape[-1]
+    if dim != a * b:
+        raise ValueError(f"rows of {dim} columns do not match a * b = {a * b}")
+    dev = x.device
+    _need(fa, "fa", torch.float32, dev)
+    rows = x.numel() // dim
+    lead = tuple(x.shape[:-1])
+    G = _resolve(dim, b, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(0, rows, dim, b, bits, group, 0, 1, None))
+    cshape = lead + ((dim,) if bits == 8 else (dim // 2,))
+    cdtype = torch.int8 if bits == 8 else torch.uint8
+    if codes is None:
+        codes = torch.empty(cshape, dtype=cdtype, device=dev)
+    else:
+        _need(codes, "codes", cdtype, dev, rows * cshape[-1])
+    if scales is None:
+        scales = torch.empty(lead + (dim // G,), dtype=torch.float32, device=dev)
+    else:
+        _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if rotated_out is not None:
+        _need(rotated_out, "rotated_out", torch.float32, dev, x.numel())
+    _check(lib.hadq_rotate_quantize_kron(_ptr(x), rows, a, _ptr(fa), b, _ptr(signs), bits, group, _ptr(codes),
+                                         _ptr(scales), _ptr(rotated_out), _stream(stream)))
+    return codes, scales
+
+
+def hadq_dequant_rotate_inv_kron(codes: torch.Tensor, scales: torch.Tensor, fa: torch.Tensor, b: int,
+                                 signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                                 out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                                 stream=None) -> torch.Tensor:
+    """Inverse of :func:`hadq_rotate_quantize_kron`: ``[..., a * b]`` bf16 or fp32."""
+    lib = load_library()
+    if not codes.is_cuda or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous CUDA tensor")
+    a = fa.shape[0]
+    dim = a * b
+    dev = codes.device
+    _need(fa, "fa", torch.float32, dev, a * a)
+    per_row = dim if bits == 8 else dim // 2
+    rows = codes.numel() // per_row
+    lead = tuple(codes.shape[:-1]) if codes.shape[-1] == per_row else (rows,)
+    G = _resolve(dim, b, group)
+    if G <= 0 or dim % G:
+        _check(lib.hadq_plan(1, rows, dim, b, bits, group, 0, 1, None))
+    _need(scales, "scales", torch.float32, dev, rows * (dim // G))
+    if signs is not None:
+        _need(signs, "signs", torch.int8, dev, dim)
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        out = torch.empty(lead + (dim,), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev, rows * dim)
+    code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
+    _check(lib.hadq_dequant_rotate_inv_kron(_ptr(codes), _ptr(scales), rows, a, _ptr(fa), b, _ptr(signs), bits,
+                                            group, _ptr(out), code, _stream(stream)))
     return out

@@ -20,6 +20,7 @@
 #include "hadq_chunk.cuh"
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
+#include "hadq_kron.cuh"
 #include "hadq_kernels.h"
 
 namespace {
@@ -837,6 +838,110 @@ hadq_status hadq_dequant_rotate_inv_asym(const void* codes, const float* scales,
   a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
   a.rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
   return launch_asym(1, s, a, f32, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Kronecker rotation F (x) H_b: sizes, pointers and the shared-memory budget.
+static hadq_status kron_check(int64_t rows, int32_t a, int32_t b, int32_t bits, int32_t group, Shape* s) {
+  if (a < 1 || a > 256) return fail(HADQ_ERR_INVALID_ARG, "a must be in [1, 256] (got %d)", a);
+  if (b < 2 || !is_pow2(b)) return fail(HADQ_ERR_INVALID_ARG, "b must be a power of two >= 2 (got %d)", b);
+  if (int64_t(a) * b > HADQ_MAX_DIM)
+    return fail(HADQ_ERR_INVALID_ARG, "a * b must be at most %d (got %lld)", HADQ_MAX_DIM, (long long)a * b);
+  hadq_status st = check_sizes(rows, a * b, b, bits, group, s);
+  if (st != HADQ_OK) return st;
+  if (hadq::kron_smem_bytes(a * b, a) > size_t(227) * 1024)
+    return fail(HADQ_ERR_UNSUPPORTED, "a * b = %d with a = %d needs %zu bytes of shared memory (227 KB max)",
+                a * b, a, hadq::kron_smem_bytes(a * b, a));
+  return HADQ_OK;
+}
+
+static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, bool f32, cudaStream_t stream) {
+  const void* fn = hadq::kron_kernel_ptr(direction, s.bits);
+  const size_t smem = hadq::kron_smem_bytes(s.dim, k.a);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "Kronecker kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                cudaGetErrorString(e));
+  }
+  const int64_t cap = int64_t(resident(fn, 256, smem)) * sm_count();
+  const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
+  if (direction == 0) {
+    void* args[] = {&k};
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+  } else {
+    bool out_f32 = f32;
+    void* args[] = {&k, &out_f32};
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "Kronecker kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("Kronecker kernel");
+}
+
+hadq_status hadq_rotate_quantize_kron(const void* x, int64_t rows, int32_t a, const float* fa, int32_t b,
+                                      const int8_t* signs, int32_t bits, int32_t group, void* codes, float* scales,
+                                      float* rotated_out, hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = kron_check(rows, a, b, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (rows == 0) return HADQ_OK;
+  if (!x || !fa || !codes || !scales)
+    return fail(HADQ_ERR_INVALID_ARG, "x, fa, codes and scales must not be NULL");
+  if (!aligned(x, 2)) return fail(HADQ_ERR_MISALIGNED, "x must be 2-byte aligned");
+  if (!aligned(fa, 4) || !aligned(scales, 4) || (rotated_out && !aligned(rotated_out, 4)))
+    return fail(HADQ_ERR_MISALIGNED, "fa, scales and rotated_out must be 4-byte aligned");
+  hadq::KronArgs k{};
+  k.g.x = static_cast<const uint16_t*>(x);
+  k.g.signs = signs;
+  k.g.codes = static_cast<uint8_t*>(codes);
+  k.g.scales = scales;
+  k.g.rot = rotated_out;
+  k.g.rows = rows;
+  k.g.dim = s.dim;
+  k.g.block = b;
+  k.g.group = s.G;
+  k.g.scale_mul = (float)(1.0 / (std::sqrt(double(b)) * double((1 << (bits - 1)) - 1)));
+  k.g.rsqrt_b = (float)(1.0 / std::sqrt(double(b)));
+  k.f = fa;
+  k.a = a;
+  k.ap = (a + hadq::kKronR - 1) / hadq::kKronR * hadq::kKronR;
+  return launch_kron(0, s, k, false, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales, int64_t rows, int32_t a,
+                                         const float* fa, int32_t b, const int8_t* signs, int32_t bits,
+                                         int32_t group, void* out, hadq_out_dtype out_dtype, hadq_stream_t stream) {
+  g_last_error.clear();
+  Shape s;
+  hadq_status st = kron_check(rows, a, b, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
+    return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
+  if (rows == 0) return HADQ_OK;
+  if (!codes || !scales || !fa || !out)
+    return fail(HADQ_ERR_INVALID_ARG, "codes, scales, fa and out must not be NULL");
+  const bool f32 = out_dtype == HADQ_OUT_F32;
+  if (!aligned(fa, 4) || !aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "fa and scales must be 4-byte aligned");
+  if (!aligned(out, f32 ? 4 : 2)) return fail(HADQ_ERR_MISALIGNED, "out must be aligned to its element size");
+  hadq::KronArgs k{};
+  k.g.codes_in = static_cast<const uint8_t*>(codes);
+  k.g.scales_in = scales;
+  k.g.signs = signs;
+  k.g.rot = f32 ? static_cast<float*>(out) : nullptr;
+  k.g.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+  k.g.rows = rows;
+  k.g.dim = s.dim;
+  k.g.block = b;
+  k.g.group = s.G;
+  k.g.rsqrt_b = (float)(1.0 / std::sqrt(double(b)));
+  k.f = fa;
+  k.a = a;
+  k.ap = (a + hadq::kKronR - 1) / hadq::kKronR * hadq::kKronR;
+  return launch_kron(1, s, k, f32, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* hadq_status_str(hadq_status st) {

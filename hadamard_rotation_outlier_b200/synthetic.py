@@ -71,6 +71,9 @@ class Workload:
     keep: tuple | None = None
     # asymmetric (zero-point) quantiser: unsigned codes + one zero point per group
     asym: bool = False
+    # Kronecker rotation (F (x) H_b) with a Paley factor of order kron_a
+    # (b = dim / kron_a); 0 for none
+    kron_a: int = 0
 
     @property
     def rows(self) -> int:
@@ -179,6 +182,13 @@ WORKLOADS = {
         tensors=(Tensor("k", 8 * 131072, 8, 4, 30.0, 4),
                  Tensor("v", 8 * 131072, 8, 0, 1.0, 5)),
         dequant=True, asym=True),
+    "c6_tok8192_d5120_kron20x256_int4_g128": Workload(
+        name="c6_tok8192_d5120_kron20x256_int4_g128",
+        description="8192 tokens x 5120 (no Sylvester matrix of that width), N(0,1) with 5 channels "
+                    "x100; seeded signs, Kronecker rotation (Paley H_20 / sqrt(20)) x (H_256); "
+                    "INT4 group 128",
+        dim=5120, block=256, group=128, bits=4, with_signs=True, dist="normal",
+        tensors=(Tensor("x", 8192, 1, 5, 100.0, 7),), kron_a=20),
     "c5_tok32768_w11008_b128_signs_int4_g128": Workload(
         name="c5_tok32768_w11008_b128_signs_int4_g128",
         description="32768 tokens x 11008 (86 blocks of 128), Student-t(3); seeded signs, "
@@ -355,3 +365,20 @@ def vertical_tokens(tokens: int, n: int, seed: int, skip_head: int = 0, skip_tai
     rng = np.random.default_rng(np.random.SeedSequence([seed, 0x7E47, tokens, n]))
     lo, hi = skip_head, tokens - skip_tail
     return np.sort(rng.choice(np.arange(lo, hi), size=min(n, max(0, hi - lo)), replace=False))
+
+
+def paley_hadamard(q: int) -> np.ndarray:
+    """A +-1 Hadamard matrix of order q + 1 for a prime q = 3 (mod 4), by the
+    Paley construction (quadratic residues of GF(q)); int8 [q + 1, q + 1].
+
+    Stands in for the stored Hadamard matrices that widths without a
+    Sylvester matrix need (those files are not available here).
+    """
+    res = {(i * i) % q for i in range(1, q)}
+    chi = np.array([0] + [1 if v in res else -1 for v in range(1, q)], dtype=np.int64)
+    idx = (np.arange(q)[None, :] - np.arange(q)[:, None]) % q
+    S = np.zeros((q + 1, q + 1), dtype=np.int64)
+    S[0, 1:] = 1
+    S[1:, 0] = -1
+    S[1:, 1:] = chi[idx]
+    return (S + np.eye(q + 1, dtype=np.int64)).astype(np.int8)

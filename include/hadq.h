@@ -123,6 +123,41 @@ hadq_status hadq_dequant_rotate_inv(const void *codes, const float *scales, int6
                                     hadq_out_dtype out_dtype, hadq_stream_t stream);
 
 /*
+ * hadq_rotate_quantize_kron -- Kronecker rotation + quantisation for widths
+ * a * b without a Sylvester matrix of their own: y = (F (x) H_b)(x * s), then
+ * the symmetric quantiser of hadq_rotate_quantize.  QuaRot's online down_proj
+ * rotation uses such a Kronecker-product matrix, and widths without a
+ * Sylvester matrix take a stored Hadamard matrix ("QuaRot: rotation-based
+ * outlier suppression", msModelSlim, online rotation and FAQ).
+ *
+ *   x     device bf16 [rows, a * b]; element i * b + j of a row is X[i][j].
+ *   a     1..256; fa: device float32 [a][a], row-major, the factor exactly as
+ *         it multiplies (for a stored +-1 Hadamard matrix S_a: S_a / sqrt(a);
+ *         any orthogonal matrix gives a rotation).  y = vec(F X H_b^T).
+ *   b     power of two >= 2; H_b is the normalised Sylvester matrix.
+ *   signs, bits, group, codes, scales, rotated_out: as for
+ *         hadq_rotate_quantize with dim = a * b (group divides a * b).
+ *   Shared memory grows with a * b and a^2: combinations above 227 KB
+ *   (about a * b > 24000 for small a) return HADQ_ERR_UNSUPPORTED.
+ */
+hadq_status hadq_rotate_quantize_kron(const void *x, int64_t rows, int32_t a, const float *fa,
+                                      int32_t b, const int8_t *signs, int32_t bits, int32_t group,
+                                      void *codes, float *scales, float *rotated_out,
+                                      hadq_stream_t stream);
+
+/*
+ * hadq_dequant_rotate_inv_kron -- x_hat = ((F^T (x) H_b)(q * scale)) * s, the
+ * inverse for an orthogonal F, with the codes and scales of
+ * hadq_rotate_quantize_kron (same a, fa, b, signs, bits, group).  Output as
+ * for hadq_dequant_rotate_inv.
+ */
+hadq_status hadq_dequant_rotate_inv_kron(const void *codes, const float *scales, int64_t rows,
+                                         int32_t a, const float *fa, int32_t b,
+                                         const int8_t *signs, int32_t bits, int32_t group,
+                                         void *out, hadq_out_dtype out_dtype,
+                                         hadq_stream_t stream);
+
+/*
  * hadq_rotate_quantize_asym -- rotate, then quantise with a zero point
  * ("Hartmann rotation, lightweight QAT, streaming attention", section 2, the
  * FakeQuantize forward: x_int = round(x / scale) + zero_point, clamped to

@@ -310,7 +310,7 @@ def kron_rotate(x: np.ndarray, fa: np.ndarray, b: int, signs=None) -> np.ndarray
     if signs is not None:
         x = x * np.where(np.asarray(signs) < 0, -1.0, 1.0)
     X = x.reshape(x.shape[:-1] + (a, b))
-    Y = np.einsum("pi,...ij,qj->...pq", fa, X, sylvester(b))
+    Y = fa @ X @ sylvester(b).T
     return Y.reshape(x.shape)
 
 
@@ -321,7 +321,7 @@ def kron_inverse_rotate(y: np.ndarray, fa: np.ndarray, b: int, signs=None) -> np
     fa = np.asarray(fa, dtype=np.float64)
     a = fa.shape[0]
     Y = y.reshape(y.shape[:-1] + (a, b))
-    X = np.einsum("ip,...ij,qj->...pq", fa, Y, sylvester(b))
+    X = fa.T @ Y @ sylvester(b).T
     x = X.reshape(y.shape)
     if signs is not None:
         x = x * np.where(np.asarray(signs) < 0, -1.0, 1.0)

@@ -302,3 +302,24 @@ def test_asym_empty_calls(lib):
     assert lib.hadq_rotate_quantize_asym(None, 0, 128, 128, None, 4, 128, None, None, None, None) == B.HADQ_OK
     assert lib.hadq_dequant_rotate_inv_asym(None, None, None, 0, 128, 128, None, 4, 128, None, B.HADQ_OUT_F32,
                                             None) == B.HADQ_OK
+
+
+# ------------------------------------------------------------ Kronecker rotation
+
+@pytest.mark.parametrize("a,b,bits,group,status,msg", [
+    (0, 64, 4, -1, B.HADQ_ERR_INVALID_ARG, "a must be"),
+    (300, 64, 4, -1, B.HADQ_ERR_INVALID_ARG, "a must be"),
+    (12, 48, 4, -1, B.HADQ_ERR_INVALID_ARG, "power of two"),
+    (12, 1, 8, -1, B.HADQ_ERR_INVALID_ARG, "power of two"),
+    (200, 256, 4, -1, B.HADQ_ERR_INVALID_ARG, "at most"),
+    (12, 64, 4, 7, B.HADQ_ERR_INVALID_ARG, "does not divide"),
+    (255, 128, 4, -1, B.HADQ_ERR_UNSUPPORTED, "shared memory"),
+])
+def test_kron_entry_validates(lib, a, b, bits, group, status, msg):
+    vp = ctypes.c_void_p
+    f = vp(0x10000)
+    n0 = B.hadq_launch_count()
+    st = lib.hadq_rotate_quantize_kron(f, 4, a, f, b, None, bits, group, f, f, None, None)
+    assert st == status, B.hadq_last_error()
+    assert msg in B.hadq_last_error()
+    assert B.hadq_launch_count() == n0
