@@ -79,7 +79,15 @@ KERNEL_SOURCES = {
               "hadq_generic.cuh", "k_blocked.cu", "k_chunk.cu", "k_chunk_dq4.cu", "k_chunk_dq8.cu",
               "k_full4096.cu", "k_generic.cu"],
     "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
+    "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
+    "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
+    "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_kron.cuh", "k_kron.cu"],
 }
+
+
+def workload_family(wl) -> str:
+    """Kernel family whose sources a workload's timed kernel is built from."""
+    return "kron" if wl.kron_a else "asym" if wl.asym else "keep" if wl.keep else "quant"
 
 
 def kernel_source_hash(family: str) -> str:
@@ -511,7 +519,7 @@ def run_ours(args):
     q_bytes = wl.quant_bytes()
     q_ms = sum(quant_ms) / len(quant_ms)
     achieved = q_bytes / (q_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(wl.name, "quant")
+    traffic = recorded_traffic(wl.name, workload_family(wl))
     out = {
         "metric": METRIC,
         "value": round(value, 2),
