@@ -854,8 +854,10 @@ static hadq_status kron_check(int64_t rows, int32_t a, int32_t b, int32_t bits, 
   return HADQ_OK;
 }
 
-static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, bool f32, cudaStream_t stream) {
-  const void* fn = hadq::kron_kernel_ptr(direction, s.bits);
+static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, bool f32, cudaStream_t stream,
+                               bool reg16 = false) {
+  const void* fn = reg16 ? hadq::kron16_kernel_ptr(s.bits) : hadq::kron_kernel_ptr(direction, s.bits);
+  const int threads = reg16 ? s.dim / 16 : 256;
   const size_t smem = hadq::kron_smem_bytes(s.dim, k.a);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
@@ -863,15 +865,15 @@ static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, 
     return fail(HADQ_ERR_CUDA, "Kronecker kernel: cannot reserve %zu bytes of shared memory: %s", smem,
                 cudaGetErrorString(e));
   }
-  const int64_t cap = int64_t(resident(fn, 256, smem)) * sm_count();
+  const int64_t cap = int64_t(resident(fn, threads, smem)) * sm_count();
   const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
   if (direction == 0) {
     void* args[] = {&k};
-    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
   } else {
     bool out_f32 = f32;
     void* args[] = {&k, &out_f32};
-    e = cudaLaunchKernel(fn, dim3(grid), dim3(256), args, smem, stream);
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
   }
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -909,7 +911,12 @@ hadq_status hadq_rotate_quantize_kron(const void* x, int64_t rows, int32_t a, co
   k.f = fa;
   k.a = a;
   k.ap = (a + hadq::kKronR - 1) / hadq::kKronR * hadq::kKronR;
-  return launch_kron(0, s, k, false, reinterpret_cast<cudaStream_t>(stream));
+  // register variant: 16 consecutive elements per thread
+  const int lg = s.G / 16;
+  const bool reg16 = b >= 16 && b <= 512 && s.G % 16 == 0 && s.G <= 512 && (32 % lg) == 0 && s.dim / 16 <= 1024 &&
+                     aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)) &&
+                     (!rotated_out || aligned(rotated_out, 16));
+  return launch_kron(0, s, k, false, reinterpret_cast<cudaStream_t>(stream), reg16);
 }
 
 hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales, int64_t rows, int32_t a,

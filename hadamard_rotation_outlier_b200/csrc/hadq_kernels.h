@@ -21,6 +21,8 @@ const void* keep_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* keep_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
 // Kronecker rotation F (x) H_b (direction 0 forward, 1 inverse), 256 threads.
 const void* kron_kernel_ptr(int direction, int bits);
+// Forward register variant (b and G in 16..512, dim / 16 threads per CTA).
+const void* kron16_kernel_ptr(int bits);
 // Asymmetric (zero-point) variants (groups of 128 x 2^k columns, warp teams).
 const void* asym_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* asym_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);

@@ -4,6 +4,10 @@
 
 namespace hadq {
 
+const void* kron16_kernel_ptr(int bits) {
+  return bits == 8 ? (const void*)rq_kron16_kernel<8> : (const void*)rq_kron16_kernel<4>;
+}
+
 const void* kron_kernel_ptr(int direction, int bits) {
   if (direction == 0) return bits == 8 ? (const void*)rq_kron_kernel<8> : (const void*)rq_kron_kernel<4>;
   return bits == 8 ? (const void*)dq_kron_kernel<8> : (const void*)dq_kron_kernel<4>;
