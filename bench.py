@@ -46,6 +46,7 @@ L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
                 "wide4096": "rq_wide4096_kernel", "none": None}
+KRON_KERNELS = {"smem": "rq_kron_kernel", "reg16": "rq_kron16_kernel", "mma": "rq_kron_tc_kernel"}
 
 
 def parse_args(argv=None):
@@ -196,7 +197,7 @@ def oracle_sample_rate(wl, target_s: float, seed: int = 42):
 
     fa = None
     if wl.kron_a:
-        fa = (S.paley_hadamard(wl.kron_a - 1).astype(np.float32) / np.float32(np.sqrt(wl.kron_a))).astype(np.float64)
+        fa = S.paley_hadamard(wl.kron_a - 1).astype(np.float64) / np.sqrt(wl.kron_a)
 
     def run(nrows):
         x = S.tensor_rows(wl, 0, 0, nrows, seed)
@@ -544,7 +545,9 @@ def run_ours(args):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": ("rq_kron_kernel" if wl.kron_a else "rq_chunk_asym_kernel" if wl.asym else
+            "kernel": (KRON_KERNELS[B.hadq_kron_plan(0, wl.rows, wl.kron_a, wl.dim // wl.kron_a, wl.bits,
+                                                     wl.group)] if wl.kron_a else
+                       "rq_chunk_asym_kernel" if wl.asym else
                        KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group,
                                                 wl.with_signs, True)]),
             "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
@@ -618,9 +621,9 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
                     h_out[r0:r1].copy_(st.out[r0:r1], non_blocking=True)
                     h_kept[h0:h1].copy_(st.kept[h0:h1], non_blocking=True)
                 elif wl.kron_a:
-                    B.hadq_rotate_quantize_kron(st.x[r0:r1], st.fa, wl.dim // wl.kron_a, signs=st.signs,
-                                                bits=wl.bits, group=wl.group, codes=st.codes[r0:r1],
-                                                scales=st.scales[r0:r1], stream=s)
+                    B.hadq_rotate_quantize_kron_pm1(st.x[r0:r1], st.sa, wl.dim // wl.kron_a, signs=st.signs,
+                                                    bits=wl.bits, group=wl.group, codes=st.codes[r0:r1],
+                                                    scales=st.scales[r0:r1], stream=s)
                 elif wl.asym:
                     B.hadq_rotate_quantize_asym(st.x[r0:r1], block=wl.block, signs=st.signs, bits=wl.bits,
                                                 group=wl.group, codes=st.codes[r0:r1], scales=st.scales[r0:r1],

@@ -17,16 +17,19 @@ from .binding import (  # noqa: F401
     hadq_dequant_rotate_inv,
     hadq_dequant_rotate_inv_asym,
     hadq_dequant_rotate_inv_kron,
+    hadq_dequant_rotate_inv_kron_pm1,
     hadq_dequant_rotate_inv_keep,
     hadq_kv_decode_attention,
     hadq_kv_decode_attention_noalloc,
     hadq_kv_decode_workspace_size,
     hadq_last_error,
     hadq_launch_count,
+    hadq_kron_plan,
     hadq_plan,
     hadq_rotate_quantize,
     hadq_rotate_quantize_asym,
     hadq_rotate_quantize_kron,
+    hadq_rotate_quantize_kron_pm1,
     hadq_rotate_quantize_keep,
     hyquant_keep_slots,
     hadq_status_str,

@@ -20,13 +20,14 @@ LIB_PATH = os.path.join(_PKG, "libhadq.so")
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
 PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096"}
+KRON_VARIANTS = {0: "smem", 1: "reg16", 2: "mma"}
 MAX_DIM = 32768
 
 EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quantize_kron",
-            "hadq_dequant_rotate_inv_kron", "hadq_rotate_quantize_asym",
+            "hadq_dequant_rotate_inv_kron", "hadq_rotate_quantize_kron_pm1", "hadq_dequant_rotate_inv_kron_pm1", "hadq_rotate_quantize_asym",
             "hadq_dequant_rotate_inv_asym", "hadq_rotate_quantize_keep",
             "hadq_dequant_rotate_inv_keep", "hadq_kv_decode_attention",
-            "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_status_str", "hadq_last_error",
+            "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_kron_plan", "hadq_status_str", "hadq_last_error",
             "hadq_launch_count", "hadq_version")
 
 
@@ -61,6 +62,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_dequant_rotate_inv_kron.argtypes = [vp, vp, c_i64, c_i32, vp, c_i32, vp, c_i32, c_i32, vp,
                                                  ctypes.c_int, vp]
     lib.hadq_dequant_rotate_inv_kron.restype = ctypes.c_int
+    lib.hadq_rotate_quantize_kron_pm1.argtypes = lib.hadq_rotate_quantize_kron.argtypes
+    lib.hadq_rotate_quantize_kron_pm1.restype = ctypes.c_int
+    lib.hadq_dequant_rotate_inv_kron_pm1.argtypes = lib.hadq_dequant_rotate_inv_kron.argtypes
+    lib.hadq_dequant_rotate_inv_kron_pm1.restype = ctypes.c_int
     lib.hadq_rotate_quantize_asym.argtypes = [vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp, vp, vp, vp]
     lib.hadq_rotate_quantize_asym.restype = ctypes.c_int
     lib.hadq_dequant_rotate_inv_asym.argtypes = [vp, vp, vp, c_i64, c_i32, c_i32, vp, c_i32, c_i32, vp,
@@ -86,6 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_plan.argtypes = [c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
                               ctypes.POINTER(ctypes.c_int)]
     lib.hadq_plan.restype = ctypes.c_int
+    lib.hadq_kron_plan.argtypes = [c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(ctypes.c_int)]
+    lib.hadq_kron_plan.restype = ctypes.c_int
     lib.hadq_status_str.argtypes = [ctypes.c_int]
     lib.hadq_status_str.restype = ctypes.c_char_p
     lib.hadq_last_error.argtypes = []
@@ -155,6 +162,15 @@ def hadq_plan(direction: int, rows: int, dim: int, block: int = -1, bits: int = 
     _check(load_library().hadq_plan(direction, rows, dim, block, bits, group, int(has_signs),
                                     int(aligned16), ctypes.byref(path)))
     return PATH_NAMES[path.value]
+
+
+def hadq_kron_plan(direction: int, rows: int, a: int, b: int, bits: int = 4, group: int = -1,
+                   aligned16: bool = True) -> str:
+    """Host-only: validate the sizes of a Kronecker call and name the kernel
+    variant it would launch ("smem", "reg16" or "mma")."""
+    v = ctypes.c_int(0)
+    _check(load_library().hadq_kron_plan(direction, rows, a, b, bits, group, int(aligned16), ctypes.byref(v)))
+    return KRON_VARIANTS[v.value]
 
 
 def hadq_rotate_quantize(x: torch.Tensor, block: int = -1, signs: torch.Tensor | None = None,
@@ -509,6 +525,19 @@ def hadq_rotate_quantize_kron(x: torch.Tensor, fa: torch.Tensor, b: int, signs: 
     """Kronecker rotation (F (x) H_b) then quantisation of a bf16 ``[..., a * b]``
     tensor; ``fa``: float32 CUDA ``[a, a]`` (as it multiplies).  Returns
     ``(codes, scales)`` as :func:`hadq_rotate_quantize`."""
+    return _kron_forward(False, x, fa, b, signs, bits, group, codes, scales, rotated_out, stream)
+
+
+def hadq_rotate_quantize_kron_pm1(x: torch.Tensor, sa: torch.Tensor, b: int, signs: torch.Tensor | None = None,
+                                  bits: int = 4, group: int = -1, codes: torch.Tensor | None = None,
+                                  scales: torch.Tensor | None = None, rotated_out: torch.Tensor | None = None,
+                                  stream=None):
+    """As :func:`hadq_rotate_quantize_kron` with the factor given as a +-1
+    matrix: ``sa`` int8 CUDA ``[a, a]``, F = sa / sqrt(a)."""
+    return _kron_forward(True, x, sa, b, signs, bits, group, codes, scales, rotated_out, stream)
+
+
+def _kron_forward(pm1, x, fa, b, signs, bits, group, codes, scales, rotated_out, stream):
     lib = load_library()
     if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous bf16 CUDA tensor")
@@ -519,7 +548,7 @@ def hadq_rotate_quantize_kron(x: torch.Tensor, fa: torch.Tensor, b: int, signs: 
     if dim != a * b:
         raise ValueError(f"rows of {dim} columns do not match a * b = {a * b}")
     dev = x.device
-    _need(fa, "fa", torch.float32, dev)
+    _need(fa, "sa" if pm1 else "fa", torch.int8 if pm1 else torch.float32, dev)
     rows = x.numel() // dim
     lead = tuple(x.shape[:-1])
     G = _resolve(dim, b, group)
@@ -539,8 +568,9 @@ def hadq_rotate_quantize_kron(x: torch.Tensor, fa: torch.Tensor, b: int, signs: 
         _need(signs, "signs", torch.int8, dev, dim)
     if rotated_out is not None:
         _need(rotated_out, "rotated_out", torch.float32, dev, x.numel())
-    _check(lib.hadq_rotate_quantize_kron(_ptr(x), rows, a, _ptr(fa), b, _ptr(signs), bits, group, _ptr(codes),
-                                         _ptr(scales), _ptr(rotated_out), _stream(stream)))
+    fn = lib.hadq_rotate_quantize_kron_pm1 if pm1 else lib.hadq_rotate_quantize_kron
+    _check(fn(_ptr(x), rows, a, _ptr(fa), b, _ptr(signs), bits, group, _ptr(codes), _ptr(scales), _ptr(rotated_out),
+              _stream(stream)))
     return codes, scales
 
 
@@ -549,13 +579,25 @@ def hadq_dequant_rotate_inv_kron(codes: torch.Tensor, scales: torch.Tensor, fa: 
                                  out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
                                  stream=None) -> torch.Tensor:
     """Inverse of :func:`hadq_rotate_quantize_kron`: ``[..., a * b]`` bf16 or fp32."""
+    return _kron_inverse(False, codes, scales, fa, b, signs, bits, group, out, out_dtype, stream)
+
+
+def hadq_dequant_rotate_inv_kron_pm1(codes: torch.Tensor, scales: torch.Tensor, sa: torch.Tensor, b: int,
+                                     signs: torch.Tensor | None = None, bits: int = 4, group: int = -1,
+                                     out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
+                                     stream=None) -> torch.Tensor:
+    """Inverse of :func:`hadq_rotate_quantize_kron_pm1` (``sa`` int8 +-1 ``[a, a]``)."""
+    return _kron_inverse(True, codes, scales, sa, b, signs, bits, group, out, out_dtype, stream)
+
+
+def _kron_inverse(pm1, codes, scales, fa, b, signs, bits, group, out, out_dtype, stream):
     lib = load_library()
     if not codes.is_cuda or not codes.is_contiguous():
         raise ValueError("codes must be a contiguous CUDA tensor")
     a = fa.shape[0]
     dim = a * b
     dev = codes.device
-    _need(fa, "fa", torch.float32, dev, a * a)
+    _need(fa, "sa" if pm1 else "fa", torch.int8 if pm1 else torch.float32, dev, a * a)
     per_row = dim if bits == 8 else dim // 2
     rows = codes.numel() // per_row
     lead = tuple(codes.shape[:-1]) if codes.shape[-1] == per_row else (rows,)
@@ -572,6 +614,7 @@ def hadq_dequant_rotate_inv_kron(codes: torch.Tensor, scales: torch.Tensor, fa: 
     else:
         _need(out, "out", out_dtype, dev, rows * dim)
     code = HADQ_OUT_F32 if out_dtype == torch.float32 else HADQ_OUT_BF16
-    _check(lib.hadq_dequant_rotate_inv_kron(_ptr(codes), _ptr(scales), rows, a, _ptr(fa), b, _ptr(signs), bits,
-                                            group, _ptr(out), code, _stream(stream)))
+    fn = lib.hadq_dequant_rotate_inv_kron_pm1 if pm1 else lib.hadq_dequant_rotate_inv_kron
+    _check(fn(_ptr(codes), _ptr(scales), rows, a, _ptr(fa), b, _ptr(signs), bits, group, _ptr(out), code,
+              _stream(stream)))
     return out

@@ -854,11 +854,24 @@ static hadq_status kron_check(int64_t rows, int32_t a, int32_t b, int32_t bits, 
   return HADQ_OK;
 }
 
+// Kernel variants of the Kronecker rotation (see hadq_kron_plan).
+static int kron_variant(int direction, const Shape& s, int a, int b, bool a16) {
+  if (direction != 0) return HADQ_KRON_SMEM;
+  const int G = s.G;
+  const bool reg = b >= 16 && b <= 512 && G % 16 == 0 && G <= 512 && (32 % (G / 16)) == 0 && s.dim / 16 <= 1024 &&
+                   a16;
+  if (!reg) return HADQ_KRON_SMEM;
+  if (a <= 32 && s.dim % 512 == 0 && s.dim / 16 <= 512) return HADQ_KRON_MMA;
+  return HADQ_KRON_REG16;
+}
+
 static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, bool f32, cudaStream_t stream,
-                               bool reg16 = false) {
-  const void* fn = reg16 ? hadq::kron16_kernel_ptr(s.bits) : hadq::kron_kernel_ptr(direction, s.bits);
-  const int threads = reg16 ? s.dim / 16 : 256;
-  const size_t smem = hadq::kron_smem_bytes(s.dim, k.a);
+                               int variant = HADQ_KRON_SMEM) {
+  const void* fn = variant == HADQ_KRON_MMA     ? hadq::kron_tc_kernel_ptr(s.bits, (k.a + 7) / 8, k.s != nullptr)
+                   : variant == HADQ_KRON_REG16 ? hadq::kron16_kernel_ptr(s.bits)
+                                                : hadq::kron_kernel_ptr(direction, s.bits);
+  const int threads = variant == HADQ_KRON_SMEM ? 256 : s.dim / 16;
+  const size_t smem = variant == HADQ_KRON_MMA ? hadq::kron_tc_smem_bytes(k.a, s.B) : hadq::kron_smem_bytes(s.dim, k.a);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -883,19 +896,34 @@ static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, 
   return after_launch("Kronecker kernel");
 }
 
-hadq_status hadq_rotate_quantize_kron(const void* x, int64_t rows, int32_t a, const float* fa, int32_t b,
-                                      const int8_t* signs, int32_t bits, int32_t group, void* codes, float* scales,
-                                      float* rotated_out, hadq_stream_t stream) {
+hadq_status hadq_kron_plan(int32_t direction, int64_t rows, int32_t a, int32_t b, int32_t bits, int32_t group,
+                           int32_t aligned16, int32_t* variant) {
+  g_last_error.clear();
+  if (direction != 0 && direction != 1)
+    return fail(HADQ_ERR_INVALID_ARG, "direction must be 0 or 1 (got %d)", direction);
+  Shape s;
+  hadq_status st = kron_check(rows, a, b, bits, group, &s);
+  if (st != HADQ_OK) return st;
+  if (variant) *variant = kron_variant(direction, s, a, b, aligned16 != 0);
+  return HADQ_OK;
+}
+
+// Forward Kronecker call with a float32 factor fa or a +-1 factor sa (one of
+// them non-null).
+static hadq_status kron_forward(bool pm1, const void* x, int64_t rows, int32_t a, const float* fa,
+                                const int8_t* sa, int32_t b, const int8_t* signs, int32_t bits, int32_t group, void* codes,
+                                float* scales, float* rotated_out, hadq_stream_t stream) {
   g_last_error.clear();
   Shape s;
   hadq_status st = kron_check(rows, a, b, bits, group, &s);
   if (st != HADQ_OK) return st;
   if (rows == 0) return HADQ_OK;
-  if (!x || !fa || !codes || !scales)
-    return fail(HADQ_ERR_INVALID_ARG, "x, fa, codes and scales must not be NULL");
+  if (!x || !(fa || sa) || !codes || !scales)
+    return fail(HADQ_ERR_INVALID_ARG, "x, %s, codes and scales must not be NULL", pm1 ? "sa" : "fa");
   if (!aligned(x, 2)) return fail(HADQ_ERR_MISALIGNED, "x must be 2-byte aligned");
-  if (!aligned(fa, 4) || !aligned(scales, 4) || (rotated_out && !aligned(rotated_out, 4)))
+  if ((fa && !aligned(fa, 4)) || !aligned(scales, 4) || (rotated_out && !aligned(rotated_out, 4)))
     return fail(HADQ_ERR_MISALIGNED, "fa, scales and rotated_out must be 4-byte aligned");
+  const double inv_sqrt_a = sa ? 1.0 / std::sqrt(double(a)) : 1.0;
   hadq::KronArgs k{};
   k.g.x = static_cast<const uint16_t*>(x);
   k.g.signs = signs;
@@ -909,19 +937,25 @@ hadq_status hadq_rotate_quantize_kron(const void* x, int64_t rows, int32_t a, co
   k.g.scale_mul = (float)(1.0 / (std::sqrt(double(b)) * double((1 << (bits - 1)) - 1)));
   k.g.rsqrt_b = (float)(1.0 / std::sqrt(double(b)));
   k.f = fa;
+  k.s = sa;
+  k.s_mul = (float)inv_sqrt_a;
   k.a = a;
   k.ap = (a + hadq::kKronR - 1) / hadq::kKronR * hadq::kKronR;
-  // register variant: 16 consecutive elements per thread
-  const int lg = s.G / 16;
-  const bool reg16 = b >= 16 && b <= 512 && s.G % 16 == 0 && s.G <= 512 && (32 % lg) == 0 && s.dim / 16 <= 1024 &&
-                     aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)) &&
-                     (!rotated_out || aligned(rotated_out, 16));
-  return launch_kron(0, s, k, false, reinterpret_cast<cudaStream_t>(stream), reg16);
+  const bool a16 = aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)) &&
+                   (!rotated_out || aligned(rotated_out, 16));
+  const int variant = kron_variant(0, s, a, b, a16);
+  if (variant == HADQ_KRON_MMA && sa) {
+    // the tensor-core kernel mixes with S itself: 1 / sqrt(a) joins the
+    // output multipliers
+    k.g.scale_mul = (float)(inv_sqrt_a / (std::sqrt(double(b)) * double((1 << (bits - 1)) - 1)));
+    k.g.rsqrt_b = (float)(inv_sqrt_a / std::sqrt(double(b)));
+  }
+  return launch_kron(0, s, k, false, reinterpret_cast<cudaStream_t>(stream), variant);
 }
 
-hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales, int64_t rows, int32_t a,
-                                         const float* fa, int32_t b, const int8_t* signs, int32_t bits,
-                                         int32_t group, void* out, hadq_out_dtype out_dtype, hadq_stream_t stream) {
+static hadq_status kron_inverse(bool pm1, const void* codes, const float* scales, int64_t rows, int32_t a,
+                                const float* fa, const int8_t* sa, int32_t b, const int8_t* signs, int32_t bits, int32_t group,
+                                void* out, hadq_out_dtype out_dtype, hadq_stream_t stream) {
   g_last_error.clear();
   Shape s;
   hadq_status st = kron_check(rows, a, b, bits, group, &s);
@@ -929,10 +963,11 @@ hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales,
   if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
     return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
   if (rows == 0) return HADQ_OK;
-  if (!codes || !scales || !fa || !out)
-    return fail(HADQ_ERR_INVALID_ARG, "codes, scales, fa and out must not be NULL");
+  if (!codes || !scales || !(fa || sa) || !out)
+    return fail(HADQ_ERR_INVALID_ARG, "codes, scales, %s and out must not be NULL", pm1 ? "sa" : "fa");
   const bool f32 = out_dtype == HADQ_OUT_F32;
-  if (!aligned(fa, 4) || !aligned(scales, 4)) return fail(HADQ_ERR_MISALIGNED, "fa and scales must be 4-byte aligned");
+  if ((fa && !aligned(fa, 4)) || !aligned(scales, 4))
+    return fail(HADQ_ERR_MISALIGNED, "fa and scales must be 4-byte aligned");
   if (!aligned(out, f32 ? 4 : 2)) return fail(HADQ_ERR_MISALIGNED, "out must be aligned to its element size");
   hadq::KronArgs k{};
   k.g.codes_in = static_cast<const uint8_t*>(codes);
@@ -946,9 +981,36 @@ hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales,
   k.g.group = s.G;
   k.g.rsqrt_b = (float)(1.0 / std::sqrt(double(b)));
   k.f = fa;
+  k.s = sa;
+  k.s_mul = (float)(1.0 / std::sqrt(double(a)));
   k.a = a;
   k.ap = (a + hadq::kKronR - 1) / hadq::kKronR * hadq::kKronR;
   return launch_kron(1, s, k, f32, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hadq_status hadq_rotate_quantize_kron(const void* x, int64_t rows, int32_t a, const float* fa, int32_t b,
+                                      const int8_t* signs, int32_t bits, int32_t group, void* codes, float* scales,
+                                      float* rotated_out, hadq_stream_t stream) {
+  return kron_forward(false, x, rows, a, fa, nullptr, b, signs, bits, group, codes, scales, rotated_out, stream);
+}
+
+hadq_status hadq_rotate_quantize_kron_pm1(const void* x, int64_t rows, int32_t a, const int8_t* sa, int32_t b,
+                                          const int8_t* signs, int32_t bits, int32_t group, void* codes,
+                                          float* scales, float* rotated_out, hadq_stream_t stream) {
+  return kron_forward(true, x, rows, a, nullptr, sa, b, signs, bits, group, codes, scales, rotated_out, stream);
+}
+
+hadq_status hadq_dequant_rotate_inv_kron(const void* codes, const float* scales, int64_t rows, int32_t a,
+                                         const float* fa, int32_t b, const int8_t* signs, int32_t bits,
+                                         int32_t group, void* out, hadq_out_dtype out_dtype, hadq_stream_t stream) {
+  return kron_inverse(false, codes, scales, rows, a, fa, nullptr, b, signs, bits, group, out, out_dtype, stream);
+}
+
+hadq_status hadq_dequant_rotate_inv_kron_pm1(const void* codes, const float* scales, int64_t rows, int32_t a,
+                                             const int8_t* sa, int32_t b, const int8_t* signs, int32_t bits,
+                                             int32_t group, void* out, hadq_out_dtype out_dtype,
+                                             hadq_stream_t stream) {
+  return kron_inverse(true, codes, scales, rows, a, nullptr, sa, b, signs, bits, group, out, out_dtype, stream);
 }
 
 const char* hadq_status_str(hadq_status st) {

@@ -18,6 +18,8 @@
 // The 1/sqrt(b) of H_b is folded into the scale, as everywhere else.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "hadq_generic.cuh"
 
 namespace hadq {
@@ -25,11 +27,18 @@ namespace hadq {
 constexpr int kKronR = 8;  // outputs per thread in the mixing step
 
 struct KronArgs {
-  GenericArgs g;   // x / codes_in, scales, signs, codes / out, rows, dim = a * b, block = b, group
-  const float* f;  // [a][a] factor, row-major, device memory
+  GenericArgs g;      // x / codes_in, scales, signs, codes / out, rows, dim = a * b, block = b, group
+  const float* f;     // [a][a] factor, row-major, device memory (null when s is given)
+  const int8_t* s;    // [a][a] +-1 matrix S, row-major: the factor is S * s_mul (null when f is given)
+  float s_mul;        // 1 / sqrt(a) for s
   int a;
-  int ap;          // a rounded up to a multiple of kKronR (pitch of the transposed coefficients)
+  int ap;             // a rounded up to a multiple of kKronR (pitch of the transposed coefficients)
 };
+
+// Entry (r, i) of the factor.
+__device__ __forceinline__ float kron_factor(const KronArgs& k, int r, int i) {
+  return k.s ? float(k.s[r * k.a + i]) * k.s_mul : __ldg(k.f + r * k.a + i);
+}
 
 // Shared memory: in[dim] | out[dim] | coefficients [a][ap] | codes [dim] (int8);
 // the register variant pads in and out by 4 floats per 32 (see kron_pad) and
@@ -41,10 +50,11 @@ __host__ __device__ inline size_t kron_smem_bytes(int dim, int a) {
 
 // Coefficients of the mixing step, transposed: ct[i * ap + r] = C[r][i] for
 // C = F (transpose == false) or C = F^T; columns r >= a are zero.
-__device__ __forceinline__ void kron_load_coeffs(const float* f, int a, int ap, bool transpose, float* ct) {
+__device__ __forceinline__ void kron_load_coeffs(const KronArgs& k, bool transpose, float* ct) {
+  const int a = k.a, ap = k.ap;
   for (int e = threadIdx.x; e < a * ap; e += blockDim.x) {
     const int i = e / ap, r = e - i * ap;
-    ct[e] = r < a ? (transpose ? f[i * a + r] : f[r * a + i]) : 0.0f;
+    ct[e] = r < a ? (transpose ? kron_factor(k, i, r) : kron_factor(k, r, i)) : 0.0f;
   }
 }
 
@@ -106,7 +116,7 @@ __global__ void __launch_bounds__(256) rq_kron_kernel(KronArgs k) {
   int8_t* scode = reinterpret_cast<int8_t*>(ct + k.a * k.ap);
   const int ngroups = dim / G;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  kron_load_coeffs(k.f, k.a, k.ap, false, ct);
+  kron_load_coeffs(k, false, ct);
 
   for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
     const int64_t base = row * dim;
@@ -164,7 +174,7 @@ __global__ void __launch_bounds__(256) dq_kron_kernel(KronArgs k, bool out_f32) 
   float* ct = kbuf + 2 * dim;
   int* stiny = reinterpret_cast<int*>(ct + k.a * k.ap);
   const int ngroups = dim / G;
-  kron_load_coeffs(k.f, k.a, k.ap, true, ct);
+  kron_load_coeffs(k, true, ct);
 
   for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
     const int64_t base = row * dim;
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
   const int lanes_b = b >> 4;  // lanes per sub-block
   const int lanes_g = G >> 4;  // lanes per scale group
   const int lb = kron_log2(b);
-  kron_load_coeffs(k.f, k.a, k.ap, false, ct);
+  kron_load_coeffs(k, false, ct);
   // sign masks of this thread's 16 columns (bf16 pairs)
   uint32_t smask[8];
 #pragma unroll
@@ -298,6 +308,273 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
       *reinterpret_cast<uint2*>(a.codes + (base + e0) / 2) = make_uint2(pack_i4x8(cc0), pack_i4x8(cc1));
     }
     __syncthreads();  // sin / sout are reused by the next row
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core variant of the forward transform for a <= 32.
+//
+// F (x) H_b = (I (x) H_b)(F (x) I): the mixing may run first, on the signed
+// bf16 input itself, which bf16 holds exactly.  Per row, the mixing is then
+// the product W[r][j] = sum_i F[r][i] X[i][j], a GEMM of M = b (columns j),
+// N = a (rows r of F) and K = a, which runs as warp-level bf16 MMAs with
+// float32 accumulation:
+//   - F is split into three bf16 terms hi + mid + lo (exact to about 2^-24
+//     of each entry; the products with the bf16 data are exact), applied
+//     smallest first into one accumulator;
+//   - X sits in shared memory as bf16 [i][j]; ldmatrix.trans hands each warp
+//     the A fragments (16 columns j x 16 or 8 rows i), and the F terms stay in
+//     registers as B fragments for the whole kernel;
+//   - K and N are padded to multiples of 8 with zero rows of X and zero
+//     entries of F.
+// W goes to shared memory as float32, each thread reads back its 16
+// consecutive outputs and finishes as the register variant does: bits 0-3
+// of the b-butterflies in registers, the rest across lanes, then the group
+// maxima and the codes.  KA = ceil(a / 8).
+//
+// Shared memory: X [8 KA][kron_tc_px(b) bytes] | W [a][kron_tc_pw(b) floats].
+// Row pitches: X rows are 2b + 16 bytes (an odd number of 16-byte units, so
+// the eight rows of an ldmatrix tile fall in different banks); W rows hold
+// b floats with 4 of padding after every 32 (the 128-bit reads of 16
+// consecutive floats are conflict-free) and a pitch of 4 mod 32 words, so that
+// the accumulator stores (8 columns x 4 row pairs per warp) are conflict-free
+// too.
+
+__host__ __device__ inline int kron_tc_px(int b) { return 2 * b + 16; }
+
+__host__ __device__ inline int kron_tc_pw(int b) {
+  const int base = b + (b >> 5) * 4;
+  return base + ((36 - (base & 31)) & 31);
+}
+
+__host__ __device__ inline size_t kron_tc_smem_bytes(int a, int b) {
+  const int ka = (a + 7) / 8;
+  return size_t(8) * ka * kron_tc_px(b) + size_t(a) * kron_tc_pw(b) * 4;
+}
+
+__device__ __forceinline__ int kron_tc_inner(int j) { return j + ((j >> 5) << 2); }
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_k16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// The three bf16 terms of f (term 0 largest), as 16-bit patterns.
+__device__ __forceinline__ void bf16_split3(float f, uint32_t (&t)[3]) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(f);
+  const float r1 = f - __bfloat162float(h);  // exact
+  const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(m);  // exact
+  const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+  t[0] = __bfloat16_as_ushort(h);
+  t[1] = __bfloat16_as_ushort(m);
+  t[2] = __bfloat16_as_ushort(l);
+}
+
+template <int BITS, int KA, int NS>
+__global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
+  static_assert(NS == 1 || NS == 3, "one term (a +-1 factor) or three (a float32 factor)");
+  constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
+  const GenericArgs& a = k.g;
+  extern __shared__ __align__(16) unsigned char tbuf[];
+  const int dim = a.dim, b = a.block, G = a.group, fa = k.a;
+  const int px = kron_tc_px(b), pw = kron_tc_pw(b);
+  unsigned char* xs = tbuf;
+  float* ws = reinterpret_cast<float*>(tbuf + size_t(8) * KA * px);
+  const int t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int e0 = 16 * t;
+  const int lb = kron_log2(b);
+  const int lanes_b = b >> 4, lanes_g = G >> 4;
+  const int xi = e0 >> lb, xj = e0 & (b - 1);  // this thread's row and first column
+
+  // zero X (rows a .. 8 KA - 1 stay zero: the K padding)
+  for (int e = t; e < 8 * KA * px / 16; e += blockDim.x) reinterpret_cast<uint4*>(xs)[e] = make_uint4(0, 0, 0, 0);
+
+  // B fragments: bf[s][nt][kk] = {C[r][i], C[r][i + 1]} (term s) with
+  // r = 8 nt + g, i = 8 kk + 2 t4; zero outside a x a.  C = S itself for a
+  // +-1 factor (one exact term; its 1 / sqrt(a) is in scale_mul and rsqrt_b),
+  // else F in three terms.
+  uint32_t bf[NS][KA][KA];
+#pragma unroll
+  for (int nt = 0; nt < KA; ++nt) {
+#pragma unroll
+    for (int kk = 0; kk < KA; ++kk) {
+      const int r = 8 * nt + g, i = 8 * kk + 2 * t4;
+      if constexpr (NS == 1) {
+        const float f0 = (r < fa && i < fa) ? float(k.s[r * fa + i]) : 0.0f;
+        const float f1 = (r < fa && i + 1 < fa) ? float(k.s[r * fa + i + 1]) : 0.0f;
+        bf[0][nt][kk] = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(f0))) |
+                        (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(f1))) << 16);
+      } else {
+        const float f0 = (r < fa && i < fa) ? __ldg(k.f + r * fa + i) : 0.0f;
+        const float f1 = (r < fa && i + 1 < fa) ? __ldg(k.f + r * fa + i + 1) : 0.0f;
+        uint32_t s0[3], s1[3];
+        bf16_split3(f0, s0);
+        bf16_split3(f1, s1);
+#pragma unroll
+        for (int s = 0; s < 3; ++s) bf[s][nt][kk] = s0[s] | (s1[s] << 16);
+      }
+    }
+  }
+
+  // sign masks of this thread's 16 columns (bf16 pairs)
+  uint32_t smask[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) smask[i] = 0u;
+  if (a.signs) {
+    const uint4 sg = *reinterpret_cast<const uint4*>(a.signs + e0);
+    const uint32_t w[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t word = w[i >> 1];
+      const int sh = 16 * (i & 1);
+      smask[i] = (((word >> (sh + 7)) & 1u) << 15) | (((word >> (sh + 15)) & 1u) << 31);
+    }
+  }
+
+  // this lane's ldmatrix row address (bytes, shared window) for k16 step 0 of
+  // m-tile 0: x4 tiles (i 0-7, j 0-7), (i 0-7, j 8-15), (i 8-15, j 0-7),
+  // (i 8-15, j 8-15) -> a0..a3; the x2 tail uses the first two
+  const uint32_t xs_base = static_cast<uint32_t>(__cvta_generic_to_shared(xs));
+  const int lm = lane >> 3, lr = lane & 7;
+  const uint32_t a_addr = xs_base + uint32_t(((lm >> 1) * 8 + lr) * px + (lm & 1) * 16);
+  const uint32_t a_addr_tail = xs_base + uint32_t(((KA - 1) * 8 + lr) * px + (lm & 1) * 16);
+  const int half = (t >> 2) & 1;  // store order of the two 16-byte halves
+
+  uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+  if (int64_t(blockIdx.x) < a.rows) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(blockIdx.x) * dim + e0);
+    n0 = src[0];
+    n1 = src[1];
+  }
+
+  for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
+    const int64_t base = row * dim;
+    {
+      const uint4 s0 = make_uint4(n0.x ^ smask[0], n0.y ^ smask[1], n0.z ^ smask[2], n0.w ^ smask[3]);
+      const uint4 s1 = make_uint4(n1.x ^ smask[4], n1.y ^ smask[5], n1.z ^ smask[6], n1.w ^ smask[7]);
+      uint4* dst = reinterpret_cast<uint4*>(xs + xi * px + 2 * xj);
+      dst[half] = half ? s1 : s0;
+      dst[half ^ 1] = half ? s0 : s1;
+    }
+    if (row + gridDim.x < a.rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + (row + gridDim.x) * dim + e0);
+      n0 = src[0];
+      n1 = src[1];
+    }
+    __syncthreads();
+
+    // mixing: m-tile mt covers columns j = 16 mt .. 16 mt + 15
+    for (int mt = warp; mt < (b >> 4); mt += nwarps) {
+      float d[KA][4];
+#pragma unroll
+      for (int nt = 0; nt < KA; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.0f;
+#pragma unroll
+      for (int kp = 0; kp < KA / 2; ++kp) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(a_addr + uint32_t(kp * 16 * px + mt * 32), a0, a1, a2, a3);
+        // smallest term first; consecutive MMAs go to different accumulators
+#pragma unroll
+        for (int s = NS - 1; s >= 0; --s) {
+#pragma unroll
+          for (int nt = 0; nt < KA; ++nt)
+            mma_bf16_k16(d[nt], a0, a1, a2, a3, bf[s][nt][2 * kp], bf[s][nt][2 * kp + 1]);
+        }
+      }
+      if constexpr (KA & 1) {
+        uint32_t a0, a1;
+        ldsm_x2_trans(a_addr_tail + uint32_t(mt * 32), a0, a1);
+#pragma unroll
+        for (int s = NS - 1; s >= 0; --s) {
+#pragma unroll
+          for (int nt = 0; nt < KA; ++nt) mma_bf16_k8(d[nt], a0, a1, bf[s][nt][KA - 1]);
+        }
+      }
+      // d[nt] = W[r][j], W[r + 1][j], W[r][j + 8], W[r + 1][j + 8] with
+      // r = 8 nt + 2 t4, j = 16 mt + g
+      const int j = 16 * mt + g;
+      const int c0 = kron_tc_inner(j), c1 = kron_tc_inner(j + 8);
+#pragma unroll
+      for (int nt = 0; nt < KA; ++nt) {
+        const int r = 8 * nt + 2 * t4;
+        if (r < fa) {
+          ws[r * pw + c0] = d[nt][0];
+          ws[r * pw + c1] = d[nt][2];
+        }
+        if (r + 1 < fa) {
+          ws[(r + 1) * pw + c0] = d[nt][1];
+          ws[(r + 1) * pw + c1] = d[nt][3];
+        }
+      }
+    }
+    __syncthreads();
+
+    // butterflies along j of this thread's 16 outputs, then the quantiser
+    float v[16];
+    {
+      const float* src = ws + xi * pw + kron_tc_inner(xj);
+#pragma unroll
+      for (int i = 0; i < 16; i += 4) {
+        const float4 q = *reinterpret_cast<const float4*>(src + i);
+        v[i] = q.x;
+        v[i + 1] = q.y;
+        v[i + 2] = q.z;
+        v[i + 3] = q.w;
+      }
+    }
+    reg_fwht<16, 4>(v);
+    for (int m = 1; m < lanes_b; m <<= 1) {  // bits 4.. of the column index: lanes
+      const float sg = (lane & m) ? -1.0f : 1.0f;
+      lane_stage<16>(v, m, sg);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+    for (int o = 1; o < lanes_g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((t & (lanes_g - 1)) == 0) a.scales[(base + e0) / G] = m * a.scale_mul;
+    if (a.rot) {
+      float4* dst = reinterpret_cast<float4*>(a.rot + base + e0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_float4(v[4 * i] * a.rsqrt_b, v[4 * i + 1] * a.rsqrt_b, v[4 * i + 2] * a.rsqrt_b,
+                             v[4 * i + 3] * a.rsqrt_b);
+    }
+    uint32_t cc0[8], cc1[8];
+    quantize8(v, m, QMAX, cc0);
+    quantize8(v + 8, m, QMAX, cc1);
+    if constexpr (BITS == 8) {
+      *reinterpret_cast<uint4*>(a.codes + base + e0) =
+          make_uint4(pack_i8x4(cc0[0], cc0[1], cc0[2], cc0[3]), pack_i8x4(cc0[4], cc0[5], cc0[6], cc0[7]),
+                     pack_i8x4(cc1[0], cc1[1], cc1[2], cc1[3]), pack_i8x4(cc1[4], cc1[5], cc1[6], cc1[7]));
+    } else {
+      *reinterpret_cast<uint2*>(a.codes + (base + e0) / 2) = make_uint2(pack_i4x8(cc0), pack_i4x8(cc1));
+    }
   }
 }
 

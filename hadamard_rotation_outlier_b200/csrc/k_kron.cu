@@ -13,4 +13,20 @@ const void* kron_kernel_ptr(int direction, int bits) {
   return bits == 8 ? (const void*)dq_kron_kernel<8> : (const void*)dq_kron_kernel<4>;
 }
 
+template <int BITS, int NS>
+static const void* kron_tc_for(int ka) {
+  switch (ka) {
+    case 1: return (const void*)rq_kron_tc_kernel<BITS, 1, NS>;
+    case 2: return (const void*)rq_kron_tc_kernel<BITS, 2, NS>;
+    case 3: return (const void*)rq_kron_tc_kernel<BITS, 3, NS>;
+    case 4: return (const void*)rq_kron_tc_kernel<BITS, 4, NS>;
+    default: return nullptr;
+  }
+}
+
+const void* kron_tc_kernel_ptr(int bits, int ka, bool pm1) {
+  if (pm1) return bits == 8 ? kron_tc_for<8, 1>(ka) : kron_tc_for<4, 1>(ka);
+  return bits == 8 ? kron_tc_for<8, 3>(ka) : kron_tc_for<4, 3>(ka);
+}
+
 }  // namespace hadq

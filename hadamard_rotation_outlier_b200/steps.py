@@ -57,10 +57,9 @@ class WorkloadStep:
                             if wl.asym else None)
         self.out = (torch.empty((self.rows, dim), dtype=torch.bfloat16, device=self.device)
                     if wl.dequant else None)
-        self.fa = None
+        self.sa = None   # the stored +-1 factor S_a of a Kronecker workload (F = S_a / sqrt(a))
         if wl.kron_a:
-            P = S.paley_hadamard(wl.kron_a - 1).astype(np.float32) / np.float32(np.sqrt(wl.kron_a))
-            self.fa = torch.from_numpy(P).to(self.device)
+            self.sa = torch.from_numpy(S.paley_hadamard(wl.kron_a - 1)).to(self.device)
         self.keep_slot = self.kept = None
         if wl.keep:
             n_sink, window, n_vertical = wl.keep
@@ -86,7 +85,7 @@ class WorkloadStep:
     def quantize(self, stream=None, rotated_out=None):
         wl = self.wl
         if wl.kron_a:
-            B.hadq_rotate_quantize_kron(self.x, self.fa, wl.dim // wl.kron_a, signs=self.signs, bits=wl.bits,
+            B.hadq_rotate_quantize_kron_pm1(self.x, self.sa, wl.dim // wl.kron_a, signs=self.signs, bits=wl.bits,
                                         group=wl.group, codes=self.codes, scales=self.scales,
                                         rotated_out=rotated_out, stream=stream)
             return

@@ -185,8 +185,8 @@ WORKLOADS = {
     "c6_tok8192_d5120_kron20x256_int4_g128": Workload(
         name="c6_tok8192_d5120_kron20x256_int4_g128",
         description="8192 tokens x 5120 (no Sylvester matrix of that width), N(0,1) with 5 channels "
-                    "x100; seeded signs, Kronecker rotation (Paley H_20 / sqrt(20)) x (H_256); "
-                    "INT4 group 128",
+                    "x100; seeded signs, Kronecker rotation (Paley S_20 / sqrt(20)) x (H_256) with the "
+                    "factor given as the stored +-1 matrix S_20; INT4 group 128",
         dim=5120, block=256, group=128, bits=4, with_signs=True, dist="normal",
         tensors=(Tensor("x", 8192, 1, 5, 100.0, 7),), kron_a=20),
     "c5_tok32768_w11008_b128_signs_int4_g128": Workload(

@@ -76,6 +76,17 @@ typedef enum {
                               one block per warp, in-warp transpose         */
 } hadq_path;
 
+/* Kernel variant of a Kronecker-rotation call (see hadq_kron_plan). */
+typedef enum {
+  HADQ_KRON_SMEM = 0,   /* one CTA per row, the row in shared memory; any
+                           valid shape, and every inverse                   */
+  HADQ_KRON_REG16 = 1,  /* forward: 16 elements per thread, butterflies in
+                           registers and lanes, mixing on the FP32 cores    */
+  HADQ_KRON_MMA = 2     /* forward, a <= 32: mixing first, as bf16 tensor-
+                           core MMAs against a three-term split of F, then
+                           the register butterflies                         */
+} hadq_kron_variant;
+
 enum { HADQ_MAX_DIM = 32768 };
 
 /*
@@ -156,6 +167,49 @@ hadq_status hadq_dequant_rotate_inv_kron(const void *codes, const float *scales,
                                          const int8_t *signs, int32_t bits, int32_t group,
                                          void *out, hadq_out_dtype out_dtype,
                                          hadq_stream_t stream);
+
+/*
+ * hadq_rotate_quantize_kron_pm1 / hadq_dequant_rotate_inv_kron_pm1 -- the
+ * same transforms with the factor given as the stored +-1 Hadamard matrix
+ * itself: F = S_a / sqrt(a) ("QuaRot: rotation-based outlier suppression",
+ * msModelSlim, online rotation: widths without a Sylvester matrix use a
+ * stored Hadamard matrix).
+ *
+ *   sa    device int8 [a][a], row-major, entries +1 / -1 (other values are
+ *         used as given: the factor is whatever S_a / sqrt(a) they form).
+ *   All other arguments, layouts, errors and outputs as for
+ *   hadq_rotate_quantize_kron / hadq_dequant_rotate_inv_kron.
+ * With a +-1 factor the tensor-core variant (see hadq_kron_plan) mixes with
+ * S_a exactly, one bf16 term instead of three, and folds 1 / sqrt(a) into the
+ * scale; the other variants multiply S_a by 1 / sqrt(a) (rounded to float32)
+ * as they load it.
+ */
+hadq_status hadq_rotate_quantize_kron_pm1(const void *x, int64_t rows, int32_t a, const int8_t *sa,
+                                          int32_t b, const int8_t *signs, int32_t bits,
+                                          int32_t group, void *codes, float *scales,
+                                          float *rotated_out, hadq_stream_t stream);
+hadq_status hadq_dequant_rotate_inv_kron_pm1(const void *codes, const float *scales, int64_t rows,
+                                             int32_t a, const int8_t *sa, int32_t b,
+                                             const int8_t *signs, int32_t bits, int32_t group,
+                                             void *out, hadq_out_dtype out_dtype,
+                                             hadq_stream_t stream);
+
+/*
+ * hadq_kron_plan -- host-only: validate the sizes of a Kronecker call
+ * (direction 0 = hadq_rotate_quantize_kron, 1 = its inverse) and report the
+ * kernel variant it would launch.  `aligned16` says whether every pointer of
+ * the call is 16-byte aligned.  The forward takes
+ *   HADQ_KRON_MMA    for a <= 32, 16 <= b <= 512, a * b a multiple of 512 and
+ *                    at most 8192, groups of 16..512 columns with
+ *                    G / 16 dividing 32, all pointers 16-byte aligned;
+ *   HADQ_KRON_REG16  for the same b, group and alignment otherwise, with
+ *                    a * b <= 16384;
+ *   HADQ_KRON_SMEM   for everything else.
+ * Returns the status the call would return for these sizes (pointer checks
+ * aside) and writes the variant to *variant.  Touches no GPU.
+ */
+hadq_status hadq_kron_plan(int32_t direction, int64_t rows, int32_t a, int32_t b, int32_t bits,
+                           int32_t group, int32_t aligned16, int32_t *variant);
 
 /*
  * hadq_rotate_quantize_asym -- rotate, then quantise with a zero point

@@ -323,3 +323,32 @@ def test_kron_entry_validates(lib, a, b, bits, group, status, msg):
     assert st == status, B.hadq_last_error()
     assert msg in B.hadq_last_error()
     assert B.hadq_launch_count() == n0
+
+
+@pytest.mark.parametrize("direction,a,b,group,a16,variant", [
+    (0, 20, 256, 128, True, "mma"),     # the 5120-column workload
+    (0, 8, 64, 64, True, "mma"),
+    (0, 32, 128, 128, True, "mma"),
+    (0, 1, 512, 512, True, "mma"),
+    (0, 20, 256, 128, False, "smem"),   # pointers not 16-byte aligned
+    (0, 12, 32, 64, True, "reg16"),     # 384 columns: not a multiple of 512
+    (0, 40, 128, 128, True, "reg16"),   # a > 32
+    (0, 28, 512, 128, True, "reg16"),   # 14336 columns: above 8192
+    (0, 7, 32, 56, True, "smem"),       # group of 56 columns
+    (0, 16, 8, 64, True, "smem"),       # b < 16
+    (1, 20, 256, 128, True, "smem"),    # every inverse
+])
+def test_kron_plan_variants(lib, direction, a, b, group, a16, variant):
+    assert B.hadq_kron_plan(direction, 100, a, b, 4, group, a16) == variant
+
+
+def test_kron_plan_rejects_like_the_call(lib):
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_kron_plan(0, 4, 12, 48)
+    assert e.value.status == B.HADQ_ERR_INVALID_ARG and "power of two" in str(e.value)
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_kron_plan(2, 4, 12, 64)
+    assert e.value.status == B.HADQ_ERR_INVALID_ARG
+    with pytest.raises(B.HadqError) as e:
+        B.hadq_kron_plan(0, 4, 255, 128)
+    assert e.value.status == B.HADQ_ERR_UNSUPPORTED

@@ -90,7 +90,7 @@ def test_full_workload_sampled_parity(name):
         x, g_codes, g_scales, idx = x[keep_q], g_codes[keep_q], g_scales[keep_q], idx[torch.from_numpy(keep_q).to("cuda")]
         assert len(x) > 20
     if wl.kron_a:
-        F = (S.paley_hadamard(wl.kron_a - 1).astype(np.float32) / np.float32(np.sqrt(wl.kron_a))).astype(np.float64)
+        F = S.paley_hadamard(wl.kron_a - 1).astype(np.float64) / np.sqrt(wl.kron_a)   # the exact factor
         ref = O.rotate_quantize_kron(x, F, dim // wl.kron_a, signs, bits, wl.group)
         check_scales(g_scales, ref["scales"])
         check_codes(gpu_codes_to_int(g_codes, bits, dim), ref["q"], ref["pre_round"])
