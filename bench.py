@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
-                "wide4096": "rq_wide4096_kernel", "none": None}
+                "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_mma_kernel", "none": None}
 KRON_KERNELS = {"smem": "rq_kron_kernel", "reg16": "rq_kron16_kernel", "mma": "rq_kron_tc_kernel"}
 
 
@@ -82,13 +82,23 @@ KERNEL_SOURCES = {
     "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
     "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
-    "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_kron.cuh", "k_kron.cu"],
+    "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_mma.cuh", "hadq_kron.cuh", "k_kron.cu"],
+    "h4096": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_h4096.cuh", "k_h4096.cu"],
 }
 
 
 def workload_family(wl) -> str:
     """Kernel family whose sources a workload's timed kernel is built from."""
-    return "kron" if wl.kron_a else "asym" if wl.asym else "keep" if wl.keep else "quant"
+    from hadamard_rotation_outlier_b200 import binding as B
+    if wl.kron_a:
+        return "kron"
+    if wl.asym:
+        return "asym"
+    if wl.keep:
+        return "keep"
+    if B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True) == "wide4096_mma":
+        return "h4096"
+    return "quant"
 
 
 def kernel_source_hash(family: str) -> str:

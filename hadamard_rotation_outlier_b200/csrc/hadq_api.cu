@@ -20,6 +20,7 @@
 #include "hadq_chunk.cuh"
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
+#include "hadq_h4096.cuh"
 #include "hadq_kron.cuh"
 #include "hadq_kernels.h"
 
@@ -100,7 +101,8 @@ bool chunk_ok(int direction, const Shape& s) {
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
-  if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096) return HADQ_PATH_WIDE4096;
+  if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096)
+    return (s.dim == 4096 || !s.has_signs) ? HADQ_PATH_WIDE4096_MMA : HADQ_PATH_WIDE4096;
   if (aligned16 && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) && s.dim % 32 == 0 &&
       s.dim <= 16384 && blocked_group_ok(s.G, s.B))
     return HADQ_PATH_BLOCKED;
@@ -246,7 +248,7 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   return launch_chunk_args(direction, s, ka, false, f32, stream);
 }
 
-hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream, bool mma) {
   a.cpr = s.dim / hadq::kCK;
   a.nchunks = s.rows * a.cpr;
   a.slab_chunks = 32;
@@ -254,19 +256,20 @@ hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stre
   a.dim = s.dim;
   a.log_g = -1;
   a.gpc = 32;
-  const void* fn = hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
-  const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
+  const void* fn = mma ? hadq::h4096_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr) : hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
+  const size_t smem = mma ? hadq::h4096_smem_bytes(s.has_signs) : hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
+  const int threads = mma ? hadq::kH4096Warps * 32 : hadq::kCT;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(HADQ_ERR_CUDA, "4096-block kernel: cannot reserve %zu bytes of shared memory: %s", smem,
                 cudaGetErrorString(e));
   }
-  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
-  const int64_t want = (a.nchunks / 32 + 3) / 4;  // one block per warp
+  const int64_t cap = int64_t(resident(fn, threads, smem)) * sm_count();
+  const int64_t want = (a.nchunks / 32 + threads / 32 - 1) / (threads / 32);  // one block per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
-  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -535,7 +538,7 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.rsqrt_b = rsqrt_b;
     return launch_chunk(0, s, a, false, cs);
   }
-  if (path == HADQ_PATH_WIDE4096) {
+  if (path == HADQ_PATH_WIDE4096 || path == HADQ_PATH_WIDE4096_MMA) {
     hadq::ChunkArgs a{};
     a.x = static_cast<const uint16_t*>(x);
     a.signs = signs;
@@ -544,7 +547,7 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.rot = rotated_out;
     a.scale_mul = scale_mul;
     a.rsqrt_b = rsqrt_b;
-    return launch_wide4096(s, a, cs);
+    return launch_wide4096(s, a, cs, path == HADQ_PATH_WIDE4096_MMA);
   }
   if (path == HADQ_PATH_FULL4096) {
     hadq::FullArgs a{};

@@ -31,6 +31,8 @@ const void* asym_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* asym_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
 // 4096-column blocks, one scale per block, one block per warp.
 const void* wide4096_kernel_ptr(int bits, bool signs);
+// The same with the first 16-point stage on tensor cores (kH4096Warps warps).
+const void* h4096_mma_kernel_ptr(int bits, bool signs, bool rot);
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);
 const void* generic_kernel_ptr(int direction, int bits);
 

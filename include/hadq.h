@@ -72,8 +72,11 @@ typedef enum {
   HADQ_PATH_GENERIC = 3,   /* shared-memory kernel, any valid combination   */
   HADQ_PATH_CHUNK = 4,     /* one 128-column chunk per thread, blocks <= 128,
                               slabs staged through shared memory            */
-  HADQ_PATH_WIDE4096 = 5   /* 4096-column blocks with one scale per block:
+  HADQ_PATH_WIDE4096 = 5,  /* 4096-column blocks with one scale per block:
                               one block per warp, in-warp transpose         */
+  HADQ_PATH_WIDE4096_MMA = 6 /* the same blocks (dim = 4096 when signs are
+                              given) with the first 16-point stage as a bf16
+                              tensor-core MMA against H_16                  */
 } hadq_path;
 
 /* Kernel variant of a Kronecker-rotation call (see hadq_kron_plan). */

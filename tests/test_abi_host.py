@@ -75,7 +75,9 @@ def test_plan_rejects(lib, args, msg):
     (0, 0, 128, -1, 8, -1, False, True, "none"),
     (0, 524288, 128, -1, 8, -1, False, True, "chunk"),            # Q/K heads, INT8
     (0, 256, 4096, 128, 4, -1, False, True, "chunk"),             # per-token over 32 blocks
-    (0, 16384, 4096, -1, 4, -1, True, True, "wide4096"),          # full 4096 + signs
+    (0, 16384, 4096, -1, 4, -1, True, True, "wide4096_mma"),      # full 4096 + signs
+    (0, 16, 8192, 4096, 4, 4096, True, True, "wide4096"),         # two 4096 blocks + signs
+    (0, 16, 8192, 4096, 4, 4096, False, True, "wide4096_mma"),    # two 4096 blocks, no signs
     (0, 16384, 4096, -1, 4, 128, True, True, "full4096"),         # 4096 block, group 128
     (0, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV cache
     (1, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV dequant

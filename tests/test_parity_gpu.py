@@ -92,10 +92,13 @@ CASES = [
     (6, 8192, 256, 1024, 8, True, "blocked"),
     (129, 64, 64, 32, 4, False, "blocked"),         # dim not a multiple of 128
     (61, 96, 32, 8, 8, True, "blocked"),
-    (21, 4096, -1, -1, 4, True, "wide4096"),        # full 4096 + signs, per token
-    (22, 4096, -1, -1, 8, False, "wide4096"),
+    (21, 4096, -1, -1, 4, True, "wide4096_mma"),    # full 4096 + signs, per token
+    (22, 4096, -1, -1, 8, False, "wide4096_mma"),
+    (37, 4096, -1, -1, 8, True, "wide4096_mma"),    # INT8 with signs; more rows than one CTA's warps
+    (1, 4096, -1, -1, 4, False, "wide4096_mma"),    # a single row
     (5, 8192, 4096, 4096, 8, True, "wide4096"),     # two 4096-blocks per row, scale per block
-    (3, 12288, 4096, 4096, 4, False, "wide4096"),
+    (4, 8192, 4096, 4096, 4, True, "wide4096"),
+    (3, 12288, 4096, 4096, 4, False, "wide4096_mma"),   # three blocks per row, no signs
     (19, 4096, -1, 128, 8, False, "full4096"),
     (7, 4096, 4096, 64, 4, True, "full4096"),
     (11, 4096, -1, 1024, 8, True, "full4096"),
@@ -212,3 +215,22 @@ def test_binding_rejects_bad_tensors():
     assert e.value.status == B.HADQ_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         B.hadq_rotate_quantize(torch.zeros((128, 4), dtype=torch.bfloat16, device=DEV).t(), bits=8)
+
+
+@pytest.mark.parametrize("bits,with_signs", [(4, True), (8, False)])
+def test_wide4096_mma_edge_rows(bits, with_signs):
+    # the tensor-core 4096 path: zero, one-hot, tiny (1e-30, bf16 subnormal
+    # 1e-39), huge (1e30) and spiky rows, and a row count that leaves some
+    # warps of the last CTA without a block
+    rng = np.random.default_rng(31)
+    dim = 4096
+    rows = [np.zeros(dim, np.float32),
+            np.eye(dim, dtype=np.float32)[1234] * 3.0,
+            (rng.normal(size=dim) * 1e-30).astype(np.float32),
+            (rng.normal(size=dim) * 1e-39).astype(np.float32),
+            (rng.normal(size=dim) * 1e30).astype(np.float32),
+            np.where(rng.random(dim) < 0.001, 5e3, rng.normal(size=dim)).astype(np.float32),
+            rng.normal(size=dim).astype(np.float32)]
+    x = S.f32_to_bf16_bits(np.stack(rows))
+    assert B.hadq_plan(0, len(rows), dim, -1, bits, -1, with_signs, True) == "wide4096_mma"
+    run_case(len(rows), dim, -1, -1, bits, with_signs, seed=12, x_bits=x)
