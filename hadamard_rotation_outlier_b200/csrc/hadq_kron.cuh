@@ -241,6 +241,8 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
   const int lanes_b = b >> 4;  // lanes per sub-block
   const int lanes_g = G >> 4;  // lanes per scale group
   const int lb = kron_log2(b);
+  const int lg = kron_log2(G);
+  const int gpr = dim >> lg, my_g = e0 >> lg;  // scale groups per row, this thread's group
   kron_load_coeffs(k, false, ct);
   // sign masks of this thread's 16 columns (bf16 pairs)
   uint32_t smask[8];
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
     for (int o = 1; o < lanes_g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((t & (lanes_g - 1)) == 0) a.scales[(base + e0) / G] = m * a.scale_mul;
+    if ((t & (lanes_g - 1)) == 0) a.scales[row * gpr + my_g] = m * a.scale_mul;
     if (a.rot) {
       float4* dst = reinterpret_cast<float4*>(a.rot + base + e0);
 #pragma unroll
@@ -333,7 +335,8 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
 // of the b-butterflies in registers, the rest across lanes, then the group
 // maxima and the codes.  KA = ceil(a / 8).
 //
-// Shared memory: X [8 KA][kron_tc_px(b) bytes] | W [a][kron_tc_pw(b) floats].
+// Shared memory: X [8 KA][kron_tc_px(b) bytes] | W [8 KA][kron_tc_pw(b) floats]
+// (W rows a .. 8 KA - 1 take the zero outputs of the N padding; never read).
 // Row pitches: X rows are 2b + 16 bytes (an odd number of 16-byte units, so
 // the eight rows of an ldmatrix tile fall in different banks); W rows hold
 // b floats with 4 of padding after every 32 (the 128-bit reads of 16
@@ -350,7 +353,7 @@ __host__ __device__ inline int kron_tc_pw(int b) {
 
 __host__ __device__ inline size_t kron_tc_smem_bytes(int a, int b) {
   const int ka = (a + 7) / 8;
-  return size_t(8) * ka * kron_tc_px(b) + size_t(a) * kron_tc_pw(b) * 4;
+  return size_t(8) * ka * kron_tc_px(b) + size_t(8) * ka * kron_tc_pw(b) * 4;
 }
 
 __device__ __forceinline__ int kron_tc_inner(int j) { return j + ((j >> 5) << 2); }
@@ -383,6 +386,8 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
   const int e0 = 16 * t;
   const int lb = kron_log2(b);
   const int lanes_b = b >> 4, lanes_g = G >> 4;
+  const int lg = kron_log2(G);
+  const int gpr = dim >> lg, my_g = e0 >> lg;  // scale groups per row, this thread's group
   const int xi = e0 >> lb, xj = e0 & (b - 1);  // this thread's row and first column
 
   // zero X (rows a .. 8 KA - 1 stay zero: the K padding)
@@ -492,17 +497,14 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
       // r = 8 nt + 2 t4, j = 16 mt + g
       const int j = 16 * mt + g;
       const int c0 = kron_tc_inner(j), c1 = kron_tc_inner(j + 8);
+      float* w0 = ws + 2 * t4 * pw;
 #pragma unroll
       for (int nt = 0; nt < KA; ++nt) {
-        const int r = 8 * nt + 2 * t4;
-        if (r < fa) {
-          ws[r * pw + c0] = d[nt][0];
-          ws[r * pw + c1] = d[nt][2];
-        }
-        if (r + 1 < fa) {
-          ws[(r + 1) * pw + c0] = d[nt][1];
-          ws[(r + 1) * pw + c1] = d[nt][3];
-        }
+        float* wr = w0 + 8 * nt * pw;  // row r = 8 nt + 2 t4 (rows >= a hold zeros, never read)
+        wr[c0] = d[nt][0];
+        wr[c1] = d[nt][2];
+        wr[pw + c0] = d[nt][1];
+        wr[pw + c1] = d[nt][3];
       }
     }
     __syncthreads();
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
     for (int o = 1; o < lanes_g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((t & (lanes_g - 1)) == 0) a.scales[(base + e0) / G] = m * a.scale_mul;
+    if ((t & (lanes_g - 1)) == 0) a.scales[row * gpr + my_g] = m * a.scale_mul;
     if (a.rot) {
       float4* dst = reinterpret_cast<float4*>(a.rot + base + e0);
 #pragma unroll
@@ -537,9 +539,18 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
         dst[i] = make_float4(v[4 * i] * a.rsqrt_b, v[4 * i + 1] * a.rsqrt_b, v[4 * i + 2] * a.rsqrt_b,
                              v[4 * i + 3] * a.rsqrt_b);
     }
+    // one multiplier for the 16 codes, paired magic-number FMAs
+    const QInv q = make_qinv(m, QMAX);
+    if (q.tiny) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] *= 18446744073709551616.0f;
+    }
     uint32_t cc0[8], cc1[8];
-    quantize8(v, m, QMAX, cc0);
-    quantize8(v + 8, m, QMAX, cc1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      magic_code2(v[2 * i], v[2 * i + 1], q.inv, cc0[2 * i], cc0[2 * i + 1]);
+      magic_code2(v[8 + 2 * i], v[9 + 2 * i], q.inv, cc1[2 * i], cc1[2 * i + 1]);
+    }
     if constexpr (BITS == 8) {
       *reinterpret_cast<uint4*>(a.codes + base + e0) =
           make_uint4(pack_i8x4(cc0[0], cc0[1], cc0[2], cc0[3]), pack_i8x4(cc0[4], cc0[5], cc0[6], cc0[7]),
