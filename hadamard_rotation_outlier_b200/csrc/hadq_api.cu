@@ -870,7 +870,7 @@ static int kron_variant(int direction, const Shape& s, int a, int b, bool a16) {
 
 static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, bool f32, cudaStream_t stream,
                                int variant = HADQ_KRON_SMEM) {
-  const void* fn = variant == HADQ_KRON_MMA     ? hadq::kron_tc_kernel_ptr(s.bits, (k.a + 7) / 8, k.s != nullptr)
+  const void* fn = variant == HADQ_KRON_MMA     ? hadq::kron_tc_kernel_ptr(s.bits, (k.a + 7) / 8, k.s != nullptr, s.B == 256)
                    : variant == HADQ_KRON_REG16 ? hadq::kron16_kernel_ptr(s.bits)
                                                 : hadq::kron_kernel_ptr(direction, s.bits);
   const int threads = variant == HADQ_KRON_SMEM ? 256 : s.dim / 16;

@@ -24,8 +24,9 @@ const void* kron_kernel_ptr(int direction, int bits);
 // Forward register variant (b and G in 16..512, dim / 16 threads per CTA).
 const void* kron16_kernel_ptr(int bits);
 // Forward tensor-core variant (a <= 32, ka = ceil(a / 8); dim / 16 threads);
-// pm1: the factor is a +-1 matrix times 1 / sqrt(a).
-const void* kron_tc_kernel_ptr(int bits, int ka, bool pm1);
+// pm1: the factor is a +-1 matrix times 1 / sqrt(a); s256: b = 256 (strided
+// shared-memory pass instead of lane shuffles).
+const void* kron_tc_kernel_ptr(int bits, int ka, bool pm1, bool s256);
 // Asymmetric (zero-point) variants (groups of 128 x 2^k columns, warp teams).
 const void* asym_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* asym_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);

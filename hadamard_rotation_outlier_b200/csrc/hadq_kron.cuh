@@ -370,7 +370,10 @@ __device__ __forceinline__ void bf16_split3(float f, uint32_t (&t)[3]) {
   t[2] = __bfloat16_as_ushort(l);
 }
 
-template <int BITS, int KA, int NS>
+// S256 (b = 256): bits 4-7 of the column index run as a strided pass over W
+// (16 columns u + 16 k per thread, 4 register stages, written back) before the
+// consecutive pass, instead of four lane-shuffle stages.
+template <int BITS, int KA, int NS, bool S256>
 __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
   static_assert(NS == 1 || NS == 3, "one term (a +-1 factor) or three (a float32 factor)");
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
@@ -511,6 +514,15 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
 
     // butterflies along j of this thread's 16 outputs, then the quantiser
     float v[16];
+    if constexpr (S256) {
+      float* col = ws + xi * pw + (t & 15);  // row xi, columns (t & 15) + 16 kk
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) v[kk] = col[16 * kk + 4 * (kk >> 1)];
+      reg_fwht<16, 4>(v);
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) col[16 * kk + 4 * (kk >> 1)] = v[kk];
+      __syncthreads();
+    }
     {
       const float* src = ws + xi * pw + kron_tc_inner(xj);
 #pragma unroll
@@ -523,9 +535,11 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
       }
     }
     reg_fwht<16, 4>(v);
-    for (int m = 1; m < lanes_b; m <<= 1) {  // bits 4.. of the column index: lanes
-      const float sg = (lane & m) ? -1.0f : 1.0f;
-      lane_stage<16>(v, m, sg);
+    if constexpr (!S256) {
+      for (int m = 1; m < lanes_b; m <<= 1) {  // bits 4.. of the column index: lanes
+        const float sg = (lane & m) ? -1.0f : 1.0f;
+        lane_stage<16>(v, m, sg);
+      }
     }
     float m = 0.0f;
 #pragma unroll
