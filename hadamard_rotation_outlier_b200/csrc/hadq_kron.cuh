@@ -342,11 +342,15 @@ __global__ void __launch_bounds__(1024) rq_kron16_kernel(KronArgs k) {
 // b floats with 4 of padding after every 32 (the 128-bit reads of 16
 // consecutive floats are conflict-free) and a pitch of 4 mod 32 words, so that
 // the accumulator stores (8 columns x 4 row pairs per warp) are conflict-free
-// too.
+// too.  For b = 256 (the strided pass) the pitch is 16 mod 32 and column j of
+// row r sits at (j ^ 8 ((r >> 1) & 3)) + 4 (j >> 5): the accumulator stores,
+// the strided pass (two rows per warp) and the 128-bit reads are then all
+// conflict-free.
 
 __host__ __device__ inline int kron_tc_px(int b) { return 2 * b + 16; }
 
 __host__ __device__ inline int kron_tc_pw(int b) {
+  if (b == 256) return 304;
   const int base = b + (b >> 5) * 4;
   return base + ((36 - (base & 31)) & 31);
 }
@@ -373,8 +377,16 @@ __device__ __forceinline__ void bf16_split3(float f, uint32_t (&t)[3]) {
 // S256 (b = 256): bits 4-7 of the column index run as a strided pass over W
 // (16 columns u + 16 k per thread, 4 register stages, written back) before the
 // consecutive pass, instead of four lane-shuffle stages.
+// Register caps: 64 (a 320-thread CTA three times per SM) wherever the B
+// fragments allow it, 96 (twice) for the three-term split of a <= 24, 128 for
+// a <= 32 with the split.
+template <int KA, int NS>
+constexpr int kron_tc_maxreg() {
+  return NS == 3 ? (KA <= 2 ? 64 : KA == 3 ? 96 : 128) : (KA <= 3 ? 64 : 96);
+}
+
 template <int BITS, int KA, int NS, bool S256>
-__global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
+__global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronArgs k) {
   static_assert(NS == 1 || NS == 3, "one term (a +-1 factor) or three (a float32 factor)");
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   const GenericArgs& a = k.g;
@@ -499,7 +511,9 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
       // d[nt] = W[r][j], W[r + 1][j], W[r][j + 8], W[r + 1][j + 8] with
       // r = 8 nt + 2 t4, j = 16 mt + g
       const int j = 16 * mt + g;
-      const int c0 = kron_tc_inner(j), c1 = kron_tc_inner(j + 8);
+      // rows 8 nt + 2 t4 (+1) have (r >> 1) & 3 = t4
+      const int c0 = S256 ? (j ^ (8 * t4)) + 4 * (j >> 5) : kron_tc_inner(j);
+      const int c1 = S256 ? ((j + 8) ^ (8 * t4)) + 4 * ((j + 8) >> 5) : kron_tc_inner(j + 8);
       float* w0 = ws + 2 * t4 * pw;
 #pragma unroll
       for (int nt = 0; nt < KA; ++nt) {
@@ -515,15 +529,32 @@ __global__ void __launch_bounds__(512) rq_kron_tc_kernel(KronArgs k) {
     // butterflies along j of this thread's 16 outputs, then the quantiser
     float v[16];
     if constexpr (S256) {
-      float* col = ws + xi * pw + (t & 15);  // row xi, columns (t & 15) + 16 kk
+      // columns u + 16 kk of row xi (u = t & 15), swizzled: even kk at pe,
+      // odd kk at po, each + 36 (kk >> 1)
+      const int f = (xi >> 1) & 3, u = t & 15;
+      float* rowp = ws + xi * pw + (u ^ (8 * (f & 1)));
+      float* pe = rowp + 16 * (f >> 1);
+      float* po = rowp + 16 - 16 * (f >> 1);
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) v[kk] = col[16 * kk + 4 * (kk >> 1)];
+      for (int kk = 0; kk < 16; ++kk) v[kk] = ((kk & 1) ? po : pe)[36 * (kk >> 1)];
       reg_fwht<16, 4>(v);
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) col[16 * kk + 4 * (kk >> 1)] = v[kk];
+      for (int kk = 0; kk < 16; ++kk) ((kk & 1) ? po : pe)[36 * (kk >> 1)] = v[kk];
       __syncthreads();
-    }
-    {
+      // the thread's 16 consecutive columns 16 u .. 16 u + 15: float4 i at
+      // offset 4 (i ^ 2 (f & 1)) from the swizzled run start
+      const float* base = ws + xi * pw + 36 * (u >> 1) + 16 * ((u & 1) ^ (f >> 1));
+      const float* q0 = base + 8 * (f & 1);
+      const float* q1 = base + 8 - 8 * (f & 1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 q = *reinterpret_cast<const float4*>((i < 2 ? q0 : q1) + 4 * (i & 1));
+        v[4 * i] = q.x;
+        v[4 * i + 1] = q.y;
+        v[4 * i + 2] = q.z;
+        v[4 * i + 3] = q.w;
+      }
+    } else {
       const float* src = ws + xi * pw + kron_tc_inner(xj);
 #pragma unroll
       for (int i = 0; i < 16; i += 4) {
