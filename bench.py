@@ -45,7 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
-                "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_mma_kernel", "none": None}
+                "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_mma_kernel",
+                "chunk_mma": "rq_chunk_mma_kernel", "none": None}
 KRON_KERNELS = {"smem": "rq_kron_kernel", "reg16": "rq_kron16_kernel", "mma": "rq_kron_tc_kernel"}
 
 
@@ -77,8 +78,8 @@ def measured_peaks():
 # figure stays valid while these files hash the same.
 KERNEL_SOURCES = {
     "quant": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_blocked.cuh", "hadq_full4096.cuh",
-              "hadq_generic.cuh", "k_blocked.cu", "k_chunk.cu", "k_chunk_dq4.cu", "k_chunk_dq8.cu",
-              "k_full4096.cu", "k_generic.cu"],
+              "hadq_generic.cuh", "hadq_mma.cuh", "hadq_chunk_mma.cuh", "k_blocked.cu", "k_chunk.cu",
+              "k_chunk_dq4.cu", "k_chunk_dq8.cu", "k_chunk_mma.cu", "k_full4096.cu", "k_generic.cu"],
     "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
     "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],

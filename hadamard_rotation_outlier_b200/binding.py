@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libhadq.so")
 
 HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
 HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
-PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096", 6: "wide4096_mma"}
+PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096", 6: "wide4096_mma", 7: "chunk_mma"}
 KRON_VARIANTS = {0: "smem", 1: "reg16", 2: "mma"}
 MAX_DIM = 32768
 

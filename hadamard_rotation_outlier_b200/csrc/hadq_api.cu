@@ -18,6 +18,7 @@
 #include "hadq_attn.cuh"
 #include "hadq_blocked.cuh"
 #include "hadq_chunk.cuh"
+#include "hadq_chunk_mma.cuh"
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
 #include "hadq_h4096.cuh"
@@ -100,6 +101,8 @@ bool chunk_ok(int direction, const Shape& s) {
 
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
+  if (aligned16 && direction == 0 && s.B == 128 && s.G == 128 && s.dim % 128 == 0 && !s.has_signs)
+    return HADQ_PATH_CHUNK_MMA;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
   if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096)
     return (s.dim == 4096 || !s.has_signs) ? HADQ_PATH_WIDE4096_MMA : HADQ_PATH_WIDE4096;
@@ -246,6 +249,35 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   hadq::ChunkKeepArgs ka{};
   static_cast<hadq::ChunkArgs&>(ka) = a;
   return launch_chunk_args(direction, s, ka, false, f32, stream);
+}
+
+hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+  a.cpr = s.dim / hadq::kCK;
+  a.nchunks = s.rows * a.cpr;
+  a.slab_chunks = 32;
+  a.G = s.G;
+  a.dim = s.dim;
+  a.log_g = 7;
+  a.gpc = 1;
+  const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, a.rot != nullptr);
+  const size_t smem = hadq::chunk_smem_bytes(s.dim, false, false);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "128-block tensor-core kernel: cannot reserve %zu bytes of shared memory: %s", smem,
+                cudaGetErrorString(e));
+  }
+  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab of 32 blocks per warp
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  void* args[] = {&a};
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "128-block tensor-core kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("128-block tensor-core kernel");
 }
 
 hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream, bool mma) {
@@ -537,6 +569,16 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.scale_mul = scale_mul;
     a.rsqrt_b = rsqrt_b;
     return launch_chunk(0, s, a, false, cs);
+  }
+  if (path == HADQ_PATH_CHUNK_MMA) {
+    hadq::ChunkArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.codes = static_cast<uint8_t*>(codes);
+    a.scales = scales;
+    a.rot = rotated_out;
+    a.scale_mul = scale_mul;
+    a.rsqrt_b = rsqrt_b;
+    return launch_chunk_mma(s, a, cs);
   }
   if (path == HADQ_PATH_WIDE4096 || path == HADQ_PATH_WIDE4096_MMA) {
     hadq::ChunkArgs a{};

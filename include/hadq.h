@@ -74,9 +74,13 @@ typedef enum {
                               slabs staged through shared memory            */
   HADQ_PATH_WIDE4096 = 5,  /* 4096-column blocks with one scale per block:
                               one block per warp, in-warp transpose         */
-  HADQ_PATH_WIDE4096_MMA = 6 /* the same blocks (dim = 4096 when signs are
+  HADQ_PATH_WIDE4096_MMA = 6, /* the same blocks (dim = 4096 when signs are
                               given) with the first 16-point stage as a bf16
                               tensor-core MMA against H_16                  */
+  HADQ_PATH_CHUNK_MMA = 7  /* forward, 128-point blocks with one scale per
+                              block and no signs: the first 16-point stage
+                              as a bf16 MMA over 16 blocks at a time, the
+                              other three in registers                      */
 } hadq_path;
 
 /* Kernel variant of a Kronecker-rotation call (see hadq_kron_plan). */

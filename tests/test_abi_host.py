@@ -73,13 +73,13 @@ def test_plan_rejects(lib, args, msg):
 
 @pytest.mark.parametrize("direction,rows,dim,block,bits,group,signs,a16,path", [
     (0, 0, 128, -1, 8, -1, False, True, "none"),
-    (0, 524288, 128, -1, 8, -1, False, True, "chunk"),            # Q/K heads, INT8
+    (0, 524288, 128, -1, 8, -1, False, True, "chunk_mma"),        # Q/K heads, INT8
     (0, 256, 4096, 128, 4, -1, False, True, "chunk"),             # per-token over 32 blocks
     (0, 16384, 4096, -1, 4, -1, True, True, "wide4096_mma"),      # full 4096 + signs
     (0, 16, 8192, 4096, 4, 4096, True, True, "wide4096"),         # two 4096 blocks + signs
     (0, 16, 8192, 4096, 4, 4096, False, True, "wide4096_mma"),    # two 4096 blocks, no signs
     (0, 16384, 4096, -1, 4, 128, True, True, "full4096"),         # 4096 block, group 128
-    (0, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV cache
+    (0, 2097152, 128, 128, 4, 128, False, True, "chunk_mma"),     # KV cache
     (1, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV dequant
     (1, 10, 1024, 256, 4, 64, False, True, "blocked"),            # 256-point dequant
     (0, 32768, 11008, 128, 4, 128, True, True, "chunk"),          # 86 blocks of 128
@@ -89,7 +89,9 @@ def test_plan_rejects(lib, args, msg):
     (0, 10, 128, -1, 8, -1, False, False, "generic"),             # unaligned pointers
     (0, 10, 4096, -1, 4, 32, False, True, "generic"),             # small groups on 4096
     (0, 10, 8192, -1, 4, -1, False, True, "generic"),             # 8192-point block
-    (0, 10, 32768, 128, 4, 128, False, True, "chunk"),            # widest row, group 128
+    (0, 10, 32768, 128, 4, 128, False, True, "chunk_mma"),        # widest row, group 128
+    (0, 10, 32768, 128, 4, 128, True, True, "chunk"),             # the same with signs
+    (0, 10, 256, 128, 4, 64, False, True, "chunk"),               # groups smaller than the block
     (0, 10, 12, 4, 8, 3, False, True, "generic"),
     (1, 10, 4096, -1, 4, -1, True, True, "generic"),              # 4096 dequant
 ])

@@ -30,7 +30,7 @@ def oracle_method(dim, block):
 
 
 def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", outliers=(),
-             x_bits=None, offset=0, check_dequant=True):
+             x_bits=None, offset=0, check_dequant=True, max_mismatches=None):
     if x_bits is None:
         x_bits = S.random_bf16(rows, dim, seed, dist=dist, outlier_cols=outliers)
     s = S.random_signs(dim, seed) if with_signs else None
@@ -49,7 +49,7 @@ def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", o
     torch.cuda.synchronize()
     check_values(rot.cpu().numpy(), ref["rotated"], "rotated")
     check_scales(scales.cpu().numpy(), ref["scales"])
-    check_codes(gpu_codes_to_int(codes.cpu().numpy(), bits, dim), ref["q"], ref["pre_round"])
+    check_codes(gpu_codes_to_int(codes.cpu().numpy(), bits, dim), ref["q"], ref["pre_round"], max_mismatches)
 
     # the same codes without the optional float output (the timed configuration)
     codes2, scales2 = B.hadq_rotate_quantize(x, block=block, signs=sg, bits=bits, group=group)
@@ -73,8 +73,12 @@ def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", o
 
 # (rows, dim, block, group, bits, signs, expected forward path)
 CASES = [
-    (300, 128, -1, -1, 8, False, "chunk"),          # Q/K heads, INT8, per row
-    (301, 128, 128, 128, 4, False, "chunk"),        # KV rows, INT4, group 128
+    (300, 128, -1, -1, 8, False, "chunk_mma"),      # Q/K heads, INT8, per row
+    (301, 128, 128, 128, 4, False, "chunk_mma"),    # KV rows, INT4, group 128
+    (33, 384, 128, 128, 8, False, "chunk_mma"),     # three blocks per row, a short last slab
+    (7, 11008, 128, 128, 4, False, "chunk_mma"),    # 86 blocks per row
+    (1, 128, 128, 128, 4, False, "chunk_mma"),      # one block
+    (65, 1024, 128, 128, 8, False, "chunk_mma"),
     (37, 4096, 128, -1, 4, False, "chunk"),         # per-token scale over 32 blocks
     (9, 11008, 128, 128, 4, True, "chunk"),         # 86 blocks, signs
     (5, 11008, 128, -1, 8, True, "chunk"),          # 86 blocks, one scale per row
@@ -234,3 +238,23 @@ def test_wide4096_mma_edge_rows(bits, with_signs):
     x = S.f32_to_bf16_bits(np.stack(rows))
     assert B.hadq_plan(0, len(rows), dim, -1, bits, -1, with_signs, True) == "wide4096_mma"
     run_case(len(rows), dim, -1, -1, bits, with_signs, seed=12, x_bits=x)
+
+
+@pytest.mark.parametrize("dim,bits", [(128, 8), (384, 4)])
+def test_chunk_mma_edge_rows(dim, bits):
+    # the tensor-core 128 path: zero, one-hot, tiny (1e-30, bf16 subnormal
+    # 1e-39), huge (1e30) and spiky rows; 40 rows = one full slab of 32
+    # blocks plus a short one.  A block with K spikes of 5e3 puts pre-round
+    # values next to the ties 7 k / K, so boundary mismatches (each still
+    # within 1e-4 of a .5 boundary) are not capped at one here.
+    rng = np.random.default_rng(dim + bits)
+    base = [np.zeros(dim, np.float32),
+            np.eye(dim, dtype=np.float32)[dim // 3] * 3.0,
+            (rng.normal(size=dim) * 1e-30).astype(np.float32),
+            (rng.normal(size=dim) * 1e-39).astype(np.float32),
+            (rng.normal(size=dim) * 1e30).astype(np.float32),
+            np.where(rng.random(dim) < 0.02, 5e3, rng.normal(size=dim)).astype(np.float32)]
+    rows = base + [rng.normal(size=dim).astype(np.float32) for _ in range(40 - len(base))]
+    x = S.f32_to_bf16_bits(np.stack(rows))
+    assert B.hadq_plan(0, len(rows), dim, 128, bits, 128, False, True) == "chunk_mma"
+    run_case(len(rows), dim, 128, 128, bits, False, seed=13, x_bits=x, max_mismatches=16)
