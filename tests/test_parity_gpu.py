@@ -81,6 +81,7 @@ CASES = [
     (65, 1024, 128, 128, 8, False, "chunk_mma"),
     (37, 4096, 128, -1, 4, False, "chunk"),         # per-token scale over 32 blocks
     (9, 11008, 128, 128, 4, True, "chunk"),         # 86 blocks, signs
+    (45, 1152, 128, 128, 8, True, "chunk"),         # signs, 9 blocks per row, a short last slab
     (5, 11008, 128, -1, 8, True, "chunk"),          # 86 blocks, one scale per row
     (300, 256, 32, 8, 4, False, "chunk"),           # groups smaller than a block
     (70, 512, 64, 16, 8, True, "chunk"),
