@@ -11,8 +11,16 @@ step of attention over the rotated INT4 KV cache: one launch that reads every
 cached K/V code and scale once.  Inputs are resident in HBM before the
 timed region.  Between timed steps a 256 MiB buffer is written to flush the
 126 MB L2; that write sits outside the CUDA events that time each step.  The
-default workload is the Q/K rotation (2 x [1, 32, 8192, 128] bf16, full
-128-point Hadamard, per token-head INT8).
+default workload is the largest of the five synthetic configurations: 32768
+tokens x 11008 columns of Student-t(3) bf16 values, seeded signs, 86 blocks of
+the 128-point Hadamard, INT4 codes with one fp32 scale per 128 columns.
+
+The same line carries ``per_config``: every one of the five configurations
+(and the KV-cache dequantiser) timed the same way, plus a ``sustained``
+figure per kernel taken back to back with no flush, where each launch also
+pays the write-back of the previous launch's outputs still dirty in L2.
+Fractions are given against the measured copy bandwidth and against the
+nominal 8 TB/s of the B200's HBM3e.
 
 Multi-GPU (torchrun, one process per GPU): rows are independent, so every rank
 runs its own copy of the workload with no data-path collective ("weak"
@@ -26,7 +34,6 @@ instead (rank 0 only, bounded samples of the same workload).
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
 import statistics
@@ -39,9 +46,12 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-DEFAULT_WORKLOAD = "c2_qk_h32_s8192_d128_int8"
+DEFAULT_WORKLOAD = "c5_tok32768_w11008_b128_signs_int4_g128"
+PER_CONFIG = ["c1_tok256_h4096_b128_int4", "c2_qk_h32_s8192_d128_int8", "c3_tok16384_h4096_full_signs_int4",
+              "c4_kv_h8_t131072_d128_int4_g128", "c5_tok32768_w11008_b128_signs_int4_g128"]
 METRIC = "fused Hadamard+quantize GB/s (bf16 in→int4/int8 out), % of B200 HBM peak"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, vendor figure
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
@@ -61,6 +71,10 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="time only the headline workload")
+    p.add_argument("--config-steps", type=int, default=50,
+                   help="timed steps per per_config entry (flushed and back to back each)")
     return p.parse_args(argv)
 
 
@@ -74,62 +88,8 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# Device sources each kernel family is built from; a recorded DRAM traffic
-# figure stays valid while these files hash the same.
-KERNEL_SOURCES = {
-    "quant": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_blocked.cuh", "hadq_full4096.cuh",
-              "hadq_generic.cuh", "hadq_mma.cuh", "hadq_chunk_mma.cuh", "k_blocked.cu", "k_chunk.cu",
-              "k_chunk_dq4.cu", "k_chunk_dq8.cu", "k_chunk_mma.cu", "k_full4096.cu", "k_generic.cu"],
-    "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
-    "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
-    "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
-    "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_mma.cuh", "hadq_kron.cuh", "k_kron.cu"],
-    "h4096": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_h4096.cuh", "k_h4096.cu"],
-}
-
-
-def workload_family(wl) -> str:
-    """Kernel family whose sources a workload's timed kernel is built from."""
-    from hadamard_rotation_outlier_b200 import binding as B
-    if wl.kron_a:
-        return "kron"
-    if wl.asym:
-        return "asym"
-    if wl.keep:
-        return "keep"
-    if B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True) == "wide4096_mma":
-        return "h4096"
-    return "quant"
-
-
-def kernel_source_hash(family: str) -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "hadamard_rotation_outlier_b200", "csrc")
-    for name in sorted(KERNEL_SOURCES[family]):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
-    return h.hexdigest()[:16]
-
-
-def recorded_traffic(workload: str, family: str):
-    """DRAM bytes per launch of the workload's timed kernel from a committed ncu
-    summary.
-
-    ``profiles/dram_traffic.txt`` holds lines ``workload source_hash bytes``;
-    the figure is used only while the kernel family's sources still hash the
-    same (see ``KERNEL_SOURCES``).
-    """
-    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    try:
-        lines = open(path).read().splitlines()
-    except OSError:
-        return None
-    h = kernel_source_hash(family)
-    for ln in lines:
-        parts = ln.split()
-        if len(parts) == 3 and not ln.startswith("#") and parts[0] == workload and parts[1] == h:
-            return int(parts[2])
-    return None
+from hadamard_rotation_outlier_b200.records import (KERNEL_SOURCES, kernel_source_hash,  # noqa: E402,F401
+                                                    recorded_parity, recorded_traffic, workload_family)
 
 
 # ------------------------------------------------------------------ clocks
@@ -190,12 +150,28 @@ class ClockSampler:
 # ------------------------------------------------------------ CPU oracle
 
 def cpu_threads() -> int:
+    """Threads of the BLAS pool the oracle's matrix products run on."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
         return int(max(n)) if n else 1
     except Exception:
         return 1
+
+
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def single_thread(fn, *a, **kw):
+    """``fn(*a, **kw)`` with the BLAS pool limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(1):
+        return fn(*a, **kw)
 
 
 def oracle_sample_rate(wl, target_s: float, seed: int = 42):
@@ -461,10 +437,91 @@ def run_decode(args):
     if not args.no_cpu_baseline:
         rate, info = decode_oracle_rate(dw, args.cpu_seconds)
         out_line["cpu_baseline"] = {
-            "value": round(rate, 4), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+            "value": round(rate, 4), "unit": "GB/s", "cores": host_cores(), "blas_threads": cpu_threads(),
+            "kind": "oracle",
             "sample": f"{info['q_heads']} query heads over {info['tokens']} cached tokens of one KV head "
                       f"through the float64 oracle in {info['seconds']} s"}
     return out_line
+
+
+class TimedRuns:
+    """CUDA-event durations of the launches of one workload step.
+
+    ``flushed``: the L2 is flushed before every step (outside the events), so
+    each launch starts cold and leaves its dirty lines behind.  Back to back
+    (``flushed=False``) each launch also pays the write-back of the previous
+    launch's outputs, the figure a long stream of such steps sustains.  The
+    stream is held by a bounded device sleep while the host enqueues, so no
+    event brackets host launch latency.
+    """
+
+    def __init__(self, st, stream, steps: int, flusher=None, clocks=None):
+        import torch
+        wl = st.wl
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3 if wl.dequant else 2)]
+              for _ in range(steps)]
+        done = torch.cuda.Event()
+        torch.cuda.synchronize(stream.device)
+        torch.cuda._sleep(hold_cycles(steps))
+        for e in ev:
+            if flusher is not None:
+                flusher()
+            e[0].record(stream)
+            st.quantize(stream)
+            e[1].record(stream)
+            if wl.dequant:
+                st.dequantize(stream)
+                e[2].record(stream)
+        done.record(stream)
+        if clocks is not None:
+            clocks.poll_until(done)
+        torch.cuda.synchronize(stream.device)
+        self.quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+        self.dequant_ms = [e[1].elapsed_time(e[2]) for e in ev] if wl.dequant else []
+        self.step_ms = [q + d for q, d in zip(self.quant_ms, self.dequant_ms or [0.0] * steps)]
+
+
+def kernel_name(wl) -> str:
+    from hadamard_rotation_outlier_b200 import binding as B
+    if wl.kron_a:
+        return KRON_KERNELS[B.hadq_kron_plan(0, wl.rows, wl.kron_a, wl.dim // wl.kron_a, wl.bits, wl.group)]
+    if wl.asym:
+        return "rq_chunk_asym_kernel"
+    return KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)]
+
+
+def dequant_kernel_name(wl) -> str:
+    from hadamard_rotation_outlier_b200 import binding as B
+    if wl.asym:
+        return "dq_chunk_asym_kernel"
+    path = B.hadq_plan(1, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)
+    return {"chunk": "dq_chunk_kernel", "blocked": "dq_blocked_kernel", "generic": "dq_generic_kernel"}.get(path, path)
+
+
+def bandwidth(nbytes: int, ms: float, peak: float) -> dict:
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"avg_launch_ms": round(ms, 5), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+            "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4)}
+
+
+def config_entry(wl, flushed: TimedRuns, sustained: TimedRuns, peak: float) -> dict:
+    """One per_config entry: the quantise kernel (and the dequantiser) of a
+    workload, flushed and back to back."""
+    avg = lambda v: sum(v) / len(v)
+    q_bytes = wl.quant_bytes()
+    fam = workload_family(wl)
+    e = {"workload": wl.name, "kernel": kernel_name(wl), "bytes": q_bytes,
+         **bandwidth(q_bytes, avg(flushed.quant_ms), peak),
+         "rows_per_s": round(wl.rows / (avg(flushed.quant_ms) * 1e-3), 1),
+         "traffic": recorded_traffic(wl.name, fam),
+         "sustained": bandwidth(q_bytes, avg(sustained.quant_ms), peak),
+         "parity": recorded_parity(wl.name, fam)}
+    if wl.dequant:
+        d_bytes = wl.dequant_bytes(2)
+        e["dequant"] = {"kernel": dequant_kernel_name(wl), "bytes": d_bytes,
+                        **bandwidth(d_bytes, avg(flushed.dequant_ms), peak),
+                        "sustained": bandwidth(d_bytes, avg(sustained.dequant_ms), peak)}
+    return e
 
 
 def run_ours(args):
@@ -485,6 +542,7 @@ def run_ours(args):
     warmup = max(3, args.warmup)
     steps = max(1, args.steps)
     dev = torch.device("cuda", local if world > 1 else 0)
+    peak, peak_kind = measured_peaks()
 
     st = WorkloadStep(wl, dev, pinned_host=True)
     flusher = L2Flush(dev)
@@ -496,47 +554,52 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
 
     # ---- device-resident timed region ----
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    qends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)] if wl.dequant else None
-    done = torch.cuda.Event()
     clocks = ClockSampler(dev.index)
     _barrier(world)
     torch.cuda.synchronize(dev)
     n0 = B.hadq_launch_count()
-    # Hold the stream with a bounded device sleep (outside every step's events)
-    # while the host enqueues all steps, so no step's events bracket host-side
-    # launch latency.
-    torch.cuda._sleep(hold_cycles(steps))
-    for i in range(steps):
-        flusher()
-        starts[i].record(stream)
-        st.quantize(stream)
-        if wl.dequant:
-            qends[i].record(stream)
-            st.dequantize(stream)
-        ends[i].record(stream)
-    done.record(stream)
-    clocks.poll_until(done)
-    torch.cuda.synchronize(dev)
+    timed = TimedRuns(st, stream, steps, flusher, clocks)
     _barrier(world)
     launches = B.hadq_launch_count() - n0
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = _max_over_ranks(world, sum(step_ms))
-    quant_ms = ([s.elapsed_time(e) for s, e in zip(starts, qends)] if wl.dequant else step_ms)
+    total_ms = _max_over_ranks(world, sum(timed.step_ms))
+
+    # ---- the same launches back to back, no flush (sustained) ----
+    sustained = TimedRuns(st, stream, min(steps, max(1, args.config_steps)))
 
     # ---- end to end through the public API with host buffers ----
     e2e = run_e2e(st, stream, args.e2e_steps, world)
 
+    headline = config_entry(wl, timed, sustained, peak) if rank == 0 else None
+    del st
+
+    # ---- every configuration the target is stated on ----
+    per_config = None
+    if not args.no_per_config:
+        per_config = []
+        for name in PER_CONFIG:
+            if name == wl.name:
+                per_config.append(headline)
+                continue
+            cw = S.WORKLOADS[name]
+            cs = WorkloadStep(cw, dev)
+            for _ in range(3):
+                flusher()
+                cs.step(stream)
+            n = max(1, args.config_steps)
+            f = TimedRuns(cs, stream, n, flusher)
+            b = TimedRuns(cs, stream, n)
+            if rank == 0:
+                per_config.append(config_entry(cw, f, b, peak))
+            del cs
+            torch.cuda.empty_cache()
+        _barrier(world)
+
     if rank != 0:
         return None
-    bytes_step = st.bytes_per_step
+    bytes_step = wl.quant_bytes() + (wl.dequant_bytes(2) if wl.dequant else 0)
     value = aggregate_gbs(world, bytes_step, steps, total_ms)
-    peak, peak_kind = measured_peaks()
-    q_bytes = wl.quant_bytes()
-    q_ms = sum(quant_ms) / len(quant_ms)
-    achieved = q_bytes / (q_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(wl.name, workload_family(wl))
+    q_ms = sum(timed.quant_ms) / steps
+    achieved = wl.quant_bytes() / (q_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -561,29 +624,42 @@ def run_ours(args):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": (KRON_KERNELS[B.hadq_kron_plan(0, wl.rows, wl.kron_a, wl.dim // wl.kron_a, wl.bits,
-                                                     wl.group)] if wl.kron_a else
-                       "rq_chunk_asym_kernel" if wl.asym else
-                       KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group,
-                                                wl.with_signs, True)]),
+            "kernel": headline["kernel"],
             "achieved": round(achieved, 1), "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
-            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-            "algorithmic_bytes_per_launch": q_bytes, "avg_launch_ms": round(q_ms, 5),
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "nominal_peak": NOMINAL_HBM_GBS,
+            "traffic": headline["traffic"],
+            "algorithmic_bytes_per_launch": wl.quant_bytes(), "avg_launch_ms": round(q_ms, 5),
         },
+        "sustained": {**headline["sustained"],
+                      "note": "the same launches back to back with no L2 flush: each pays the write-back "
+                              "of the previous launch's dirty lines"},
+        "parity": headline["parity"],
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
     if wl.dequant:
-        dq_ms = [e.elapsed_time(f) for e, f in zip(qends, ends)]
-        out["roofline"]["dequant_achieved"] = round(wl.dequant_bytes(2) / (sum(dq_ms) / steps * 1e-3) / 1e9, 1)
+        out["roofline"]["dequant_achieved"] = headline["dequant"]["gbs"]
+    if per_config is not None:
+        out["per_config"] = per_config
     if not args.no_cpu_baseline:
-        rate, info = oracle_sample_rate(wl, args.cpu_seconds)
-        out["cpu_baseline"] = {"value": round(rate, 4), "unit": "GB/s", "cores": cpu_threads(),
-                               "kind": "oracle",
-                               "sample": f"{info['passes']} pass(es) over {info['rows']} rows of {wl.name} "
-                                         f"through the float64 oracle in {info['seconds']} s"}
+        out["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     return out
+
+
+def cpu_baseline(wl, target_s: float) -> dict:
+    """The oracle on a bounded row sample, on every BLAS thread and on one."""
+    r, info = oracle_sample_rate(wl, target_s)
+    r1, info1 = single_thread(oracle_sample_rate, wl, max(1.0, target_s / 2))
+    return {"value": round(r, 4), "unit": "GB/s", "cores": host_cores(), "blas_threads": cpu_threads(),
+            "kind": "oracle",
+            "sample": f"{info['passes']} pass(es) over {info['rows']} rows of {wl.name} "
+                      f"through the float64 oracle in {info['seconds']} s",
+            "single_thread": {"value": round(r1, 4), "unit": "GB/s",
+                              "sample": f"{info1['passes']} pass(es) over {info1['rows']} rows in "
+                                        f"{info1['seconds']} s, BLAS limited to one thread"}}
 
 
 def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
@@ -696,8 +772,22 @@ def run_e2e(st, stream, steps: int, world: int, nchunks: int = 8):
 
 # ------------------------------------------------------------ reference arm
 
+REFERENCE_BUDGET_S = 120.0
+
+
+def reference_step_seconds(args) -> float:
+    """CPU time of one reference-arm step: the whole run (warm-up and timed
+    steps) stays near two minutes, each step between 0.3 s and half the
+    baseline target."""
+    n = max(1, args.steps) + max(0, args.warmup)
+    return max(0.3, min(args.cpu_seconds / 2, REFERENCE_BUDGET_S / n))
+
+
 def run_reference(args):
-    """The CPU oracle as it stands, timed on this host's cores (rank 0 only)."""
+    """The CPU oracle as it stands, timed on this host's cores (rank 0 only).
+
+    Exactly ``--steps`` timed steps after ``--warmup`` untimed ones; each step
+    is one bounded row sample of the workload (see reference_step_seconds)."""
     from hadamard_rotation_outlier_b200 import synthetic as S
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -706,20 +796,16 @@ def run_reference(args):
     if args.workload in S.DECODE_WORKLOADS:
         return run_reference_decode(args, S.DECODE_WORKLOADS[args.workload], world)
     wl = S.WORKLOADS[args.workload]
-    steps = max(1, args.steps if args.steps <= 5 else 3)
-    target = max(1.0, args.cpu_seconds / 2)
-    for _ in range(max(0, min(args.warmup, 1))):
-        oracle_sample_rate(wl, 0.5)
-    rates, infos = [], []
-    for _ in range(steps):
-        r, info = oracle_sample_rate(wl, target)
-        rates.append(r)
-        infos.append(info)
+    steps = max(1, args.steps)
+    target = reference_step_seconds(args)
+    for _ in range(max(0, args.warmup)):
+        oracle_sample_rate(wl, target)
+    infos = [oracle_sample_rate(wl, target)[1] for _ in range(steps)]
     total_bytes = sum(i["bytes"] for i in infos)
     total_s = sum(i["seconds"] for i in infos)
     value = total_bytes / total_s / 1e9
     sample = (f"{steps} steps, each {infos[0]['passes']} pass(es) over {infos[0]['rows']} rows of {wl.name} "
-              f"through the float64 oracle (numpy, dense matrix products)")
+              f"through the float64 oracle (numpy, dense matrix products), about {target:.1f} s of CPU each")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": steps, "warmup": args.warmup,
@@ -727,8 +813,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "rows": wl.rows, "dim": wl.dim, "block": wl.block,
                    "group": wl.group, "bits": wl.bits, "signs": wl.with_signs},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
-                         "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": host_cores(),
+                         "blas_threads": cpu_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -736,13 +822,11 @@ def run_reference(args):
 
 
 def run_reference_decode(args, dw, world):
-    steps = max(1, args.steps if args.steps <= 5 else 3)
-    target = max(1.0, args.cpu_seconds / 2)
-    rates, infos = [], []
-    for _ in range(steps):
-        r, info = decode_oracle_rate(dw, target)
-        rates.append(r)
-        infos.append(info)
+    steps = max(1, args.steps)
+    target = reference_step_seconds(args)
+    for _ in range(max(0, args.warmup)):
+        decode_oracle_rate(dw, target)
+    infos = [decode_oracle_rate(dw, target)[1] for _ in range(steps)]
     total_bytes = sum(i["bytes"] for i in infos)
     total_s = sum(i["seconds"] for i in infos)
     value = total_bytes / total_s / 1e9
@@ -755,8 +839,8 @@ def run_reference_decode(args, dw, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": dw.name, "batch": dw.batch, "n_q_heads": dw.n_q_heads,
                    "n_kv_heads": dw.n_kv_heads, "tokens": dw.tokens, "dim": dw.dim},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cpu_threads(),
-                         "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": host_cores(),
+                         "blas_threads": cpu_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

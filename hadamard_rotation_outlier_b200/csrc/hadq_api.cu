@@ -12,6 +12,7 @@
 #include <mutex>
 #include <string>
 #include <unordered_map>
+#include <vector>
 
 #include "../../include/hadq.h"
 #include "hadq_asym.cuh"
@@ -128,27 +129,47 @@ int sm_count() {
   return n;
 }
 
-// Resident CTAs per SM for (kernel, threads, dynamic smem), cached per device.
-int resident(const void* fn, int threads, size_t smem) {
-  static std::mutex mu;
-  static std::unordered_map<std::string, int> cache;
+// One launch configuration per (device, kernel, block size, dynamic shared
+// memory): the dynamic shared memory above the 48 KB default is reserved and
+// the resident CTAs per SM are read once; later calls only find the entry.
+struct LaunchEntry {
+  int dev;
+  const void* fn;
+  int threads;
+  size_t smem;
+  int resident;
+};
+std::mutex g_launch_mu;
+std::vector<LaunchEntry> g_launch_cache;
+
+hadq_status prepare(const void* fn, int threads, size_t smem, const char* what, int* resident_out) {
   int dev = 0;
   cudaGetDevice(&dev);
-  char key[96];
-  snprintf(key, sizeof key, "%d:%p:%d:%zu", dev, fn, threads, smem);
   {
-    std::lock_guard<std::mutex> lk(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    for (const LaunchEntry& e : g_launch_cache)
+      if (e.dev == dev && e.fn == fn && e.threads == threads && e.smem == smem) {
+        *resident_out = e.resident;
+        return HADQ_OK;
+      }
+  }
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(HADQ_ERR_CUDA, "%s: cannot reserve %zu bytes of shared memory: %s", what, smem,
+                  cudaGetErrorString(e));
+    }
   }
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess || n < 1) {
     cudaGetLastError();
     n = 1;
   }
-  std::lock_guard<std::mutex> lk(mu);
-  cache[key] = n;
-  return n;
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  g_launch_cache.push_back({dev, fn, threads, smem, n});
+  *resident_out = n;
+  return HADQ_OK;
 }
 
 hadq_status after_launch(const char* what) {
@@ -188,7 +209,10 @@ hadq_status launch_blocked(int direction, const Shape& s, hadq::BlockedArgs a, b
   a.tpr = p.tpr;
   const void* fn = hadq::blocked_kernel_ptr(direction, s.bits, s.B, s.has_signs, f32, p.threads);
   const size_t smem = direction == 0 ? p.smem : 0;
-  const int64_t cap = int64_t(resident(fn, p.threads, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, p.threads, smem, "blocked kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
   const unsigned grid = (unsigned)(p.nslabs < cap ? p.nslabs : cap);
   void* args[] = {&a};
   cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(p.threads), args, smem, stream);
@@ -225,13 +249,11 @@ hadq_status launch_chunk_args(int direction, const Shape& s, hadq::ChunkKeepArgs
     fn = direction == 0 ? hadq::chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G >= hadq::kCK, team)
                         : hadq::dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, s.G < s.B, f32);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, direction == 0 && team != 32);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(HADQ_ERR_CUDA, "chunk kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                cudaGetErrorString(e));
-  }
-  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, hadq::kCT, smem, "chunk kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  cudaError_t e;
   const int64_t teams = team == 32 ? hadq::kCT / 32 : 1;
   const int64_t want = ((a.nchunks + a.slab_chunks - 1) / a.slab_chunks + teams - 1) / teams;  // CTAs for one slab per team
   const unsigned grid = (unsigned)(want < cap ? want : cap);
@@ -261,13 +283,11 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
   a.gpc = 1;
   const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, a.rot != nullptr);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, false, false);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(HADQ_ERR_CUDA, "128-block tensor-core kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                cudaGetErrorString(e));
-  }
-  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, hadq::kCT, smem, "128-block tensor-core kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  cudaError_t e;
   const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab of 32 blocks per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
@@ -291,13 +311,11 @@ hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stre
   const void* fn = mma ? hadq::h4096_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr) : hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
   const size_t smem = mma ? hadq::h4096_smem_bytes(s.has_signs) : hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
   const int threads = mma ? hadq::kH4096Warps * 32 : hadq::kCT;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(HADQ_ERR_CUDA, "4096-block kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                cudaGetErrorString(e));
-  }
-  const int64_t cap = int64_t(resident(fn, threads, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, threads, smem, "4096-block kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  cudaError_t e;
   const int64_t want = (a.nchunks / 32 + threads / 32 - 1) / (threads / 32);  // one block per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
@@ -316,7 +334,10 @@ hadq_status launch_full4096(const Shape& s, hadq::FullArgs a, cudaStream_t strea
   a.rows = s.rows;
   const int lg = ilog2(s.G);
   const void* fn = hadq::full4096_kernel_ptr(s.bits, s.has_signs, lg);
-  const int64_t cap = int64_t(resident(fn, 64, 0)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, 64, 0, "4096-point kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
   const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
   void* args[] = {&a};
   cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(64), args, 0, stream);
@@ -345,15 +366,10 @@ hadq_status launch_generic(int direction, const Shape& s, hadq::GenericArgs a, b
     fn = hadq::generic_kernel_ptr(1, s.bits);
     smem = size_t(s.dim) * 4 + ((size_t(s.dim / s.B) + 15) & ~size_t(15));
   }
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(HADQ_ERR_CUDA, "generic kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                  cudaGetErrorString(e));
-    }
-  }
-  const int64_t cap = int64_t(resident(fn, 256, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, 256, smem, "generic kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
   const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
   cudaError_t e;
   if (direction == 0) {
@@ -454,7 +470,10 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
   // One wave of CTAs: split the tokens of each head group so that all CTAs
   // are resident at once (a CTA beyond the wave would run alone afterwards);
   // at least 64 tokens (a tile per warp) per split.
-  const int64_t wave = int64_t(resident(fn, hadq::kAttnThreads, 0)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, hadq::kAttnThreads, 0, "decode attention kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t wave = int64_t(res) * sm_count();
   int64_t splits = wave / as.groups;
   if (splits > as.max_splits) splits = as.max_splits;
   if (splits < 1) splits = 1;
@@ -812,13 +831,11 @@ static hadq_status launch_asym(int direction, const Shape& s, hadq::ChunkAsymArg
   const void* fn = direction == 0 ? hadq::asym_chunk_kernel_ptr(s.bits, s.B, s.has_signs)
                                   : hadq::asym_dq_chunk_kernel_ptr(s.bits, s.B, s.has_signs, f32);
   const size_t smem = hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(HADQ_ERR_CUDA, "asymmetric kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                cudaGetErrorString(e));
-  }
-  const int64_t cap = int64_t(resident(fn, hadq::kCT, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, hadq::kCT, smem, "asymmetric kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  cudaError_t e;
   const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
@@ -917,13 +934,11 @@ static hadq_status launch_kron(int direction, const Shape& s, hadq::KronArgs k, 
                                                 : hadq::kron_kernel_ptr(direction, s.bits);
   const int threads = variant == HADQ_KRON_SMEM ? 256 : s.dim / 16;
   const size_t smem = variant == HADQ_KRON_MMA ? hadq::kron_tc_smem_bytes(k.a, s.B) : hadq::kron_smem_bytes(s.dim, k.a);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(HADQ_ERR_CUDA, "Kronecker kernel: cannot reserve %zu bytes of shared memory: %s", smem,
-                cudaGetErrorString(e));
-  }
-  const int64_t cap = int64_t(resident(fn, threads, smem)) * sm_count();
+  int res = 1;
+  const hadq_status pst = prepare(fn, threads, smem, "Kronecker kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  cudaError_t e;
   const unsigned grid = (unsigned)(s.rows < cap ? s.rows : cap);
   if (direction == 0) {
     void* args[] = {&k};

@@ -2,8 +2,9 @@
 
 Runs last: it checks that the scratch counters are left at zero by every call,
 so that later calls in the same process see a clean scratch.  Each call is
-compared with the float64 oracle, and device memory is checked to be
-unchanged across calls (nothing allocated per call).
+compared with the float64 oracle, and memory is checked to be unchanged across
+calls (nothing allocated per call): torch's allocator always, the device-wide
+free memory when no other process is on the device.
 """
 
 import numpy as np
@@ -20,6 +21,18 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 DIM = 128
+
+
+def _alone_on_device() -> bool:
+    """True when NVML lists at most one compute process on device 0 (this one),
+    so that the device-wide free-memory figure reflects only this process."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+        return len(pynvml.nvmlDeviceGetComputeRunningProcesses(h)) <= 1
+    except Exception:
+        return False
 
 
 def _dev(a):
@@ -58,7 +71,10 @@ def test_noalloc_matches_oracle_and_allocates_nothing(batch, nqh, nkv, tokens, w
     torch.cuda.synchronize()
     assert B.hadq_launch_count() == n0 + 3
     assert torch.cuda.memory_allocated() == alloc0
-    assert torch.cuda.mem_get_info()[0] == free0
+    if _alone_on_device():
+        # a device allocation takes at least one 2 MiB page; other processes
+        # on the device would move this figure, so it is read only when alone
+        assert torch.cuda.mem_get_info()[0] > free0 - (2 << 20)
     check_attention(out.cpu().numpy(), want, allow, "no-alloc entry")
 
 
