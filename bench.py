@@ -495,7 +495,8 @@ def dequant_kernel_name(wl) -> str:
     if wl.asym:
         return "dq_chunk_asym_kernel"
     path = B.hadq_plan(1, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)
-    return {"chunk": "dq_chunk_kernel", "blocked": "dq_blocked_kernel", "generic": "dq_generic_kernel"}.get(path, path)
+    return {"chunk_mma": "dq_chunk_mma_kernel", "chunk": "dq_chunk_kernel", "blocked": "dq_blocked_kernel",
+            "generic": "dq_generic_kernel"}.get(path, path)
 
 
 def bandwidth(nbytes: int, ms: float, peak: float) -> dict:

@@ -20,6 +20,7 @@
 #include "hadq_blocked.cuh"
 #include "hadq_chunk.cuh"
 #include "hadq_chunk_mma.cuh"
+#include "hadq_dq_mma.cuh"
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
 #include "hadq_h4096.cuh"
@@ -102,7 +103,9 @@ bool chunk_ok(int direction, const Shape& s) {
 
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
-  if (aligned16 && direction == 0 && s.B == 128 && s.G == 128 && s.dim % 128 == 0 && !s.has_signs)
+  if (aligned16 && direction == 0 && s.B == 128 && s.G == 128 && s.dim % 128 == 0)
+    return HADQ_PATH_CHUNK_MMA;
+  if (aligned16 && direction == 1 && s.B == 128 && s.G % 128 == 0 && s.dim % 128 == 0)
     return HADQ_PATH_CHUNK_MMA;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
   if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096)
@@ -130,8 +133,10 @@ int sm_count() {
 }
 
 // One launch configuration per (device, kernel, block size, dynamic shared
-// memory): the dynamic shared memory above the 48 KB default is reserved and
-// the resident CTAs per SM are read once; later calls only find the entry.
+// memory): the resident CTAs per SM are read once; later calls only find the
+// entry.  The dynamic shared-memory limit is an attribute of the kernel, not
+// of a launch, so it is raised to the largest size any call has needed (a
+// smaller launch of the same kernel stays valid under a larger limit).
 struct LaunchEntry {
   int dev;
   const void* fn;
@@ -139,26 +144,39 @@ struct LaunchEntry {
   size_t smem;
   int resident;
 };
+struct SmemLimit {
+  int dev;
+  const void* fn;
+  size_t smem;
+};
 std::mutex g_launch_mu;
 std::vector<LaunchEntry> g_launch_cache;
+std::vector<SmemLimit> g_smem_limits;
 
 hadq_status prepare(const void* fn, int threads, size_t smem, const char* what, int* resident_out) {
   int dev = 0;
   cudaGetDevice(&dev);
-  {
-    std::lock_guard<std::mutex> lk(g_launch_mu);
-    for (const LaunchEntry& e : g_launch_cache)
-      if (e.dev == dev && e.fn == fn && e.threads == threads && e.smem == smem) {
-        *resident_out = e.resident;
-        return HADQ_OK;
-      }
-  }
+  std::lock_guard<std::mutex> lk(g_launch_mu);
+  for (const LaunchEntry& e : g_launch_cache)
+    if (e.dev == dev && e.fn == fn && e.threads == threads && e.smem == smem) {
+      *resident_out = e.resident;
+      return HADQ_OK;
+    }
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-      cudaGetLastError();
-      return fail(HADQ_ERR_CUDA, "%s: cannot reserve %zu bytes of shared memory: %s", what, smem,
-                  cudaGetErrorString(e));
+    SmemLimit* lim = nullptr;
+    for (SmemLimit& l : g_smem_limits)
+      if (l.dev == dev && l.fn == fn) lim = &l;
+    if (!lim || lim->smem < smem) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(HADQ_ERR_CUDA, "%s: cannot reserve %zu bytes of shared memory: %s", what, smem,
+                    cudaGetErrorString(e));
+      }
+      if (lim)
+        lim->smem = smem;
+      else
+        g_smem_limits.push_back({dev, fn, smem});
     }
   }
   int n = 0;
@@ -166,7 +184,6 @@ hadq_status prepare(const void* fn, int threads, size_t smem, const char* what, 
     cudaGetLastError();
     n = 1;
   }
-  std::lock_guard<std::mutex> lk(g_launch_mu);
   g_launch_cache.push_back({dev, fn, threads, smem, n});
   *resident_out = n;
   return HADQ_OK;
@@ -281,8 +298,8 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
   a.dim = s.dim;
   a.log_g = 7;
   a.gpc = 1;
-  const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, a.rot != nullptr);
-  const size_t smem = hadq::chunk_smem_bytes(s.dim, false, false);
+  const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr);
+  const size_t smem = hadq::chunk_mma_smem_bytes(s.dim, s.has_signs);
   int res = 1;
   const hadq_status pst = prepare(fn, hadq::kCT, smem, "128-block tensor-core kernel", &res);
   if (pst != HADQ_OK) return pst;
@@ -298,6 +315,32 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
     return fail(HADQ_ERR_CUDA, "128-block tensor-core kernel launch failed: %s", cudaGetErrorString(e));
   }
   return after_launch("128-block tensor-core kernel");
+}
+
+hadq_status launch_dq_chunk_mma(const Shape& s, hadq::ChunkArgs a, bool f32, cudaStream_t stream) {
+  a.cpr = s.dim / hadq::kCK;
+  a.nchunks = s.rows * a.cpr;
+  a.slab_chunks = 32;
+  a.G = s.G;
+  a.dim = s.dim;
+  a.log_g = -1;
+  a.gpc = s.G / hadq::kCK;
+  const void* fn = hadq::dq_chunk_mma_kernel_ptr(s.bits, s.has_signs, f32);
+  const size_t smem = hadq::dq_mma_smem_bytes(s.bits, s.dim, s.has_signs);
+  int res = 1;
+  const hadq_status pst = prepare(fn, hadq::kCT, smem, "128-block tensor-core inverse", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = int64_t(res) * sm_count();
+  const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab of 32 blocks per warp
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  void* args[] = {&a};
+  cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "128-block tensor-core inverse launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("128-block tensor-core inverse");
 }
 
 hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream, bool mma) {
@@ -592,6 +635,7 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
   if (path == HADQ_PATH_CHUNK_MMA) {
     hadq::ChunkArgs a{};
     a.x = static_cast<const uint16_t*>(x);
+    a.signs = signs;
     a.codes = static_cast<uint8_t*>(codes);
     a.scales = scales;
     a.rot = rotated_out;
@@ -652,6 +696,16 @@ hadq_status hadq_dequant_rotate_inv(const void* codes, const float* scales, int6
   const hadq_path path = choose_path(1, s, a16);
   const float rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == HADQ_PATH_CHUNK_MMA) {
+    hadq::ChunkArgs a{};
+    a.codes_in = static_cast<const uint8_t*>(codes);
+    a.scales_in = scales;
+    a.signs = signs;
+    a.rot = f32 ? static_cast<float*>(out) : nullptr;
+    a.out_bf16 = f32 ? nullptr : static_cast<uint16_t*>(out);
+    a.rsqrt_b = rsqrt_b;
+    return launch_dq_chunk_mma(s, a, f32, cs);
+  }
   if (path == HADQ_PATH_CHUNK) {
     hadq::ChunkArgs a{};
     a.codes_in = static_cast<const uint8_t*>(codes);

@@ -1,5 +1,6 @@
-// Forward 128-point Hadamard blocks with one scale per block (G = B = 128,
-// no sign vector) with the first 16-point stage on tensor cores.
+// Forward 128-point Hadamard blocks with one scale per block (G = B = 128),
+// optionally preceded by a +-1 sign vector, with the first 16-point stage on
+// tensor cores.
 //
 // H_128 = H_8 (x) H_16 on the index split j = 16 p + q of a block.  The bf16
 // input is exact in bf16 and H_16 holds only +-1, so the transform along q is
@@ -19,6 +20,17 @@
 //   3. per block: maximum over the lane's 32 outputs and a two-step shuffle
 //      over the block's four lanes, scale, codes into the block's slot;
 //   4. the usual coalesced copy-out of the codes.
+//
+// Signs.  The sign of an element flips the sign bit of its bf16 value, so it
+// is an XOR on the A fragments before the MMA (the products stay exact).  A
+// lane's fragments of tile row p hold columns 16 p + 2 t4 (+1) and 16 p + 8 +
+// 2 t4 (+1) of its two blocks; over the eight p those are 32 sign bits per
+// block and lane quarter t4.  A per-CTA table keeps them as two words per
+// (column block, t4), bit 15 - p and bit 31 - p holding the pair of tile row
+// p, so the mask of a fragment register is (word << p) & 0x80008000: a shift
+// and one three-input logic operation.  Each lane reads the four table
+// entries of its blocks once per slab; the blocks of a slab span rows, so a
+// block's column position is its chunk index modulo the chunks per row.
 #pragma once
 
 #include "hadq_chunk.cuh"
@@ -26,9 +38,30 @@
 
 namespace hadq {
 
+// Shared-memory bytes of the sign-word table: one uint2 per (column block, t4).
+__host__ __device__ inline size_t chunk_mma_sign_bytes(int dim) { return size_t(dim / 128) * 4 * sizeof(uint2); }
+__host__ __device__ inline size_t chunk_mma_smem_bytes(int dim, bool signs) {
+  return size_t(2) * chunk_stage_bytes() + (signs ? chunk_mma_sign_bytes(dim) : 0);
+}
+
+// Sign-word table of one row (all threads; the caller synchronises): entry
+// (cb, t4) = {W0, W1}, W0 bit 15 - p / 31 - p = sign of column 16 p + 2 t4 /
+// + 1 of block cb negative, W1 the same for columns 16 p + 8 + 2 t4 / + 1.
+__device__ __forceinline__ void load_mma_sign_words(const int8_t* signs, int cpr, uint2* sw) {
+  for (int e = threadIdx.x; e < cpr * 4; e += blockDim.x) {
+    const int8_t* s = signs + (e >> 2) * 128 + 2 * (e & 3);
+    uint32_t w0 = 0, w1 = 0;
+    for (int p = 0; p < 8; ++p) {
+      w0 |= (uint32_t)(s[16 * p] < 0) << (15 - p) | (uint32_t)(s[16 * p + 1] < 0) << (31 - p);
+      w1 |= (uint32_t)(s[16 * p + 8] < 0) << (15 - p) | (uint32_t)(s[16 * p + 9] < 0) << (31 - p);
+    }
+    sw[e] = make_uint2(w0, w1);
+  }
+}
+
 // ROT: also write the rotated float32 values (a.rot); a separate instance so
 // that the codes-only kernel carries no registers for them.
-template <int BITS, bool ROT>
+template <int BITS, bool SIGNS, bool ROT>
 __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
   using T = Team<32>;
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
@@ -36,6 +69,14 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int tt = T::tid();
   const int g = tt >> 2, t4 = tt & 3;
+  const uint2* s_sw = reinterpret_cast<const uint2*>(smem + 2 * chunk_stage_bytes());
+  if constexpr (SIGNS) {
+    load_mma_sign_words(a.signs, a.cpr, reinterpret_cast<uint2*>(smem + 2 * chunk_stage_bytes()));
+    __syncthreads();
+  }
+  // column block of this warp's first slab block, advanced from slab to slab
+  int colc = SIGNS ? (int)((T::first() * 32) % a.cpr) : 0;
+  const int col_step = SIGNS ? (int)((T::stride() * 32) % a.cpr) : 0;
 
   // B fragments of H_16 (bf16 +-1) with permuted columns: in n-tile nt,
   // column g holds output n = 4 (g >> 1) + 2 nt + (g & 1); k = 2 t4 + 8 kh
@@ -73,6 +114,18 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
       cp_async_commit();
     }
     const int nch = slab_count(c, a.nchunks, 32);  // blocks beyond nch hold stale data: computed, never stored
+    // sign words of this lane's blocks g + 8 r + 16 grp (index 2 grp + r)
+    uint2 sgw[4];
+    if constexpr (SIGNS) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t cb = (uint32_t)(colc + g + 8 * i);  // i = 2 grp + r: block offset 16 grp + 8 r
+        cb = a.cpr >= 32 ? (cb >= (uint32_t)a.cpr ? cb - a.cpr : cb) : cb % (uint32_t)a.cpr;
+        sgw[i] = s_sw[cb * 4 + t4];
+      }
+      colc += col_step;
+      if (colc >= a.cpr) colc -= a.cpr;
+    }
 
     // 1. H_16 along q: u[64 grp + 8 p + 4 r + e] = output n = 4 t4 + e of row
     // p of block 16 grp + g + 8 r
@@ -84,6 +137,12 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
       for (int p = 0; p < 8; ++p) {
         uint32_t a0, a1, a2, a3;
         ldsm_x4(cur_s + lm_off + uint32_t(grp * 16 * kCPad + p * 32), a0, a1, a2, a3);
+        if constexpr (SIGNS) {  // a0 / a2: block g (+16 grp), a1 / a3: block g + 8
+          a0 ^= (sgw[2 * grp].x << p) & 0x80008000u;
+          a1 ^= (sgw[2 * grp + 1].x << p) & 0x80008000u;
+          a2 ^= (sgw[2 * grp].y << p) & 0x80008000u;
+          a3 ^= (sgw[2 * grp + 1].y << p) & 0x80008000u;
+        }
         float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         mma_bf16_k16(d0, a0, a1, a2, a3, hb[0][0], hb[0][1]);
         mma_bf16_k16(d1, a0, a1, a2, a3, hb[1][0], hb[1][1]);

@@ -30,9 +30,12 @@ const void* kron_tc_kernel_ptr(int bits, int ka, bool pm1, bool s256);
 // Asymmetric (zero-point) variants (groups of 128 x 2^k columns, warp teams).
 const void* asym_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* asym_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
-// 128-point blocks, one scale per block, no signs: first 16-point stage on
-// tensor cores (warp teams of 32 blocks).
-const void* chunk_mma_kernel_ptr(int bits, bool rot);
+// 128-point blocks, one scale per block, with or without signs: first
+// 16-point stage on tensor cores (warp teams of 32 blocks).
+const void* chunk_mma_kernel_ptr(int bits, bool signs, bool rot);
+// Inverse of 128-point blocks whose scale group covers whole blocks: first
+// 16-point stage on tensor cores (f16 MMA on the integer codes).
+const void* dq_chunk_mma_kernel_ptr(int bits, bool signs, bool f32);
 // 4096-column blocks, one scale per block, one block per warp.
 const void* wide4096_kernel_ptr(int bits, bool signs);
 // The same with the first 16-point stage on tensor cores (kH4096Warps warps).

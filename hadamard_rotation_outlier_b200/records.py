@@ -27,7 +27,8 @@ ROOT = os.path.dirname(PKG)
 KERNEL_SOURCES = {
     "quant": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_blocked.cuh", "hadq_full4096.cuh",
               "hadq_generic.cuh", "hadq_mma.cuh", "hadq_chunk_mma.cuh", "k_blocked.cu", "k_chunk.cu",
-              "k_chunk_dq4.cu", "k_chunk_dq8.cu", "k_chunk_mma.cu", "k_full4096.cu", "k_generic.cu"],
+              "k_chunk_dq4.cu", "k_chunk_dq8.cu", "k_chunk_mma.cu", "k_full4096.cu", "k_generic.cu",
+              "hadq_dq_mma.cuh", "k_dq_mma.cu"],
     "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
     "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],

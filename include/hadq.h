@@ -77,10 +77,13 @@ typedef enum {
   HADQ_PATH_WIDE4096_MMA = 6, /* the same blocks (dim = 4096 when signs are
                               given) with the first 16-point stage as a bf16
                               tensor-core MMA against H_16                  */
-  HADQ_PATH_CHUNK_MMA = 7  /* forward, 128-point blocks with one scale per
-                              block and no signs: the first 16-point stage
-                              as a bf16 MMA over 16 blocks at a time, the
-                              other three in registers                      */
+  HADQ_PATH_CHUNK_MMA = 7  /* 128-point blocks, signs or none, the first
+                              16-point stage as an MMA over 16 blocks at a
+                              time and the other three in registers.
+                              Forward (one scale per block): bf16 MMA on
+                              the input, signs as XOR masks on its operand.
+                              Inverse (scale groups of whole blocks): f16
+                              MMA on the integer codes                      */
 } hadq_path;
 
 /* Kernel variant of a Kronecker-rotation call (see hadq_kron_plan). */

@@ -80,9 +80,14 @@ def test_plan_rejects(lib, args, msg):
     (0, 16, 8192, 4096, 4, 4096, False, True, "wide4096_mma"),    # two 4096 blocks, no signs
     (0, 16384, 4096, -1, 4, 128, True, True, "full4096"),         # 4096 block, group 128
     (0, 2097152, 128, 128, 4, 128, False, True, "chunk_mma"),     # KV cache
-    (1, 2097152, 128, 128, 4, 128, False, True, "chunk"),         # KV dequant
+    (1, 2097152, 128, 128, 4, 128, False, True, "chunk_mma"),     # KV dequant
+    (1, 32768, 11008, 128, 4, 128, True, True, "chunk_mma"),      # dequant of 86 signed blocks
+    (1, 100, 4096, 128, 8, -1, False, True, "chunk_mma"),         # dequant, one scale over 32 blocks
+    (1, 100, 768, 128, 4, 384, True, True, "chunk_mma"),          # dequant, groups of 3 blocks
+    (1, 100, 256, 128, 4, 64, False, True, "chunk"),              # dequant, groups inside a block
+    (1, 100, 1024, 64, 4, 128, False, True, "chunk"),             # dequant, 64-point blocks
     (1, 10, 1024, 256, 4, 64, False, True, "blocked"),            # 256-point dequant
-    (0, 32768, 11008, 128, 4, 128, True, True, "chunk"),          # 86 blocks of 128
+    (0, 32768, 11008, 128, 4, 128, True, True, "chunk_mma"),      # 86 blocks of 128, signs
     (0, 10, 1024, 256, 4, 64, True, True, "blocked"),             # 256-point blocks
     (0, 10, 96, 32, 8, -1, False, True, "blocked"),               # dim not a multiple of 128
     (0, 10, 32768, 128, 4, -1, False, True, "generic"),           # whole-row groups past 16384
@@ -90,7 +95,7 @@ def test_plan_rejects(lib, args, msg):
     (0, 10, 4096, -1, 4, 32, False, True, "generic"),             # small groups on 4096
     (0, 10, 8192, -1, 4, -1, False, True, "generic"),             # 8192-point block
     (0, 10, 32768, 128, 4, 128, False, True, "chunk_mma"),        # widest row, group 128
-    (0, 10, 32768, 128, 4, 128, True, True, "chunk"),             # the same with signs
+    (0, 10, 32768, 128, 4, 128, True, True, "chunk_mma"),         # the same with signs
     (0, 10, 256, 128, 4, 64, False, True, "chunk"),               # groups smaller than the block
     (0, 10, 12, 4, 8, 3, False, True, "generic"),
     (1, 10, 4096, -1, 4, -1, True, True, "generic"),              # 4096 dequant

@@ -80,8 +80,13 @@ CASES = [
     (1, 128, 128, 128, 4, False, "chunk_mma"),      # one block
     (65, 1024, 128, 128, 8, False, "chunk_mma"),
     (37, 4096, 128, -1, 4, False, "chunk"),         # per-token scale over 32 blocks
-    (9, 11008, 128, 128, 4, True, "chunk"),         # 86 blocks, signs
-    (45, 1152, 128, 128, 8, True, "chunk"),         # signs, 9 blocks per row, a short last slab
+    (9, 11008, 128, 128, 4, True, "chunk_mma"),     # 86 blocks, signs
+    (45, 1152, 128, 128, 8, True, "chunk_mma"),     # signs, 9 blocks per row, a short last slab
+    (300, 128, 128, 128, 8, True, "chunk_mma"),     # signs, one block per row (every block at column 0)
+    (77, 384, 128, 128, 4, True, "chunk_mma"),      # signs, 3 blocks per row: slabs start at every column
+    (41, 4096, 128, 128, 4, True, "chunk_mma"),     # signs, exactly one slab per row
+    (23, 2560, 128, 128, 8, True, "chunk_mma"),     # signs, 20 blocks per row (< one slab)
+    (13, 5248, 128, 128, 4, True, "chunk_mma"),     # signs, 41 blocks per row (> one slab, < two)
     (5, 11008, 128, -1, 8, True, "chunk"),          # 86 blocks, one scale per row
     (300, 256, 32, 8, 4, False, "chunk"),           # groups smaller than a block
     (70, 512, 64, 16, 8, True, "chunk"),
@@ -91,7 +96,8 @@ CASES = [
     (30, 768, 128, 384, 4, False, "chunk"),         # groups of 3 chunks (CTA shared-memory max)
     (3, 16384, 128, -1, 4, True, "chunk"),          # one row per slab
     (33, 1152, 8, 64, 8, False, "chunk"),           # 8-point blocks, 9 chunks per row
-    (5, 32768, 128, 128, 4, True, "chunk"),         # widest row, groups inside chunks
+    (5, 32768, 128, 128, 4, True, "chunk_mma"),     # widest row, signs (largest sign-word table)
+    (5, 32768, 128, 64, 4, True, "chunk"),          # widest row, groups inside chunks
     (33, 1024, 256, 64, 4, True, "blocked"),        # 256-point blocks
     (17, 768, 256, -1, 8, False, "blocked"),        # row of three 256-blocks
     (6, 8192, 256, 1024, 8, True, "blocked"),
@@ -241,8 +247,9 @@ def test_wide4096_mma_edge_rows(bits, with_signs):
     run_case(len(rows), dim, -1, -1, bits, with_signs, seed=12, x_bits=x)
 
 
-@pytest.mark.parametrize("dim,bits", [(128, 8), (384, 4)])
-def test_chunk_mma_edge_rows(dim, bits):
+@pytest.mark.parametrize("dim,bits,with_signs", [(128, 8, False), (384, 4, False), (384, 8, True),
+                                                (11008, 4, True)])
+def test_chunk_mma_edge_rows(dim, bits, with_signs):
     # the tensor-core 128 path: zero, one-hot, tiny (1e-30, bf16 subnormal
     # 1e-39), huge (1e30) and spiky rows; 40 rows = one full slab of 32
     # blocks plus a short one.  A block with K spikes of 5e3 puts pre-round
@@ -257,5 +264,5 @@ def test_chunk_mma_edge_rows(dim, bits):
             np.where(rng.random(dim) < 0.02, 5e3, rng.normal(size=dim)).astype(np.float32)]
     rows = base + [rng.normal(size=dim).astype(np.float32) for _ in range(40 - len(base))]
     x = S.f32_to_bf16_bits(np.stack(rows))
-    assert B.hadq_plan(0, len(rows), dim, 128, bits, 128, False, True) == "chunk_mma"
-    run_case(len(rows), dim, 128, 128, bits, False, seed=13, x_bits=x, max_mismatches=16)
+    assert B.hadq_plan(0, len(rows), dim, 128, bits, 128, with_signs, True) == "chunk_mma"
+    run_case(len(rows), dim, 128, 128, bits, with_signs, seed=13, x_bits=x, max_mismatches=16)
