@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
       const int64_t nx = slab + T::stride();
       if (nx < nslabs) chunk_load<16, 32>(xsrc + nx * 32 * 256, slab_count(nx * 32, a.nchunks, 32), (it & 1) ? st0 : st1, tt);
       cp_async_commit();
+      const int64_t n2 = nx + T::stride();  // the slab after: into L2 now, staged next iteration
+      if (tt == 0 && n2 < nslabs) prefetch_l2_bulk(xsrc + n2 * 32 * 256, uint32_t(slab_count(n2 * 32, a.nchunks, 32)) * 256u);
     }
     const int nch = slab_count(c, a.nchunks, 32);  // blocks beyond nch hold stale data: computed, never stored
     // sign words of this lane's blocks g + 8 r + 16 grp (index 2 grp + r)
@@ -200,17 +202,26 @@ __global__ void __launch_bounds__(kCT, 3) rq_chunk_mma_kernel(ChunkArgs a) {
             for (int e = 0; e < 4; ++e) v[8 * p + e] *= 18446744073709551616.0f;
         }
         uint8_t* slot = cur + b * kCPad;
+        if constexpr (BITS == 8) {
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          uint32_t c0, c1, c2, c3;
-          magic_code2(v[8 * p], v[8 * p + 1], q.inv, c0, c1);
-          magic_code2(v[8 * p + 2], v[8 * p + 3], q.inv, c2, c3);
-          const uint32_t w = pack_i8x4(c0, c1, c2, c3);  // outputs 16 p + 4 t4 .. + 3
-          if constexpr (BITS == 8) {
-            *reinterpret_cast<uint32_t*>(slot + 16 * p + 4 * t4) = w;
-          } else {
-            const uint32_t nb = (w & 0x000F000Fu) | ((w >> 4) & 0x00F000F0u);  // nibble pairs in bytes 0 and 2
-            *reinterpret_cast<uint16_t*>(slot + 8 * p + 2 * t4) = (uint16_t)__byte_perm(nb, 0, 0x0020);
+          for (int p = 0; p < 8; ++p) {
+            uint32_t c0, c1, c2, c3;
+            magic_code2(v[8 * p], v[8 * p + 1], q.inv, c0, c1);
+            magic_code2(v[8 * p + 2], v[8 * p + 3], q.inv, c2, c3);
+            *reinterpret_cast<uint32_t*>(slot + 16 * p + 4 * t4) = pack_i8x4(c0, c1, c2, c3);  // outputs 16 p + 4 t4 .. + 3
+          }
+        } else {
+          // rows p and p + 1 in one word: its low half holds outputs 16 p + 4 t4 .. + 3, the high half those of p + 1
+#pragma unroll
+          for (int p = 0; p < 8; p += 2) {
+            uint32_t cc[8];
+            magic_code2(v[8 * p], v[8 * p + 1], q.inv, cc[0], cc[1]);
+            magic_code2(v[8 * p + 2], v[8 * p + 3], q.inv, cc[2], cc[3]);
+            magic_code2(v[8 * p + 8], v[8 * p + 9], q.inv, cc[4], cc[5]);
+            magic_code2(v[8 * p + 10], v[8 * p + 11], q.inv, cc[6], cc[7]);
+            const uint32_t wd = pack_i4x8(cc);
+            *reinterpret_cast<uint16_t*>(slot + 8 * p + 2 * t4) = (uint16_t)(wd & 0xffffu);
+            *reinterpret_cast<uint16_t*>(slot + 8 * p + 8 + 2 * t4) = (uint16_t)(wd >> 16);
           }
         }
       }

@@ -220,6 +220,13 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// Bulk prefetch of a global range into L2 (no data comes back to the SM):
+// 16-byte-aligned address, size a multiple of 16 bytes.  A warp issues it for
+// the slab after the one it is staging, so that the staging copy hits L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Code multiplier of one group: inv = qmax / m, or, for a group maximum so
 // small that this overflows, qmax / (m * 2^64) applied to v * 2^64.
 struct QInv {

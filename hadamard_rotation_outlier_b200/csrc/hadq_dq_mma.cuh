@@ -182,6 +182,9 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
         dq_mma_load<BITS>(a.codes_in + nf * 32 * L::CB, slab_count(nf * 32, a.nchunks, 32),
                           wbase + ((it + L::NS - 1) % L::NS) * 32 * L::CP, lane);
       cp_async_commit();
+      const int64_t n2 = nf + wstride;  // the slab after: into L2 now, staged next iteration
+      if (lane == 0 && n2 < nslabs)
+        prefetch_l2_bulk(a.codes_in + n2 * 32 * L::CB, uint32_t(slab_count(n2 * 32, a.nchunks, 32)) * L::CB);
       const int64_t nx = slab + wstride;
 #pragma unroll
       for (int i = 0; i < 4; ++i) sc_next[i] = nx < nslabs ? block_scale(nx * 32 + g + 8 * i) : 0.0f;
