@@ -294,22 +294,24 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
 hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
   a.cpr = s.dim / hadq::kCK;
   a.nchunks = s.rows * a.cpr;
-  a.slab_chunks = 32;
+  a.slab_chunks = hadq::kMmaSlab;
   a.G = s.G;
   a.dim = s.dim;
   a.log_g = 7;
   a.gpc = 1;
   const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr);
   const size_t smem = hadq::chunk_mma_smem_bytes(s.dim, s.has_signs);
+  const int threads = hadq::kMmaWarps * 32;
   int res = 1;
-  const hadq_status pst = prepare(fn, hadq::kCT, smem, "128-block tensor-core kernel", &res);
+  const hadq_status pst = prepare(fn, threads, smem, "128-block tensor-core kernel", &res);
   if (pst != HADQ_OK) return pst;
   const int64_t cap = int64_t(res) * sm_count();
   cudaError_t e;
-  const int64_t want = ((a.nchunks + 31) / 32 + 3) / 4;  // one slab of 32 blocks per warp
+  const int64_t slabs = (a.nchunks + hadq::kMmaSlab - 1) / hadq::kMmaSlab;
+  const int64_t want = (slabs + hadq::kMmaWarps - 1) / hadq::kMmaWarps;  // one slab per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
-  e = cudaLaunchKernel(fn, dim3(grid), dim3(hadq::kCT), args, smem, stream);
+  e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
     g_launches.fetch_add(1, std::memory_order_relaxed);

@@ -6,14 +6,16 @@
 // 256 consecutive elements; warp w of the pair takes the tiles with T bit 3 =
 // w (j11), so a lane owns eight tiles t = T & 7 (bits 8-10).
 //
-// 1. Load.  A lane reads 16 bytes per tile straight from global memory into
-//    registers: elements o = 8 lane + e (e = 0..7) of the tile, o = 32 g +
-//    8 t4 + e.  Those 8 bf16 values are exactly the lane's A fragment of one
+// 1. Load.  A lane copies 16 bytes per tile into the pair's staging buffer
+//    (cp.async) and reads them back into registers: elements o = 8 lane + e
+//    (e = 0..7) of the tile, o = 32 g + 8 t4 + e.  Those 8 bf16 values are
+//    exactly the lane's A fragment of one
 //    m16n8k16 MMA when the tile is a 16 x 16 matrix with rows m = g + 8 e2 and
 //    columns k = 2 t4 + e0 + 8 e1: bits j0, j1, j3, j4 are the MMA's k (the
-//    "q" bits it transforms), j2 and j5-j7 its rows.  The next block of the
-//    pair is prefetched into L2 with one bulk prefetch while this one is
-//    computed, so the loads hit L2.
+//    "q" bits it transforms), j2 and j5-j7 its rows.  A lane stages only its
+//    own pieces, so the staging needs no barrier: the next block's copy is
+//    issued as soon as this block's pieces went through the MMAs, and the
+//    block after that is prefetched into L2 with one bulk prefetch.
 // 2. Signs.  The element signs flip bf16 sign bits: an XOR on the fragments
 //    (the products stay exact).  Each lane's 64 sign bits are two words built
 //    once per CTA; the mask of register r of tile t is (word << i) &
@@ -41,7 +43,7 @@
 namespace hadq {
 
 constexpr int kH4PairsPerCta = 2;              // warp pairs (blocks in flight) per CTA
-constexpr int kH4PairFloats = 4096 + 8;        // transpose buffer + two pairs of max slots
+constexpr int kH4PairFloats = 4096 + 8 + 2048;  // transpose buffer, two pairs of max slots, staging (8 KB)
 
 __host__ __device__ inline size_t h4096p_smem_bytes() { return size_t(kH4PairsPerCta) * kH4PairFloats * sizeof(float); }
 
@@ -106,15 +108,29 @@ __global__ void __launch_bounds__(kH4PairsPerCta * 64, 4) rq_h4096_pair_kernel(C
   const int64_t pstride = int64_t(gridDim.x) * kH4PairsPerCta;
   const uint16_t* x = a.x;
   int parity = 0;
-  for (int64_t blk = int64_t(blockIdx.x) * kH4PairsPerCta + pair; blk < nblk; blk += pstride, parity ^= 1) {
-    if (w == 0 && lane == 0 && blk + pstride < nblk) prefetch_l2_bulk(x + (blk + pstride) * 4096, 8192);
-    // 1-3. load, signs, H_16 on tensor cores
+  int64_t blk = int64_t(blockIdx.x) * kH4PairsPerCta + pair;
+  // staging: a lane's 16-byte piece of tile t of the pair's block sits at
+  // uint4 index 256 w + 32 t + lane (the piece's own offset in the block);
+  // each lane copies in and reads back only its own pieces, so no barrier
+  uint4* stg = reinterpret_cast<uint4*>(buf + 4096 + 8) + 256 * w + lane;
+  auto stage_in = [&](int64_t k) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + k * 4096 + 2048 * w) + lane;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) cp_async16(stg + 32 * t, src + 32 * t);
+  };
+  if (blk < nblk) stage_in(blk);
+  cp_async_commit();
+  if (w == 0 && lane == 0 && blk + pstride < nblk) prefetch_l2_bulk(x + (blk + pstride) * 4096, 8192);
+  for (; blk < nblk; blk += pstride, parity ^= 1) {
+    // the block after the next one into L2 (it is staged during the next block)
+    if (w == 0 && lane == 0 && blk + 2 * pstride < nblk) prefetch_l2_bulk(x + (blk + 2 * pstride) * 4096, 8192);
+    cp_async_wait<0>();
+    // 1-3. signs, H_16 on tensor cores
     float u[64];
     {
-      const uint4* src = reinterpret_cast<const uint4*>(x + blk * 4096 + 2048 * w) + lane;
       uint4 f[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) f[t] = __ldg(src + 32 * t);
+      for (int t = 0; t < 8; ++t) f[t] = stg[32 * t];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         uint32_t a0 = f[t].x, a2 = f[t].y, a1 = f[t].z, a3 = f[t].w;
@@ -139,6 +155,9 @@ __global__ void __launch_bounds__(kH4PairsPerCta * 64, 4) rq_h4096_pair_kernel(C
         u[8 * t + 7] = d1[3];
       }
     }
+    // the MMAs have consumed this lane's pieces: its slots take the next block
+    if (blk + pstride < nblk) stage_in(blk + pstride);
+    cp_async_commit();
     // 4. j2, j8, j9, j10
     reg_stage<64, 4>(u);
     reg_stage<64, 8>(u);
