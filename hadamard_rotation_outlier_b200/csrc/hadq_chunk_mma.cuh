@@ -31,7 +31,9 @@
 // p, so the mask of a fragment register is (word << p) & 0x80008000: a shift
 // and one three-input logic operation.  Each lane reads the two table
 // entries of its blocks once per slab; the blocks of a slab span rows, so a
-// block's column position is its block index modulo the blocks per row.
+// block's column position is its block index modulo the blocks per row, and
+// the table repeats its first 16 entries after the last so that the slab's
+// start column plus the block offset indexes it directly.
 #pragma once
 
 #include "hadq_chunk.cuh"
@@ -39,15 +41,19 @@
 
 namespace hadq {
 
-// Shared-memory bytes of the sign-word table: one uint2 per (column block, t4).
-__host__ __device__ inline size_t chunk_mma_sign_bytes(int dim) { return size_t(dim / 128) * 4 * sizeof(uint2); }
+// Shared-memory bytes of the sign-word table: one uint2 per (entry, t4), with
+// entries for the column blocks 0 .. cpr - 1 followed by 16 more that repeat
+// them (entry e holds column block e mod cpr), so that a slab's column
+// positions colc + b (colc < cpr, b < 16) index it without a modulo.
+__host__ __device__ inline size_t chunk_mma_sign_bytes(int dim) { return size_t(dim / 128 + 16) * 4 * sizeof(uint2); }
 
 // Sign-word table of one row (all threads; the caller synchronises): entry
 // (cb, t4) = {W0, W1}, W0 bit 15 - p / 31 - p = sign of column 16 p + 2 t4 /
-// + 1 of block cb negative, W1 the same for columns 16 p + 8 + 2 t4 / + 1.
+// + 1 of column block cb mod cpr negative, W1 the same for columns 16 p + 8 +
+// 2 t4 / + 1; cb runs over cpr + 16 entries.
 __device__ __forceinline__ void load_mma_sign_words(const int8_t* signs, int cpr, uint2* sw) {
-  for (int e = threadIdx.x; e < cpr * 4; e += blockDim.x) {
-    const int8_t* s = signs + (e >> 2) * 128 + 2 * (e & 3);
+  for (int e = threadIdx.x; e < (cpr + 16) * 4; e += blockDim.x) {
+    const int8_t* s = signs + ((e >> 2) % cpr) * 128 + 2 * (e & 3);
     uint32_t w0 = 0, w1 = 0;
     for (int p = 0; p < 8; ++p) {
       w0 |= (uint32_t)(s[16 * p] < 0) << (15 - p) | (uint32_t)(s[16 * p + 1] < 0) << (31 - p);
@@ -164,11 +170,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkAr
     uint2 sgw[2];
     if constexpr (SIGNS) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        uint32_t cb = (uint32_t)(colc + g + 8 * r);
-        cb = a.cpr >= kMmaSlab ? (cb >= (uint32_t)a.cpr ? cb - a.cpr : cb) : cb % (uint32_t)a.cpr;
-        sgw[r] = s_sw[cb * 4 + t4];
-      }
+      for (int r = 0; r < 2; ++r) sgw[r] = s_sw[(colc + g + 8 * r) * 4 + t4];  // colc + g + 8 r < cpr + 16
       colc += col_step;
       if (colc >= a.cpr) colc -= a.cpr;
     }

@@ -116,6 +116,8 @@ __global__ void __launch_bounds__(kH4096Warps * 32, 2) rq_h4096_mma_kernel(Chunk
       const int64_t nx = slab + wstride;
       if (nx < nslabs) chunk_load<16, 32>(xsrc + nx * 32 * 256, 32, (it & 1) ? st0 : st1, lane);
       cp_async_commit();
+      const int64_t n2 = nx + wstride;  // the block after: into L2 now, staged next iteration
+      if (lane == 0 && n2 < nslabs) prefetch_l2_bulk(xsrc + n2 * 32 * 256, 8192u);
     }
 
     // 1. H_16 along q on tensor cores
