@@ -55,7 +55,7 @@ NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, vendor figure
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
-                "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_pair_kernel",
+                "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_mma_kernel",
                 "chunk_mma": "rq_chunk_mma_kernel", "none": None}
 KRON_KERNELS = {"smem": "rq_kron_kernel", "reg16": "rq_kron16_kernel", "mma": "rq_kron_tc_kernel"}
 

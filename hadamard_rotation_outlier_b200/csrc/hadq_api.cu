@@ -24,7 +24,6 @@
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
 #include "hadq_h4096.cuh"
-#include "hadq_h4096p.cuh"
 #include "hadq_kron.cuh"
 #include "hadq_kernels.h"
 
@@ -354,16 +353,15 @@ hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stre
   a.dim = s.dim;
   a.log_g = -1;
   a.gpc = 32;
-  const void* fn = mma ? hadq::h4096_pair_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr) : hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
-  const size_t smem = mma ? hadq::h4096p_smem_bytes() : hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
-  const int threads = mma ? hadq::kH4PairsPerCta * 64 : hadq::kCT;
+  const void* fn = mma ? hadq::h4096_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr) : hadq::wide4096_kernel_ptr(s.bits, s.has_signs);
+  const size_t smem = mma ? hadq::h4096_smem_bytes(s.has_signs) : hadq::chunk_smem_bytes(s.dim, s.has_signs, false);
+  const int threads = mma ? hadq::kH4096Warps * 32 : hadq::kCT;
   int res = 1;
   const hadq_status pst = prepare(fn, threads, smem, "4096-block kernel", &res);
   if (pst != HADQ_OK) return pst;
   const int64_t cap = int64_t(res) * sm_count();
   cudaError_t e;
-  const int64_t per_cta = mma ? hadq::kH4PairsPerCta : threads / 32;  // blocks in flight per CTA
-  const int64_t want = (a.nchunks / 32 + per_cta - 1) / per_cta;
+  const int64_t want = (a.nchunks / 32 + threads / 32 - 1) / (threads / 32);  // one block per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
   void* args[] = {&a};
   e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);

@@ -40,9 +40,6 @@ const void* dq_chunk_mma_kernel_ptr(int bits, bool signs, bool f32);
 const void* wide4096_kernel_ptr(int bits, bool signs);
 // The same with the first 16-point stage on tensor cores (kH4096Warps warps).
 const void* h4096_mma_kernel_ptr(int bits, bool signs, bool rot);
-// The same blocks on warp pairs (two warps per block, loads straight into the
-// MMA fragments, one shared-memory transpose); kH4PairsPerCta pairs per CTA.
-const void* h4096_pair_kernel_ptr(int bits, bool signs, bool rot);
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);
 const void* generic_kernel_ptr(int direction, int bits);
 
