@@ -12,8 +12,8 @@
 //
 // One MMA tile takes 16 blocks of a slab (rows) and the 16 q-values of one
 // p-value (columns).  The codes of a slab (32 consecutive blocks) are staged
-// in shared memory by cp.async, in a ring of NS stages per warp (INT4 codes
-// are only a fifth of the traffic, so a warp keeps two slabs ahead in flight); ldmatrix.x4 over 16-byte segments of the code
+// in shared memory by cp.async, two stages per warp, and the slab after next
+// is prefetched into L2; ldmatrix.x4 over 16-byte segments of the code
 // rows hands each lane 4 bytes of a segment of two blocks, and the choice of
 // which code bits are q bits follows what a lane receives:
 //
@@ -33,8 +33,11 @@
 // of H_16 in the B fragments are ordered so that a lane ends up with runs of
 // consecutive outputs (8 for INT4, 4 for INT8): with the three p stages in
 // registers, each run is converted to bf16, gets its signs, and goes to a
-// per-warp staging row (pitch chosen so the 16- / 8-byte stores are
-// conflict-free), from where the slab leaves with coalesced 16-byte stores.
+// per-warp staging area laid out as the slab is in global memory (8 KB of
+// bf16 rows), which leaves with one bulk asynchronous copy issued by one lane
+// (no per-lane copy-out; the copy engine reads the staging while the warp
+// computes the next slab, and the lane waits for that read before the rows
+// are written again).
 #pragma once
 
 #include "hadq_chunk.cuh"
@@ -46,8 +49,8 @@ template <int BITS>
 struct DqMmaLayout {
   static constexpr int CB = BITS == 8 ? 128 : 64;    // code bytes per block
   static constexpr int CP = CB + 16;                 // code row pitch (ldmatrix rows conflict-free)
-  static constexpr int OP = BITS == 8 ? 288 : 320;   // bf16 output row pitch (run stores conflict-free)
-  static constexpr int NS = BITS == 8 ? 2 : 3;       // code stages: slabs in flight per warp
+  static constexpr int OP = 256;                     // bf16 output rows: the slab's global layout
+  static constexpr int NS = 2;                       // code stages (the slab after next is prefetched into L2)
   static constexpr int WARP_BYTES = NS * 32 * CP + 32 * OP;
 };
 
@@ -269,6 +272,10 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
         reg_stage<64, 8>(u);
         reg_stage<64, 16>(u);
       }
+      if (!OUT_F32 && grp == 0) {  // the previous slab's bulk copy has read the staging rows
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
+      }
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int b = g + 8 * r + 16 * grp;  // block in the slab
@@ -341,26 +348,16 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
       if (colc >= a.cpr) colc -= a.cpr;
     }
     if constexpr (!OUT_F32) {
+      fence_async_shared();  // the run stores are visible to the copy engine
       __syncwarp();
-      // copy-out: 16 lanes per 256-byte block row, two blocks per instruction
-      uint8_t* gdst = reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256;
-      const int half = lane >> 4, piece = lane & 15;
-      if (nch == 32) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int b = 2 * k + half;
-          *reinterpret_cast<uint4*>(gdst + b * 256 + 16 * piece) =
-              *reinterpret_cast<const uint4*>(ostage + b * L::OP + 16 * piece);
-        }
-      } else {
-        for (int b = half; b < nch; b += 2)
-          *reinterpret_cast<uint4*>(gdst + b * 256 + 16 * piece) =
-              *reinterpret_cast<const uint4*>(ostage + b * L::OP + 16 * piece);
+      if (lane == 0) {
+        bulk_store_s2g(reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256, ostage, uint32_t(nch) * 256u);
+        bulk_commit();
       }
     }
-    __syncwarp();  // the staging rows are read before the next slab writes them
   }
   cp_async_wait<0>();
+  if (!OUT_F32 && lane == 0) bulk_wait_all();  // the staging stays valid until the last copy is done
 }
 
 }  // namespace hadq
