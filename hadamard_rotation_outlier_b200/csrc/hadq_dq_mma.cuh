@@ -12,8 +12,8 @@
 //
 // One MMA tile takes 16 blocks of a slab (rows) and the 16 q-values of one
 // p-value (columns).  The codes of a slab (32 consecutive blocks) are staged
-// in shared memory by cp.async, two stages per warp, and the slab after next
-// is prefetched into L2; ldmatrix.x4 over 16-byte segments of the code
+// in shared memory by cp.async, three stages per warp, and the slab after the
+// last staged one is prefetched into L2; ldmatrix.x4 over 16-byte segments of the code
 // rows hands each lane 4 bytes of a segment of two blocks, and the choice of
 // which code bits are q bits follows what a lane receives:
 //
@@ -50,7 +50,7 @@ struct DqMmaLayout {
   static constexpr int CB = BITS == 8 ? 128 : 64;    // code bytes per block
   static constexpr int CP = CB + 16;                 // code row pitch (ldmatrix rows conflict-free)
   static constexpr int OP = 256;                     // bf16 output rows: the slab's global layout
-  static constexpr int NS = 2;                       // code stages (the slab after next is prefetched into L2)
+  static constexpr int NS = 3;                       // code stages per warp (plus the L2 prefetch)
   static constexpr int WARP_BYTES = NS * 32 * CP + 32 * OP;
 };
 
