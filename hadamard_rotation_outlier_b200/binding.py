@@ -264,7 +264,8 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
 
     ``q``: bf16 ``[batch, n_q_heads, dim]``.  ``k_codes``/``v_codes``: uint8
     ``[batch, n_kv_heads, token_stride, dim/2]``; ``k_scales``/``v_scales``:
-    float32 ``[batch, n_kv_heads, token_stride]`` (or with a trailing 1).
+    float32 ``[batch, n_kv_heads, token_stride, dim/group]`` (one scale per row
+    for group 128 or -1, which may drop the trailing 1).
     ``tokens`` (default ``token_stride``) rows of each head are attended over.
     ``workspace``: a zero-filled uint8 CUDA tensor of at least
     :func:`hadq_kv_decode_workspace_size` bytes, reused across calls (one is
@@ -287,8 +288,9 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
         tokens = stride
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
         _need(t, name, torch.uint8, dev)
+    per_scale = dim // _resolve(dim, block, group) if group != 0 and dim % _resolve(dim, block, group) == 0 else 1
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
-        _need(t, name, torch.float32, dev, batch * nkv * stride)
+        _need(t, name, torch.float32, dev, batch * nkv * stride * per_scale)
     if per_row * 2 != dim:
         raise ValueError(f"codes rows hold {per_row} bytes, expected dim/2 = {dim // 2}")
     if signs is not None:
@@ -334,8 +336,9 @@ def hadq_kv_decode_attention_noalloc(q: torch.Tensor, k_codes: torch.Tensor, k_s
     nkv, stride = k_codes.shape[1], k_codes.shape[2]
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
         _need(t, name, torch.uint8, dev)
+    per_scale = dim // _resolve(dim, block, group) if group != 0 and dim % _resolve(dim, block, group) == 0 else 1
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
-        _need(t, name, torch.float32, dev, batch * nkv * stride)
+        _need(t, name, torch.float32, dev, batch * nkv * stride * per_scale)
     if signs is not None:
         _need(signs, "signs", torch.int8, dev, dim)
     if out.dtype not in (torch.bfloat16, torch.float32):

@@ -492,10 +492,11 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
     return fail(HADQ_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
   if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
     return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
-  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || s.G != hadq::kAttnDim || bits != 4)
+  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || (s.G != 128 && s.G != 64 && s.G != 32) || bits != 4)
     return fail(HADQ_ERR_UNSUPPORTED,
-                "decode attention supports dim 128, block 128, group 128, bits 4 (got %d, %d, %d, %d)", dim,
-                s.B, s.G, bits);
+                "decode attention supports dim 128, block 128, group 128, 64 or 32, bits 4 (got %d, %d, %d, %d)",
+                dim, s.B, s.G, bits);
+  const int ng = hadq::kAttnDim / s.G;  // scales per cached row
   if (batch == 0) return HADQ_OK;
   if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || (!workspace && !static_scratch))
     return fail(HADQ_ERR_INVALID_ARG, "q, codes, scales, out and workspace must not be NULL");
@@ -505,13 +506,17 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
     return fail(HADQ_ERR_MISALIGNED, "k_codes and v_codes must be 16-byte aligned");
   if (!aligned(k_scales, 4) || !aligned(v_scales, 4))
     return fail(HADQ_ERR_MISALIGNED, "k_scales and v_scales must be 4-byte aligned");
+  if (ng > 1 && (!aligned(k_scales, 16) || !aligned(v_scales, 16) || (token_stride * ng) % 4 != 0))
+    return fail(HADQ_ERR_MISALIGNED,
+                "with groups below 128 the scale arrays must be 16-byte aligned and token_stride * 128 / group "
+                "a multiple of 4");
   if (signs && !aligned(signs, 4)) return fail(HADQ_ERR_MISALIGNED, "signs must be 4-byte aligned");
   if (!aligned(out, f32 ? 16 : 8))
     return fail(HADQ_ERR_MISALIGNED, "out must be %d-byte aligned", f32 ? 16 : 8);
   if (!static_scratch && !aligned(workspace, 256))
     return fail(HADQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
 
-  const void* fn = hadq::kv_decode_attn_kernel_ptr();
+  const void* fn = hadq::kv_decode_attn_kernel_ptr(ng);
   // One wave of CTAs: split the tokens of each head group so that all CTAs
   // are resident at once (a CTA beyond the wave would run alone afterwards);
   // at least 64 tokens (a tile per warp) per split.

@@ -50,8 +50,11 @@ constexpr int kAttnStages = 4;                                  // ring depth pe
 constexpr int kAttnKRow = 64;                                   // bytes of INT4 codes per token
 constexpr int kAttnVRow = 80;                                   // V row padded in shared memory
 constexpr int kAttnStV = kAttnTile * kAttnKRow;                 // 1024
-constexpr int kAttnStS = kAttnStV + kAttnTile * kAttnVRow;      // 2304: 16 K scales, 16 V scales
-constexpr int kAttnStageBytes = kAttnStS + 2 * kAttnTile * 4;   // 2432
+constexpr int kAttnStS = kAttnStV + kAttnTile * kAttnVRow;      // 2304: K scales, then V scales
+// Bytes of one ring stage: 16 K and 16 V rows, then [16 tokens][NG] K scales
+// and as many V scales (NG = 128 / G scale groups per row).
+__host__ __device__ constexpr int attn_stage_bytes(int ng) { return kAttnStS + 2 * kAttnTile * 4 * ng; }
+constexpr int kAttnStageBytes = attn_stage_bytes(1);            // 2432
 constexpr int kAttnCombPitch = kAttnDim + 4;                    // floats per head in the CTA merge
 constexpr int kAttnMaxSplits = 256;
 constexpr size_t kAttnStaticScratchBytes = size_t(16) << 20;  // scratch of the allocation-free entry
@@ -76,10 +79,10 @@ struct AttnArgs {
   uint32_t vmask, vmagic;    // 0x000F000F and 0x43084308 (see int4x2_to_bf16x2)
 };
 
-template <int STAGES>
+template <int STAGES, int NG>
 struct __align__(16) AttnSmem {
   union {
-    uint8_t stage[kAttnWarps][STAGES][kAttnStageBytes];
+    uint8_t stage[kAttnWarps][STAGES][attn_stage_bytes(NG)];
     float comb[kAttnWarps][kAttnHeads][kAttnCombPitch];
   } u;
   int8_t qd[4][kAttnHeads][kAttnDim];  // query digits [digit][head][dim]; digit 3 stays 0
@@ -170,9 +173,18 @@ __device__ __forceinline__ void int4x8_to_s8x16(uint32_t w, uint32_t& even, uint
 }
 
 // STAGES: depth of each warp's cp.async ring (tiles in flight + 1).
-template <int STAGES>
+// NG: scale groups per cached row (128 / G: 1, 2 or 4).  With NG = 1 a k-step
+// of the score MMA spans the four 32-dim quarters of the row; with NG > 1 it
+// spans one quarter, so that each quarter (a group of 32, or half a group of
+// 64) has its own integer accumulator and is weighted by its own key scale,
+// and the value codes are taken four dims per quarter so that every n8 tile
+// of the P.V product lies inside one group (the A operand p * vscale is cut
+// once per group).
+template <int STAGES, int NG>
 __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const AttnArgs a) {
-  __shared__ AttnSmem<STAGES> sm;
+  static_assert(NG == 1 || NG == 2 || NG == 4, "groups of 128, 64 or 32 columns");
+  constexpr int SB = attn_stage_bytes(NG);
+  __shared__ AttnSmem<STAGES, NG> sm;
   const int tid = threadIdx.x;
   const int w = tid >> 5;
   const int lane = tid & 31;
@@ -257,16 +269,18 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
 
   // A operands of the QK product for k-step s: lane (g, j) holds rows g and
   // g+8 (head g & 3, digits g >> 2 and (g >> 2) + 2) at the dims
-  // 32j + 8s + {0,2,4,6} (a0, a1) and 32j + 8s + {1,3,5,7} (a2, a3), the same
-  // dims the key operand of that lane carries.
+  // d0 + {0,2,4,6} (a0, a1) and d0 + {1,3,5,7} (a2, a3), d0 = 32j + 8s (one
+  // scale group) or 32s + 8j (NG > 1), the same dims the key operand of that
+  // lane carries.
   uint32_t qa[4][4];
   const int hh = g & 3;
   {
     const int dr0 = g >> 2, dr1 = (g >> 2) + 2;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      const uint2 r0 = *reinterpret_cast<const uint2*>(&sm.qd[dr0][hh][32 * j + 8 * s]);
-      const uint2 r1 = *reinterpret_cast<const uint2*>(&sm.qd[dr1][hh][32 * j + 8 * s]);
+      const int d0 = NG == 1 ? 32 * j + 8 * s : 32 * s + 8 * j;  // this lane's 8 dims of k-step s
+      const uint2 r0 = *reinterpret_cast<const uint2*>(&sm.qd[dr0][hh][d0]);
+      const uint2 r1 = *reinterpret_cast<const uint2*>(&sm.qd[dr1][hh][d0]);
       qa[s][0] = __byte_perm(r0.x, r0.y, 0x6420);
       qa[s][1] = __byte_perm(r1.x, r1.y, 0x6420);
       qa[s][2] = __byte_perm(r0.x, r0.y, 0x7531);
@@ -306,10 +320,16 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   const uint8_t* g_k = kc + lane_tok * kAttnKRow + cpart * 16;
   const uint8_t* g_v = vc + lane_tok * kAttnKRow + cpart * 16;
   const float* g_s = (lane < 16 ? ksc : vsc) + t_begin + int64_t(w) * kAttnTile + (lane & 15);
+  // NG > 1: scales [token][NG] per array; lane p < 4 NG copies K piece p,
+  // lanes 4 NG .. 8 NG - 1 the V pieces (16 bytes = 4 / NG tokens each)
+  const int sg_piece = lane % (4 * NG);
+  const int sg_tok = sg_piece * 4 / NG;  // first token of this lane's piece in the tile
+  const uint32_t d_sg = kAttnStS + (lane < 4 * NG ? 0u : uint32_t(kAttnTile * 4 * NG)) + 16u * uint32_t(sg_piece);
+  const float* g_sg = (lane < 4 * NG ? ksc : vsc) + (t_begin + int64_t(w) * kAttnTile) * NG + 4 * sg_piece;
   constexpr int64_t kStepTok = int64_t(kAttnWarps) * kAttnTile;  // tokens between a warp's tiles
 
   auto issue = [&](int k) {
-    const uint32_t st = s_ring + uint32_t(k % STAGES) * kAttnStageBytes;
+    const uint32_t st = s_ring + uint32_t(k % STAGES) * SB;
     const int64_t adv = int64_t(k) * kStepTok;
     const int r0 = (w + kAttnWarps * k) * kAttnTile;  // first token of the tile, from t_begin
     if (r0 + kAttnTile <= n_tok) {
@@ -317,7 +337,11 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
       cp_async16(st + d_k + 8 * kAttnKRow, g_k + (adv + 8) * kAttnKRow);
       cp_async16(st + d_v, g_v + adv * kAttnKRow);
       cp_async16(st + d_v + 8 * kAttnVRow, g_v + (adv + 8) * kAttnKRow);
-      cp_async4(st + d_s, g_s + adv);
+      if constexpr (NG == 1) {
+        cp_async4(st + d_s, g_s + adv);
+      } else if (lane < 8 * NG) {  // 4 NG pieces of 16 bytes of K scales, then as many of V
+        cp_async16(st + d_sg, g_sg + adv * NG);
+      }
     } else {  // ragged last tile: rows past t_end are zero-filled, never read
       // (their source address is replaced by the first row of the head).
       const bool v0 = r0 + ctok < n_tok, v1 = r0 + ctok + 8 < n_tok;
@@ -327,7 +351,15 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
       cp_async16_zfill(st + d_k + 8 * kAttnKRow, v1 ? g_k + (adv + 8) * kAttnKRow : kc, v1);
       cp_async16_zfill(st + d_v, v0 ? g_v + adv * kAttnKRow : vc, v0);
       cp_async16_zfill(st + d_v + 8 * kAttnVRow, v1 ? g_v + (adv + 8) * kAttnKRow : vc, v1);
-      cp_async4_zfill(st + d_s, vs ? g_s + adv : s0, vs);
+      if constexpr (NG == 1) {
+        cp_async4_zfill(st + d_s, vs ? g_s + adv : s0, vs);
+      } else if (lane < 8 * NG) {  // the piece's tokens past t_end read nothing (zero fill)
+        const int left = (n_tok - r0 - sg_tok) * NG * 4;  // bytes of this piece inside the range
+        const int nb = left <= 0 ? 0 : left >= 16 ? 16 : left;
+        const float* s0g = (lane < 4 * NG) ? ksc : vsc;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(st + d_sg),
+                     "l"(nb > 0 ? g_sg + adv * NG : s0g), "r"(nb) : "memory");
+      }
     }
   };
 
@@ -351,37 +383,63 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     const uint8_t* st = sm.u.stage[w][k % STAGES];
     const int r0 = (w + kAttnWarps * k) * kAttnTile;
 
-    // --- scores: S^T[head x digit, token] = Qdigits . (16 * kcode) ---
-    int c0[4] = {0, 0, 0, 0}, c1[4] = {0, 0, 0, 0};
+    // --- scores: S^T[head x digit, token] = Qdigits . (16 * kcode), one
+    // integer accumulator per scale group (k-steps s with s * NG / 4 = q) ---
+    int c0[NG][4], c1[NG][4];
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c0[q][i] = c1[q][i] = 0;
     {
-      const uint4 k0 = *reinterpret_cast<const uint4*>(st + g * kAttnKRow + 16 * j);
-      const uint4 k1 = *reinterpret_cast<const uint4*>(st + (g + 8) * kAttnKRow + 16 * j);
-      const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
-      const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
+      uint32_t kw0[4], kw1[4];
+      if constexpr (NG == 1) {
+        const uint4 k0 = *reinterpret_cast<const uint4*>(st + g * kAttnKRow + 16 * j);
+        const uint4 k1 = *reinterpret_cast<const uint4*>(st + (g + 8) * kAttnKRow + 16 * j);
+        kw0[0] = k0.x; kw0[1] = k0.y; kw0[2] = k0.z; kw0[3] = k0.w;
+        kw1[0] = k1.x; kw1[1] = k1.y; kw1[2] = k1.z; kw1[3] = k1.w;
+      } else {  // dims 32 s + 8 j .. + 7 = bytes 16 s + 4 j .. + 3 of a row
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          kw0[s] = *reinterpret_cast<const uint32_t*>(st + g * kAttnKRow + 16 * s + 4 * j);
+          kw1[s] = *reinterpret_cast<const uint32_t*>(st + (g + 8) * kAttnKRow + 16 * s + 4 * j);
+        }
+      }
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         uint32_t e, od;
         int4x8_to_s8x16(kw0[s], e, od);
-        mma_s8_16832(c0, qa[s], e, od);
+        mma_s8_16832(c0[s * NG / 4], qa[s], e, od);
         int4x8_to_s8x16(kw1[s], e, od);
-        mma_s8_16832(c1, qa[s], e, od);
+        mma_s8_16832(c1[s * NG / 4], qa[s], e, od);
       }
     }
     // Scores.  Every lane holds digit partials of tokens 2j, 2j+1, 2j+8 and
     // 2j+9 for head g & 3; the lane pair (g, g ^ 4) shares that head, and the
     // low lane (g < 4) finishes tokens 2j, 2j+1 while the high lane finishes
     // 2j+8, 2j+9 (`own`), each adding the partner's partials.
-    const float pl0 = fmaf(float(c0[2]), wh, float(c0[0]) * wl);
-    const float pl1 = fmaf(float(c0[3]), wh, float(c0[1]) * wl);
-    const float pl2 = fmaf(float(c1[2]), wh, float(c1[0]) * wl);
-    const float pl3 = fmaf(float(c1[3]), wh, float(c1[1]) * wl);
-    const float x0 = __shfl_xor_sync(0xffffffffu, low ? pl2 : pl0, 16);
-    const float x1 = __shfl_xor_sync(0xffffffffu, low ? pl3 : pl1, 16);
-    const float* sc = reinterpret_cast<const float*>(st + kAttnStS);
-    const float2 ksp = *reinterpret_cast<const float2*>(sc + own);
-    const float2 vsp = *reinterpret_cast<const float2*>(sc + kAttnTile + own);
-    float sv0 = ((low ? pl0 : pl2) + x0) * (qs * ksp.x);
-    float sv1 = ((low ? pl1 : pl3) + x1) * (qs * ksp.y);
+    const float* sc = reinterpret_cast<const float*>(st + kAttnStS);  // [16][NG] K, then [16][NG] V
+    float sv0 = 0.f, sv1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      const float pl0 = fmaf(float(c0[q][2]), wh, float(c0[q][0]) * wl);
+      const float pl1 = fmaf(float(c0[q][3]), wh, float(c0[q][1]) * wl);
+      const float pl2 = fmaf(float(c1[q][2]), wh, float(c1[q][0]) * wl);
+      const float pl3 = fmaf(float(c1[q][3]), wh, float(c1[q][1]) * wl);
+      const float x0 = __shfl_xor_sync(0xffffffffu, low ? pl2 : pl0, 16);
+      const float x1 = __shfl_xor_sync(0xffffffffu, low ? pl3 : pl1, 16);
+      const float k0s = sc[own * NG + q], k1s = sc[(own + 1) * NG + q];
+      if constexpr (NG == 1) {
+        sv0 = ((low ? pl0 : pl2) + x0) * (qs * k0s);
+        sv1 = ((low ? pl1 : pl3) + x1) * (qs * k1s);
+      } else {
+        sv0 = fmaf((low ? pl0 : pl2) + x0, k0s, sv0);
+        sv1 = fmaf((low ? pl1 : pl3) + x1, k1s, sv1);
+      }
+    }
+    if constexpr (NG > 1) {
+      sv0 *= qs;
+      sv1 *= qs;
+    }
     if (r0 + kAttnTile > n_tok) {  // ragged last tile (warp-uniform): mask the missing tokens
       if (r0 + own >= n_tok) sv0 = -INFINITY;
       if (r0 + own + 1 >= n_tok) sv1 = -INFINITY;
@@ -411,21 +469,25 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     // --- A operand of PV: rows (head, part), part 0/1/2 = hi/mid/lo of
     // p * vscale, part 3 zero.  Lanes g < 4 hold parts 0 and 2, g >= 4 part 1;
     // each lane cut its own two tokens and takes the partner's parts it needs.
-    uint32_t pa[4];
-    {
+    // (NG > 1: one such operand per scale group, with that group's vscale.)
+    uint32_t pa[NG][4];
+    const float* vsc_s = sc + kAttnTile * NG;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
       uint32_t hi, mid, lo;
-      split3_bf16(p0 * vsp.x, p1 * vsp.y, hi, mid, lo);
+      split3_bf16(p0 * vsc_s[own * NG + q], p1 * vsc_s[(own + 1) * NG + q], hi, mid, lo);
       const uint32_t r1 = __shfl_xor_sync(0xffffffffu, low ? mid : hi, 16);
       const uint32_t r2 = __shfl_xor_sync(0xffffffffu, lo, 16);
-      pa[0] = low ? hi : r1;   // row g, tokens 2j, 2j+1
-      pa[1] = low ? lo : 0u;   // row g + 8, tokens 2j, 2j+1
-      pa[2] = low ? r1 : mid;  // row g, tokens 2j+8, 2j+9
-      pa[3] = low ? r2 : 0u;   // row g + 8, tokens 2j+8, 2j+9
+      pa[q][0] = low ? hi : r1;   // row g, tokens 2j, 2j+1
+      pa[q][1] = low ? lo : 0u;   // row g + 8, tokens 2j, 2j+1
+      pa[q][2] = low ? r1 : mid;  // row g, tokens 2j+8, 2j+9
+      pa[q][3] = low ? r2 : 0u;   // row g + 8, tokens 2j+8, 2j+9
     }
 
-    // --- PV: O[(head, part), dim] += P . V; lane (g, j) feeds the value
-    // codes of dims 16g + i (n8 tile i) for tokens 2j, 2j+1 / 2j+8, 2j+9 ---
-    {
+    // --- PV: O[(head, part), dim] += P . V ---
+    if constexpr (NG == 1) {
+      // lane (g, j) feeds the value codes of dims 16g + i (n8 tile i) for
+      // tokens 2j, 2j+1 / 2j+8, 2j+9
       const uint8_t* svp = st + kAttnStV + 8 * g;
       const uint2 va = *reinterpret_cast<const uint2*>(svp + (2 * j) * kAttnVRow);
       const uint2 vb = *reinterpret_cast<const uint2*>(svp + (2 * j + 1) * kAttnVRow);
@@ -438,8 +500,29 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
         const uint32_t xcd = __byte_perm(h < 2 ? vcx.x : vcx.y, h < 2 ? vd.x : vd.y, sel);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          mma_bf16_16816(o[4 * h + e], pa, int4x2_to_bf16x2(xab >> (4 * e), vmask, vmagic),
+          mma_bf16_16816(o[4 * h + e], pa[0], int4x2_to_bf16x2(xab >> (4 * e), vmask, vmagic),
                          int4x2_to_bf16x2(xcd >> (4 * e), vmask, vmagic));
+      }
+    } else {
+      // n8 tile i = 4 qt + r (quarter qt of the row, group qt * NG / 4): lane
+      // (g, j) feeds dim 32 qt + 8 (g >> 1) + 2 r + (g & 1), i.e. nibble g & 1
+      // of byte r of the word at byte 16 qt + 4 (g >> 1) of the token's row
+      const uint8_t* svp = st + kAttnStV + 4 * (g >> 1);
+      const int nsh = 4 * (g & 1);
+#pragma unroll
+      for (int qt = 0; qt < 4; ++qt) {
+        const uint32_t wa = *reinterpret_cast<const uint32_t*>(svp + (2 * j) * kAttnVRow + 16 * qt);
+        const uint32_t wb = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 1) * kAttnVRow + 16 * qt);
+        const uint32_t wc = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 8) * kAttnVRow + 16 * qt);
+        const uint32_t wd = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 9) * kAttnVRow + 16 * qt);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t sel = uint32_t(r | (r << 4) | ((4 + r) << 8) | ((4 + r) << 12));  // byte r of each word
+          const uint32_t xab = __byte_perm(wa, wb, sel) >> nsh;
+          const uint32_t xcd = __byte_perm(wc, wd, sel) >> nsh;
+          mma_bf16_16816(o[4 * qt + r], pa[qt * NG / 4], int4x2_to_bf16x2(xab, vmask, vmagic),
+                         int4x2_to_bf16x2(xcd, vmask, vmagic));
+        }
       }
     }
     __syncwarp();
@@ -465,10 +548,22 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   // the index bits, under which H_128 is unchanged.
   if (g < 4) {
     float* cb = sm.u.comb[w][g];
+    if constexpr (NG == 1) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      cb[8 * i + j] = oa[i];
-      cb[8 * i + 4 + j] = ob[i];
+      for (int i = 0; i < 16; ++i) {
+        cb[8 * i + j] = oa[i];
+        cb[8 * i + 4 + j] = ob[i];
+      }
+    } else {
+      // oa[i] holds dim 32 (i >> 2) + 8 j + 2 (i & 3), ob[i] the next one;
+      // idx(dim) = 8 (dim & 15) + 4 ((dim >> 4) & 1) + (dim >> 5)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int lo = 8 * (j & 1) + 2 * (i & 3);  // (dim & 15) of oa[i]
+        const int idx = 8 * lo + 4 * (j >> 1) + (i >> 2);
+        cb[idx] = oa[i];
+        cb[idx + 8] = ob[i];  // dim + 1: (dim & 15) + 1
+      }
     }
     if (j == 0) {
       sm.m[w][g] = m_run;

@@ -47,9 +47,9 @@ const void* generic_kernel_ptr(int direction, int bits);
 
 namespace hadq {
 
-// Decode attention over the rotated INT4 KV cache (head dim 128, one scale
-// per cached row), 128 threads per CTA.
-const void* kv_decode_attn_kernel_ptr();
+// Decode attention over the rotated INT4 KV cache (head dim 128, ng = 1, 2 or
+// 4 scales per cached row: groups of 128, 64 or 32 columns), 128 threads per CTA.
+const void* kv_decode_attn_kernel_ptr(int ng);
 // Device address (current device) of the library's static attention scratch
 // of kAttnStaticScratchBytes, or NULL if the runtime cannot resolve it.
 void* attn_static_scratch();

@@ -4,7 +4,11 @@
 
 namespace hadq {
 
-const void* kv_decode_attn_kernel_ptr() { return reinterpret_cast<const void*>(&kv_decode_attn_kernel<kAttnStages>); }
+const void* kv_decode_attn_kernel_ptr(int ng) {
+  if (ng == 4) return reinterpret_cast<const void*>(&kv_decode_attn_kernel<kAttnStages, 4>);
+  if (ng == 2) return reinterpret_cast<const void*>(&kv_decode_attn_kernel<kAttnStages, 2>);
+  return reinterpret_cast<const void*>(&kv_decode_attn_kernel<kAttnStages, 1>);
+}
 
 // Scratch of the allocation-free entry point: a static device array, zero
 // when the module loads (so its arrival counters start at zero); every call

@@ -307,8 +307,8 @@ hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales,
  * stored in the rotated basis as INT4 codes.
  *
  * The cache rows are what hadq_rotate_quantize writes for dim 128, block 128
- * (or -1), group 128 (or -1), bits 4 and the same signs: K_rot = (K * s) H and
- * V_rot = (V * s) H, quantised per row.  Because H is orthogonal,
+ * (or -1), group 128 (or -1), 64 or 32, bits 4 and the same signs:
+ * K_rot = (K * s) H and V_rot = (V * s) H, quantised per row or per group.  Because H is orthogonal,
  * (q H)(K H)^T = q K^T ("Hartmann rotation, lightweight QAT, streaming
  * attention", section 1), so the scores come from the rotated query against
  * the dequantised rotated keys, and the output is rotated back once ("QuaRot
@@ -316,23 +316,29 @@ hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales,
  * the output transformed back):
  *
  *   q_rot  = (q * s) H
- *   p      = softmax_t( softmax_scale * q_rot . kcode_t * kscale_t )
+ *   p      = softmax_t( softmax_scale * q_rot . (kcode_t * kscale_t) )
  *   out    = ((sum_t p_t * vcode_t * vscale_t) H) * s
+ *
+ * (kscale_t, vscale_t: the scale of each element's group.)
  *
  *   q            device, bfloat16 [batch, n_q_heads, dim], 8-byte aligned.
  *   k_codes,     device, uint8 [batch, n_kv_heads, token_stride, dim/2] packed
  *   v_codes      INT4 (element 2j in the low nibble of byte j), 16-byte
  *                aligned.  Only the first `tokens` rows of each head are read.
- *   k_scales,    device, float32 [batch, n_kv_heads, token_stride], 4-byte
- *   v_scales     aligned: the per-row scales of the codes.
+ *   k_scales,    device, float32 [batch, n_kv_heads, token_stride, 128/group]:
+ *   v_scales     the per-group scales of the codes (one per row for group 128),
+ *                4-byte aligned; for group 64 or 32, 16-byte aligned with
+ *                token_stride * 128/group a multiple of 4 (HADQ_ERR_MISALIGNED
+ *                otherwise).
  *   batch        >= 0 (0 = empty call).
  *   n_q_heads    >= 1, a multiple of n_kv_heads; query head h reads KV head
  *                h / (n_q_heads / n_kv_heads) (grouped-query attention).
  *   tokens       cached tokens attended over, 1 <= tokens <= token_stride,
  *                at most 2^30 (HADQ_ERR_UNSUPPORTED beyond).
  *   dim, block,  the cache's rotate+quantise parameters; the kernel supports
- *   bits, group  dim 128, block 128 or -1, bits 4, group 128 or -1 and returns
- *                HADQ_ERR_UNSUPPORTED for any other valid combination.
+ *   bits, group  dim 128, block 128 or -1, bits 4, group 128 (or -1), 64 or 32
+ *                and returns HADQ_ERR_UNSUPPORTED for any other valid
+ *                combination.
  *   signs        device int8 [dim] (4-byte aligned) or NULL, as for the cache.
  *   softmax_scale  > 0 and finite (usually 1/sqrt(dim)).
  *   out          device output [batch, n_q_heads, dim]: bfloat16 (8-byte

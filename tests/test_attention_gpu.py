@@ -35,35 +35,37 @@ def _q_tensor(bits):
     return _dev(bits.view(np.int16)).view(torch.bfloat16)
 
 
-def oracle_cache(batch, nkv, stride, seed, with_outliers=True, signs=None):
-    """K and V caches quantised by the oracle from seeded bf16 rows."""
+def oracle_cache(batch, nkv, stride, seed, with_outliers=True, signs=None, group=128):
+    """K and V caches quantised by the oracle from seeded bf16 rows; scales
+    [batch, nkv, stride] for group 128, else [batch, nkv, stride, 128/group]."""
     rows = batch * nkv * stride
     cols = (3, 77, 101) if with_outliers else ()
     kx = S.random_bf16(rows, DIM, seed, outlier_cols=cols, outlier_scale=30.0)
     vx = S.random_bf16(rows, DIM, seed + 1)
-    k = O.rotate_quantize(kx, block=128, signs=signs, bits=4, group=128, method="fwht")
-    v = O.rotate_quantize(vx, block=128, signs=signs, bits=4, group=128, method="fwht")
+    k = O.rotate_quantize(kx, block=128, signs=signs, bits=4, group=group, method="fwht")
+    v = O.rotate_quantize(vx, block=128, signs=signs, bits=4, group=group, method="fwht")
     shape = (batch, nkv, stride)
-    return (k["codes"].reshape(shape + (DIM // 2,)), k["scales"].reshape(shape),
-            v["codes"].reshape(shape + (DIM // 2,)), v["scales"].reshape(shape))
+    sshape = shape if group == 128 else shape + (DIM // group,)
+    return (k["codes"].reshape(shape + (DIM // 2,)), k["scales"].reshape(sshape),
+            v["codes"].reshape(shape + (DIM // 2,)), v["scales"].reshape(sshape))
 
 
-def run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, softmax_scale=None, workspace=None):
+def run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, softmax_scale=None, workspace=None, group=128):
     sg = None if signs is None else _dev(signs)
     out = B.hadq_kv_decode_attention(_q_tensor(qbits), _dev(kc), _dev(ks), _dev(vc), _dev(vs),
-                                     tokens=tokens, block=128, signs=sg, bits=4, group=128,
+                                     tokens=tokens, block=128, signs=sg, bits=4, group=group,
                                      softmax_scale=softmax_scale, out_dtype=out_dtype,
                                      workspace=workspace)
     torch.cuda.synchronize()
     return out
 
 
-def oracle_attention(qbits, kc, ks, vc, vs, signs=None, softmax_scale=None):
+def oracle_attention(qbits, kc, ks, vc, vs, signs=None, softmax_scale=None, group=128):
     """Oracle output and its allowance for the cache rows given."""
-    want = O.kv_decode_attention(qbits, kc, ks, vc, vs, DIM, 128, signs, 4, 128, softmax_scale)
-    scores = O.kv_decode_scores(qbits, kc, ks, DIM, 128, signs, 4, 128, softmax_scale)
-    nb, nkv, T = ks.shape
-    values = O.dequant_rotate_inv(vc.reshape(-1, DIM // 2), vs.reshape(-1), DIM, 128, signs, 4, 128,
+    want = O.kv_decode_attention(qbits, kc, ks, vc, vs, DIM, 128, signs, 4, group, softmax_scale)
+    scores = O.kv_decode_scores(qbits, kc, ks, DIM, 128, signs, 4, group, softmax_scale)
+    nb, nkv, T = ks.shape[:3]
+    values = O.dequant_rotate_inv(vc.reshape(-1, DIM // 2), vs.reshape(-1), DIM, 128, signs, 4, group,
                                   method="fwht").reshape(nb, nkv, T, DIM)
     return want, attention_allowance(want, scores, values, qbits.shape[1] // nkv)
 
@@ -197,3 +199,58 @@ def test_full_size_decode_sampled_heads():
                                 vc[:, kvh:kvh + 1], vs[:, kvh:kvh + 1])
         compare(out[:, sl].contiguous(), want, torch.bfloat16, f"full size, KV head {kvh}")
     assert torch.isfinite(out.float()).all()
+
+
+GROUP_CASES = [
+    # batch, n_q_heads, n_kv_heads, tokens, stride, signs, group (the cache's scale group)
+    (1, 4, 1, 1, 4, False, 64),        # one cached token
+    (1, 8, 2, 300, 300, False, 64),    # GQA 4
+    (1, 8, 2, 45, 46, True, 64),       # ragged tail, stride > tokens
+    (2, 8, 2, 37, 40, True, 32),       # ragged tail, groups of 32
+    (1, 32, 8, 1000, 1000, True, 32),  # GQA 4 with signs
+    (1, 16, 2, 513, 520, False, 32),   # two head groups per KV head
+    (1, 8, 1, 5000, 5000, False, 64),  # many splits
+]
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("batch,nqh,nkv,tokens,stride,with_signs,group", GROUP_CASES)
+def test_decode_attention_grouped_cache(batch, nqh, nkv, tokens, stride, with_signs, group, out_dtype):
+    # caches quantised with 2 or 4 scales per row (groups of 64 or 32 columns)
+    seed = 2000 + batch * 7 + nqh * 13 + tokens + group
+    signs = S.random_signs(DIM, seed) if with_signs else None
+    kc, ks, vc, vs = oracle_cache(batch, nkv, stride, seed, signs=signs, group=group)
+    qbits = S.decode_query(batch, nqh, DIM, seed)
+    want = oracle_attention(qbits, kc[:, :, :tokens], ks[:, :, :tokens], vc[:, :, :tokens],
+                            vs[:, :, :tokens], signs, group=group)
+    out = run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, group=group)
+    compare(out, want, out_dtype, f"attention G={group} {batch}x{nqh}/{nkv} T={tokens}")
+
+
+def test_grouped_cache_with_one_group_matches_row_scales():
+    # scales given as [.., 4] with all four equal must give the same output as
+    # the one-scale-per-row cache (the grouped path reduces to the row path)
+    kc, ks, vc, vs = oracle_cache(1, 2, 700, 9)
+    qbits = S.decode_query(1, 8, DIM, 9)
+    a = run_gpu(qbits, kc, ks, vc, vs, 700, None, torch.float32)
+    ks4 = np.repeat(ks[..., None], 4, axis=-1)
+    vs4 = np.repeat(vs[..., None], 4, axis=-1)
+    b = run_gpu(qbits, kc, ks4, vc, vs4, 700, None, torch.float32, group=32)
+    want = oracle_attention(qbits, kc, ks, vc, vs)
+    compare(b, want, torch.float32, "G=32 with equal group scales")
+    np.testing.assert_allclose(b.cpu().numpy(), a.cpu().numpy(), rtol=2e-6, atol=1e-6)
+
+
+def test_grouped_cache_rejections():
+    q = torch.zeros((1, 4, DIM), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, 1, 7, DIM // 2), dtype=torch.uint8, device="cuda")
+    ks2 = torch.ones((1, 1, 7, 2), dtype=torch.float32, device="cuda")
+    n0 = B.hadq_launch_count()
+    with pytest.raises(B.HadqError) as e:   # groups of 64 need token_stride * 2 to be a multiple of 4
+        B.hadq_kv_decode_attention(q, kc, ks2, kc, ks2, block=128, bits=4, group=64)
+    assert e.value.status == B.HADQ_ERR_MISALIGNED
+    ks8 = torch.ones((1, 1, 7, 8), dtype=torch.float32, device="cuda")
+    with pytest.raises(B.HadqError) as e:   # groups of 16 are not supported
+        B.hadq_kv_decode_attention(q, kc, ks8, kc, ks8, block=128, bits=4, group=16)
+    assert e.value.status == B.HADQ_ERR_UNSUPPORTED
+    assert B.hadq_launch_count() == n0
