@@ -56,7 +56,7 @@ L2_FLUSH_BYTES = 256 << 20
 KERNEL_NAMES = {"blocked": "rq_blocked_kernel", "full4096": "rq_full4096_kernel",
                 "generic": "rq_generic_kernel", "chunk": "rq_chunk_kernel",
                 "wide4096": "rq_wide4096_kernel", "wide4096_mma": "rq_h4096_mma_kernel",
-                "chunk_mma": "rq_chunk_mma_kernel", "none": None}
+                "chunk_mma": "rq_chunk_mma_kernel", "h4096_tc": "rq_h4096_tc_kernel", "none": None}
 KRON_KERNELS = {"smem": "rq_kron_kernel", "reg16": "rq_kron16_kernel", "mma": "rq_kron_tc_kernel"}
 
 

@@ -17,9 +17,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhadq.so")
 
-HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA = range(5)
+HADQ_OK, HADQ_ERR_INVALID_ARG, HADQ_ERR_UNSUPPORTED, HADQ_ERR_MISALIGNED, HADQ_ERR_CUDA, HADQ_ERR_DEVICE = range(6)
 HADQ_OUT_BF16, HADQ_OUT_F32 = 0, 1
-PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096", 6: "wide4096_mma", 7: "chunk_mma"}
+PATH_NAMES = {0: "none", 1: "blocked", 2: "full4096", 3: "generic", 4: "chunk", 5: "wide4096", 6: "wide4096_mma", 7: "chunk_mma", 8: "h4096_tc"}
 KRON_VARIANTS = {0: "smem", 1: "reg16", 2: "mma"}
 MAX_DIM = 32768
 
@@ -27,7 +27,7 @@ EXPORTED = ("hadq_rotate_quantize", "hadq_dequant_rotate_inv", "hadq_rotate_quan
             "hadq_dequant_rotate_inv_kron", "hadq_rotate_quantize_kron_pm1", "hadq_dequant_rotate_inv_kron_pm1", "hadq_rotate_quantize_asym",
             "hadq_dequant_rotate_inv_asym", "hadq_rotate_quantize_keep",
             "hadq_dequant_rotate_inv_keep", "hadq_kv_decode_attention",
-            "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_kron_plan", "hadq_status_str", "hadq_last_error",
+            "hadq_kv_decode_workspace_size", "hadq_kv_decode_attention_noalloc", "hadq_plan", "hadq_kron_plan", "hadq_device_status", "hadq_selftest_bounded_wait", "hadq_status_str", "hadq_last_error",
             "hadq_launch_count", "hadq_version")
 
 
@@ -93,6 +93,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hadq_plan.restype = ctypes.c_int
     lib.hadq_kron_plan.argtypes = [c_i32, c_i64, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(ctypes.c_int)]
     lib.hadq_kron_plan.restype = ctypes.c_int
+    lib.hadq_device_status.argtypes = [vp]
+    lib.hadq_device_status.restype = ctypes.c_int
+    lib.hadq_selftest_bounded_wait.argtypes = [vp, vp]
+    lib.hadq_selftest_bounded_wait.restype = ctypes.c_int
     lib.hadq_status_str.argtypes = [ctypes.c_int]
     lib.hadq_status_str.restype = ctypes.c_char_p
     lib.hadq_last_error.argtypes = []
@@ -153,6 +157,21 @@ def hadq_launch_count() -> int:
 
 def hadq_version() -> int:
     return int(load_library().hadq_version())
+
+
+def hadq_selftest_bounded_wait(scratch, stream=None) -> int:
+    """Run the bounded-wait self-test on `scratch` (a CUDA uint8 tensor of at
+    least 40976 bytes); returns the status (HADQ_ERR_DEVICE expected)."""
+    _need(scratch, "scratch", torch.uint8, scratch.device)
+    if scratch.numel() < 40976:
+        raise ValueError("scratch must hold at least 40976 bytes")
+    return int(load_library().hadq_selftest_bounded_wait(_ptr(scratch), _stream(stream)))
+
+
+def hadq_device_status(stream=None) -> None:
+    """Synchronise the stream; raise HadqError if a bounded wait inside a
+    tcgen05 kernel ran out since the last call (the record is cleared)."""
+    _check(load_library().hadq_device_status(_stream(stream)))
 
 
 def hadq_plan(direction: int, rows: int, dim: int, block: int = -1, bits: int = 4, group: int = -1,

@@ -1,8 +1,8 @@
 // C ABI of libhadq: argument checks, kernel choice and launches.
 //
 // Every entry point validates its arguments on the host, picks a kernel
-// family, launches one kernel on the caller's stream and returns.  Nothing here allocates device memory and
-// nothing synchronises.
+// family, launches one kernel on the caller's stream and returns.  Nothing here
+// allocates device memory, and only hadq_device_status synchronises.
 #include <cmath>
 #include <cstdint>
 #include <cstdarg>
@@ -24,6 +24,7 @@
 #include "hadq_full4096.cuh"
 #include "hadq_generic.cuh"
 #include "hadq_h4096.cuh"
+#include "hadq_h4096_tc.cuh"
 #include "hadq_kron.cuh"
 #include "hadq_kernels.h"
 
@@ -108,8 +109,11 @@ hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (aligned16 && direction == 1 && s.B == 128 && s.G % 128 == 0 && s.dim % 128 == 0)
     return HADQ_PATH_CHUNK_MMA;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
-  if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096)
-    return (s.dim == 4096 || !s.has_signs) ? HADQ_PATH_WIDE4096_MMA : HADQ_PATH_WIDE4096;
+  if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096) {
+    if (s.dim != 4096 && s.has_signs) return HADQ_PATH_WIDE4096;
+    // tile coordinates of the tcgen05 kernel are 32-bit
+    return s.rows * (s.dim / 4096) < (int64_t(1) << 30) ? HADQ_PATH_H4096_TC : HADQ_PATH_WIDE4096_MMA;
+  }
   if (aligned16 && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) && s.dim % 32 == 0 &&
       s.dim <= 16384 && blocked_group_ok(s.G, s.B))
     return HADQ_PATH_BLOCKED;
@@ -343,6 +347,41 @@ hadq_status launch_dq_chunk_mma(const Shape& s, hadq::ChunkArgs a, bool f32, cud
     return fail(HADQ_ERR_CUDA, "128-block tensor-core inverse launch failed: %s", cudaGetErrorString(e));
   }
   return after_launch("128-block tensor-core inverse");
+}
+
+// One persistent CTA per SM (the kernel holds all 512 TMEM columns and most
+// of the shared memory), over tiles of four 4096-point blocks.
+hadq_status launch_h4096_tc(const Shape& s, const void* x, const int8_t* signs, uint8_t* codes, float* scales,
+                            float scale_mul, cudaStream_t stream, int stall_tile = -1) {
+  hadq::TcArgs a{};
+  a.stall_tile = stall_tile;
+  a.nblocks = s.rows * (s.dim / 4096);
+  a.ntiles = (a.nblocks + hadq::kTcTileBlocks - 1) / hadq::kTcTileBlocks;
+  a.signs = signs;
+  a.codes = codes;
+  a.scales = scales;
+  a.scale_mul = scale_mul;
+  a.fault = hadq::tc_fault_word();
+  if (!a.fault) return fail(HADQ_ERR_CUDA, "tcgen05 4096-block kernel: the fault word has no device address");
+  CUtensorMap map;
+  if (!hadq::h4096_tc_encode_map(&map, x, a.nblocks))
+    return fail(HADQ_ERR_CUDA, "tcgen05 4096-block kernel: cuTensorMapEncodeTiled failed");
+  const void* fn = hadq::h4096_tc_kernel_ptr(s.bits, s.has_signs);
+  const size_t smem = hadq::h4096_tc_smem();
+  const int threads = hadq::h4096_tc_threads();
+  int res = 1;
+  const hadq_status pst = prepare(fn, threads, smem, "tcgen05 4096-block kernel", &res);
+  if (pst != HADQ_OK) return pst;
+  const int64_t cap = sm_count();
+  const unsigned grid = (unsigned)(a.ntiles < cap ? a.ntiles : cap);
+  void* args[] = {&map, &a};
+  const cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return fail(HADQ_ERR_CUDA, "tcgen05 4096-block kernel launch failed: %s", cudaGetErrorString(e));
+  }
+  return after_launch("tcgen05 4096-block kernel");
 }
 
 hadq_status launch_wide4096(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream, bool mma) {
@@ -612,7 +651,8 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     return fail(HADQ_ERR_MISALIGNED, "rotated_out must be 4-byte aligned");
   const bool a16 = aligned(x, 16) && aligned(codes, 16) && (!signs || aligned(signs, 16)) &&
                    (!rotated_out || aligned(rotated_out, 16));
-  const hadq_path path = choose_path(0, s, a16);
+  hadq_path path = choose_path(0, s, a16);
+  if (path == HADQ_PATH_H4096_TC && rotated_out) path = HADQ_PATH_WIDE4096_MMA;
   const double qmax = double((1 << (bits - 1)) - 1);
   const float scale_mul = (float)(1.0 / (std::sqrt(double(s.B)) * qmax));
   const float rsqrt_b = (float)(1.0 / std::sqrt(double(s.B)));
@@ -650,6 +690,8 @@ hadq_status hadq_rotate_quantize(const void* x, int64_t rows, int32_t dim, int32
     a.rsqrt_b = rsqrt_b;
     return launch_chunk_mma(s, a, cs);
   }
+  if (path == HADQ_PATH_H4096_TC)
+    return launch_h4096_tc(s, x, signs, static_cast<uint8_t*>(codes), scales, scale_mul, cs);
   if (path == HADQ_PATH_WIDE4096 || path == HADQ_PATH_WIDE4096_MMA) {
     hadq::ChunkArgs a{};
     a.x = static_cast<const uint16_t*>(x);
@@ -1141,8 +1183,46 @@ const char* hadq_status_str(hadq_status st) {
     case HADQ_ERR_UNSUPPORTED: return "unsupported combination";
     case HADQ_ERR_MISALIGNED: return "misaligned pointer";
     case HADQ_ERR_CUDA: return "CUDA error";
+    case HADQ_ERR_DEVICE: return "a kernel gave up a bounded wait";
   }
   return "unknown status";
+}
+
+hadq_status hadq_device_status(hadq_stream_t stream) {
+  g_last_error.clear();
+  unsigned* word = hadq::tc_fault_word();
+  if (!word) return fail(HADQ_ERR_CUDA, "the fault word has no device address");
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v) e = cudaMemset(word, 0, sizeof v);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(HADQ_ERR_CUDA, "reading the fault word failed: %s", cudaGetErrorString(e));
+  }
+  if (v) return fail(HADQ_ERR_DEVICE, "a tcgen05 kernel waited past its limit; its outputs are void");
+  return HADQ_OK;
+}
+
+hadq_status hadq_selftest_bounded_wait(void* scratch, hadq_stream_t stream) {
+  g_last_error.clear();
+  if (!scratch) return fail(HADQ_ERR_INVALID_ARG, "scratch must not be NULL");
+  if (!aligned(scratch, 16)) return fail(HADQ_ERR_MISALIGNED, "scratch must be 16-byte aligned");
+  hadq_status st = hadq_device_status(stream);  // start from a clear record
+  if (st != HADQ_OK) return st;
+  Shape s{};
+  s.rows = 4;
+  s.dim = 4096;
+  s.B = 4096;
+  s.G = 4096;
+  s.bits = 4;
+  s.has_signs = false;
+  uint8_t* buf = static_cast<uint8_t*>(scratch);
+  st = launch_h4096_tc(s, buf, nullptr, buf + 32768, reinterpret_cast<float*>(buf + 40960), 1.0f,
+                       reinterpret_cast<cudaStream_t>(stream), 0);
+  if (st != HADQ_OK) return st;
+  return hadq_device_status(stream);
 }
 
 const char* hadq_last_error(void) { return g_last_error.c_str(); }

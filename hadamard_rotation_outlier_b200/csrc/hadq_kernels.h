@@ -2,6 +2,9 @@
 // Each returns the address to pass to cudaLaunchKernel.
 #pragma once
 
+#include <cstddef>
+#include <cstdint>
+
 namespace hadq {
 
 // direction 0 = rotate+quantise, 1 = dequantise+inverse; threads = CTA size.
@@ -40,6 +43,16 @@ const void* dq_chunk_mma_kernel_ptr(int bits, bool signs, bool f32);
 const void* wide4096_kernel_ptr(int bits, bool signs);
 // The same with the first 16-point stage on tensor cores (kH4096Warps warps).
 const void* h4096_mma_kernel_ptr(int bits, bool signs, bool rot);
+// The same blocks on tcgen05 tensor cores (H_128 GEMM + five register
+// stages), fed by TMA; one persistent CTA of h4096_tc_threads() per SM.
+const void* h4096_tc_kernel_ptr(int bits, bool signs);
+size_t h4096_tc_smem();
+int h4096_tc_threads();
+// Tensor map (a CUtensorMap, 64-byte aligned) of nblocks bf16 blocks at x
+// (16-byte aligned); false if the driver entry point or the encode fails.
+bool h4096_tc_encode_map(void* map, const void* x, int64_t nblocks);
+// Device address of the word the bounded waits of the tcgen05 kernels set.
+unsigned* tc_fault_word();
 const void* full4096_kernel_ptr(int bits, bool signs, int logG);
 const void* generic_kernel_ptr(int direction, int bits);
 

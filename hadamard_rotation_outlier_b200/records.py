@@ -34,6 +34,7 @@ KERNEL_SOURCES = {
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
     "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_mma.cuh", "hadq_kron.cuh", "k_kron.cu"],
     "h4096": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_h4096.cuh", "k_h4096.cu"],
+    "h4096tc": ["hadq_common.cuh", "hadq_h4096_tc.cuh", "k_h4096_tc.cu"],
 }
 
 TRAFFIC_FILE = "dram_traffic.txt"
@@ -51,8 +52,11 @@ def workload_family(wl) -> str:
         return "keep"
     if not hasattr(wl, "block"):
         return "attn"
-    if B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True) == "wide4096_mma":
+    path = B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)
+    if path == "wide4096_mma":
         return "h4096"
+    if path == "h4096_tc":
+        return "h4096tc"
     return "quant"
 
 

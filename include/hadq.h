@@ -59,7 +59,9 @@ typedef enum {
   HADQ_ERR_INVALID_ARG = 1,  /* out-of-range size, NULL pointer, bad enum     */
   HADQ_ERR_UNSUPPORTED = 2,  /* valid maths, no kernel for it                 */
   HADQ_ERR_MISALIGNED = 3,   /* pointer not aligned to its element size       */
-  HADQ_ERR_CUDA = 4          /* the CUDA runtime reported an error            */
+  HADQ_ERR_CUDA = 4,         /* the CUDA runtime reported an error            */
+  HADQ_ERR_DEVICE = 5        /* a kernel gave up a bounded wait (see
+                                hadq_device_status); its outputs are void   */
 } hadq_status;
 
 typedef enum { HADQ_OUT_BF16 = 0, HADQ_OUT_F32 = 1 } hadq_out_dtype;
@@ -77,13 +79,18 @@ typedef enum {
   HADQ_PATH_WIDE4096_MMA = 6, /* the same blocks (dim = 4096 when signs are
                               given) with the first 16-point stage as a bf16
                               tensor-core MMA against H_16                  */
-  HADQ_PATH_CHUNK_MMA = 7  /* 128-point blocks, signs or none, the first
+  HADQ_PATH_CHUNK_MMA = 7, /* 128-point blocks, signs or none, the first
                               16-point stage as an MMA over 16 blocks at a
                               time and the other three in registers.
                               Forward (one scale per block): bf16 MMA on
                               the input, signs as XOR masks on its operand.
                               Inverse (scale groups of whole blocks): f16
                               MMA on the integer codes                      */
+  HADQ_PATH_H4096_TC = 8   /* 4096-column blocks with one scale per block
+                              (dim = 4096 when signs are given), forward, no
+                              rotated_out: TMA-fed tcgen05 GEMM against
+                              H_128 with TMEM accumulators, then five
+                              register stages; one persistent CTA per SM    */
 } hadq_path;
 
 /* Kernel variant of a Kronecker-rotation call (see hadq_kron_plan). */
@@ -396,11 +403,37 @@ hadq_status hadq_kv_decode_attention_noalloc(const void *q, const void *k_codes,
  * family it would use.  direction 0 = rotate_quantize, 1 = dequant_rotate_inv.
  * `aligned16` says whether every pointer of the call is 16-byte aligned.
  * Returns the same status the call would return for these sizes (pointer
- * checks aside) and writes the path to *path.  Touches no GPU.
+ * checks aside) and writes the path to *path.  Touches no GPU.  A forward
+ * call planned as HADQ_PATH_H4096_TC that also asks for rotated_out runs
+ * HADQ_PATH_WIDE4096_MMA instead.
  */
 hadq_status hadq_plan(int32_t direction, int64_t rows, int32_t dim, int32_t block,
                       int32_t bits, int32_t group, int32_t has_signs, int32_t aligned16,
                       hadq_path *path);
+
+/*
+ * hadq_device_status -- synchronise `stream`, then report whether any bounded
+ * wait inside the library's tcgen05 kernels (HADQ_PATH_H4096_TC) ran out on
+ * the current device since the previous call, and clear the record.
+ * HADQ_OK if none did; HADQ_ERR_DEVICE if one did (the outputs of the call
+ * that gave up are void: every role of the kernel left its loop, waited for
+ * its copies in flight and freed its tensor memory, so the context stays
+ * usable); HADQ_ERR_CUDA if the synchronisation or the read failed.
+ */
+hadq_status hadq_device_status(hadq_stream_t stream);
+
+/*
+ * hadq_selftest_bounded_wait -- test of the bounded waits: launches the
+ * HADQ_PATH_H4096_TC kernel on four blocks with the load of its only tile
+ * withheld, so that every wait for it runs out (about one second), then
+ * returns hadq_device_status(stream).  HADQ_ERR_DEVICE is the expected
+ * result; afterwards the record is clear and the context usable.
+ *   scratch  device buffer of at least 40976 bytes, 16-byte aligned, owned by
+ *            the caller (the kernel is given it as input and outputs; with
+ *            the load withheld it writes nothing).
+ * Synchronises `stream`.
+ */
+hadq_status hadq_selftest_bounded_wait(void *scratch, hadq_stream_t stream);
 
 /* Static description of a status code. */
 const char *hadq_status_str(hadq_status status);

@@ -48,7 +48,14 @@ def test_version_and_status_strings(lib):
     assert B.hadq_status_str(B.HADQ_OK) == "ok"
     assert "invalid" in B.hadq_status_str(B.HADQ_ERR_INVALID_ARG)
     assert "misaligned" in B.hadq_status_str(B.HADQ_ERR_MISALIGNED)
+    assert "bounded wait" in B.hadq_status_str(B.HADQ_ERR_DEVICE)
     assert B.hadq_status_str(99) == "unknown status"
+
+
+def test_bounded_wait_selftest_validates_before_launch(lib):
+    assert lib.hadq_selftest_bounded_wait(None, None) == B.HADQ_ERR_INVALID_ARG
+    assert "scratch" in B.hadq_last_error()
+    assert lib.hadq_selftest_bounded_wait(ctypes.c_void_p(0x1008), None) == B.HADQ_ERR_MISALIGNED
 
 
 @pytest.mark.parametrize("args,msg", [
@@ -75,9 +82,9 @@ def test_plan_rejects(lib, args, msg):
     (0, 0, 128, -1, 8, -1, False, True, "none"),
     (0, 524288, 128, -1, 8, -1, False, True, "chunk_mma"),        # Q/K heads, INT8
     (0, 256, 4096, 128, 4, -1, False, True, "chunk"),             # per-token over 32 blocks
-    (0, 16384, 4096, -1, 4, -1, True, True, "wide4096_mma"),      # full 4096 + signs
+    (0, 16384, 4096, -1, 4, -1, True, True, "h4096_tc"),          # full 4096 + signs
     (0, 16, 8192, 4096, 4, 4096, True, True, "wide4096"),         # two 4096 blocks + signs
-    (0, 16, 8192, 4096, 4, 4096, False, True, "wide4096_mma"),    # two 4096 blocks, no signs
+    (0, 16, 8192, 4096, 4, 4096, False, True, "h4096_tc"),        # two 4096 blocks, no signs
     (0, 16384, 4096, -1, 4, 128, True, True, "full4096"),         # 4096 block, group 128
     (0, 2097152, 128, 128, 4, 128, False, True, "chunk_mma"),     # KV cache
     (1, 2097152, 128, 128, 4, 128, False, True, "chunk_mma"),     # KV dequant

@@ -26,7 +26,7 @@ int main(void) {
   CHECK(hadq_plan(0, 524288, 128, -1, 8, -1, 0, 1, &path) == HADQ_OK);
   CHECK(path == HADQ_PATH_CHUNK_MMA);
   CHECK(hadq_plan(0, 16384, 4096, -1, 4, -1, 1, 1, &path) == HADQ_OK);
-  CHECK(path == HADQ_PATH_WIDE4096_MMA);
+  CHECK(path == HADQ_PATH_H4096_TC);
   CHECK(hadq_plan(0, 4, 96, 64, 8, -1, 0, 1, &path) == HADQ_ERR_INVALID_ARG);
   CHECK(strlen(hadq_last_error()) > 0);
 
