@@ -305,8 +305,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
 
   const uint8_t* kc = a.k_codes + row0 * kAttnKRow;
   const uint8_t* vc = a.v_codes + row0 * kAttnKRow;
-  const float* ksc = a.k_scales + row0;
-  const float* vsc = a.v_scales + row0;
+  const float* ksc = a.k_scales + row0 * NG;  // [batch, nkv, stride, NG]
+  const float* vsc = a.v_scales + row0 * NG;
 
   // Copy pattern of one tile (per array, 16 tokens x 4 chunks of 16 bytes):
   // lane covers token lane/4 and 8 + lane/4, chunk lane%4; the scale copy

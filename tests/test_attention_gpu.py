@@ -238,7 +238,9 @@ def test_grouped_cache_with_one_group_matches_row_scales():
     b = run_gpu(qbits, kc, ks4, vc, vs4, 700, None, torch.float32, group=32)
     want = oracle_attention(qbits, kc, ks, vc, vs)
     compare(b, want, torch.float32, "G=32 with equal group scales")
-    np.testing.assert_allclose(b.cpu().numpy(), a.cpu().numpy(), rtol=2e-6, atol=1e-6)
+    # the grouped path sums its four group partials (each weighted by its
+    # scale) where the row path scales one sum: equal up to float32 rounding
+    np.testing.assert_allclose(b.cpu().numpy(), a.cpu().numpy(), rtol=1e-5, atol=1e-5)
 
 
 def test_grouped_cache_rejections():
