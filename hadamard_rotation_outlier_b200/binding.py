@@ -279,10 +279,11 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
                              group: int = -1, softmax_scale: float | None = None,
                              out: torch.Tensor | None = None, out_dtype: torch.dtype = torch.bfloat16,
                              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """One decode step of attention over a rotated INT4 KV cache.
+    """One decode step of attention over a rotated INT4 or INT8 KV cache.
 
     ``q``: bf16 ``[batch, n_q_heads, dim]``.  ``k_codes``/``v_codes``: uint8
-    ``[batch, n_kv_heads, token_stride, dim/2]``; ``k_scales``/``v_scales``:
+    ``[batch, n_kv_heads, token_stride, dim/2]`` (INT4) or uint8/int8 ``[...,
+    dim]`` (INT8, ``bits=8``); ``k_scales``/``v_scales``:
     float32 ``[batch, n_kv_heads, token_stride, dim/group]`` (one scale per row
     for group 128 or -1, which may drop the trailing 1).
     ``tokens`` (default ``token_stride``) rows of each head are attended over.
@@ -298,7 +299,7 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
     batch, nqh, dim = q.shape
     dev = q.device
     if k_codes.dim() != 4 or v_codes.shape != k_codes.shape:
-        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim/2] alike")
+        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim*bits/8] alike")
     nkv, stride = k_codes.shape[1], k_codes.shape[2]
     if k_codes.shape[0] != batch:
         raise ValueError("k_codes batch differs from q")
@@ -306,12 +307,14 @@ def hadq_kv_decode_attention(q: torch.Tensor, k_codes: torch.Tensor, k_scales: t
     if tokens is None:
         tokens = stride
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        if t.dtype == torch.int8:  # INT8 caches may come as int8
+            t = t.view(torch.uint8)
         _need(t, name, torch.uint8, dev)
     per_scale = dim // _resolve(dim, block, group) if group != 0 and dim % _resolve(dim, block, group) == 0 else 1
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float32, dev, batch * nkv * stride * per_scale)
-    if per_row * 2 != dim:
-        raise ValueError(f"codes rows hold {per_row} bytes, expected dim/2 = {dim // 2}")
+    if per_row * 8 != dim * bits:
+        raise ValueError(f"codes rows hold {per_row} bytes, expected dim*bits/8 = {dim * bits // 8}")
     if signs is not None:
         _need(signs, "signs", torch.int8, dev, dim)
     if softmax_scale is None:
@@ -351,10 +354,14 @@ def hadq_kv_decode_attention_noalloc(q: torch.Tensor, k_codes: torch.Tensor, k_s
     batch, nqh, dim = q.shape
     dev = q.device
     if k_codes.dim() != 4 or v_codes.shape != k_codes.shape or k_codes.shape[0] != batch:
-        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim/2] alike")
+        raise ValueError("k_codes and v_codes must be [batch, n_kv_heads, token_stride, dim*bits/8] alike")
     nkv, stride = k_codes.shape[1], k_codes.shape[2]
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        if t.dtype == torch.int8:  # INT8 caches may come as int8
+            t = t.view(torch.uint8)
         _need(t, name, torch.uint8, dev)
+    if k_codes.shape[3] * 8 != dim * bits:
+        raise ValueError(f"codes rows hold {k_codes.shape[3]} bytes, expected dim*bits/8 = {dim * bits // 8}")
     per_scale = dim // _resolve(dim, block, group) if group != 0 and dim % _resolve(dim, block, group) == 0 else 1
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float32, dev, batch * nkv * stride * per_scale)

@@ -531,10 +531,10 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
     return fail(HADQ_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
   if (out_dtype != HADQ_OUT_BF16 && out_dtype != HADQ_OUT_F32)
     return fail(HADQ_ERR_INVALID_ARG, "out_dtype must be HADQ_OUT_BF16 or HADQ_OUT_F32");
-  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || (s.G != 128 && s.G != 64 && s.G != 32) || bits != 4)
+  if (dim != hadq::kAttnDim || s.B != hadq::kAttnDim || (s.G != 128 && s.G != 64 && s.G != 32))
     return fail(HADQ_ERR_UNSUPPORTED,
-                "decode attention supports dim 128, block 128, group 128, 64 or 32, bits 4 (got %d, %d, %d, %d)",
-                dim, s.B, s.G, bits);
+                "decode attention supports dim 128, block 128, group 128, 64 or 32 (got %d, %d, %d)", dim, s.B,
+                s.G);
   const int ng = hadq::kAttnDim / s.G;  // scales per cached row
   if (batch == 0) return HADQ_OK;
   if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !out || (!workspace && !static_scratch))
@@ -555,12 +555,13 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
   if (!static_scratch && !aligned(workspace, 256))
     return fail(HADQ_ERR_MISALIGNED, "workspace must be 256-byte aligned");
 
-  const void* fn = hadq::kv_decode_attn_kernel_ptr(ng);
+  const void* fn = hadq::kv_decode_attn_kernel_ptr(ng, bits);
+  const size_t smem = hadq::kv_decode_attn_smem(ng, bits);
   // One wave of CTAs: split the tokens of each head group so that all CTAs
   // are resident at once (a CTA beyond the wave would run alone afterwards);
   // at least 64 tokens (a tile per warp) per split.
   int res = 1;
-  const hadq_status pst = prepare(fn, hadq::kAttnThreads, 0, "decode attention kernel", &res);
+  const hadq_status pst = prepare(fn, hadq::kAttnThreads, smem, "decode attention kernel", &res);
   if (pst != HADQ_OK) return pst;
   const int64_t wave = int64_t(res) * sm_count();
   int64_t splits = wave / as.groups;
@@ -605,11 +606,12 @@ hadq_status attn_call(const void* q, const void* k_codes, const float* k_scales,
   a.qmul = (float)(double(softmax_scale) * 1.4426950408889634 / std::sqrt(double(hadq::kAttnDim)));
   a.inv_sqrt_dim = (float)(1.0 / std::sqrt(double(hadq::kAttnDim)));
   a.out_f32 = f32 ? 1 : 0;
-  a.vmask = 0x000F000Fu;
-  a.vmagic = 0x43084308u;
+  a.vmask = bits == 8 ? 0x007F007Fu : 0x000F000Fu;
+  a.vmagic = bits == 8 ? 0x43004300u : 0x43084308u;
+  a.vsign = 0x00800080u;
   void* args[] = {&a};
   cudaError_t e = cudaLaunchKernel(fn, dim3(unsigned(splits), unsigned(as.groups)), dim3(hadq::kAttnThreads),
-                                   args, 0, reinterpret_cast<cudaStream_t>(stream));
+                                   args, smem, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     g_launches.fetch_add(1, std::memory_order_relaxed);

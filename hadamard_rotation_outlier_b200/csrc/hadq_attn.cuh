@@ -1,9 +1,9 @@
 // Decode attention over the rotated, quantised KV cache.
 //
 // One new query token per head attends over a cache whose K and V rows were
-// rotated by H_128 (after the optional sign flip) and stored as INT4 codes with
-// one float32 scale per row, i.e. the output of the rotate+quantise kernels at
-// dim 128, block 128, group 128.  The maths ("Hartmann rotation, lightweight
+// rotated by H_128 (after the optional sign flip) and stored as INT4 or INT8
+// codes with one float32 scale per row or per group of 64 or 32 columns, i.e.
+// the output of the rotate+quantise kernels at dim 128, block 128.  The maths ("Hartmann rotation, lightweight
 // QAT, streaming attention", section 1; "QuaRot hands-on", sections 2.2-2.3):
 //
 //   q_rot = (q * s) H                     rotate the query like the keys
@@ -23,15 +23,18 @@
 // Tensor-core use (mma.sync; the contraction has only 4 query rows per KV
 // head, far below the 64-row minimum of a tcgen05 tile, and its operands are
 // born in registers):
-//  * QK: m16n8k32 s8 x s8 -> s32.  B = key codes as int8 (the nibble shifted
-//    into the high half of a byte, i.e. 16 * code, one shift and one mask per
-//    8 codes).  A = the scaled rotated query as a 24-bit fixed-point number
-//    cut into three signed 8-bit digits (rows = head x digit).  The integer
-//    sums are exact; score = (d0 + 2^8 d1 + 2^16 d2) * 2^-E / 16 * kscale.
+//  * QK: m16n8k32 s8 x s8 -> s32.  B = key codes as int8: INT4 nibbles
+//    shifted into the high half of a byte (16 * code, one shift and one mask
+//    per 8 codes); INT8 codes as they are (two byte permutes per 8 codes
+//    split even and odd dims).  A = the scaled rotated query as a 24-bit
+//    fixed-point number cut into three signed 8-bit digits (rows = head x
+//    digit).  The integer sums are exact; score = (d0 + 2^8 d1 + 2^16 d2) *
+//    2^-E * kscale (/ 16 for INT4).
 //  * PV: m16n8k16 bf16 x bf16 -> f32.  B = value codes as exact bf16 values
-//    (the nibble placed in a bf16 mantissa, then 136 subtracted).  A = p *
-//    vscale cut into three bf16 parts hi + mid + lo (rows = head x part), which
-//    together carry the full float32 value.
+//    (INT4: the nibble placed in a bf16 mantissa, then 136 subtracted; INT8:
+//    see int8x2_to_bf16x2).  A = p * vscale cut into three bf16 parts hi +
+//    mid + lo (rows = head x part), which together carry the full float32
+//    value.
 #pragma once
 
 #include <cstdint>
@@ -46,15 +49,24 @@ constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = 32 * kAttnWarps;
 constexpr int kAttnHeads = 4;                                   // query heads per CTA
 constexpr int kAttnTile = 16;                                   // tokens per tile
-constexpr int kAttnStages = 4;                                  // ring depth per warp
-constexpr int kAttnKRow = 64;                                   // bytes of INT4 codes per token
-constexpr int kAttnVRow = 80;                                   // V row padded in shared memory
-constexpr int kAttnStV = kAttnTile * kAttnKRow;                 // 1024
-constexpr int kAttnStS = kAttnStV + kAttnTile * kAttnVRow;      // 2304: K scales, then V scales
-// Bytes of one ring stage: 16 K and 16 V rows, then [16 tokens][NG] K scales
-// and as many V scales (NG = 128 / G scale groups per row).
-__host__ __device__ constexpr int attn_stage_bytes(int ng) { return kAttnStS + 2 * kAttnTile * 4 * ng; }
-constexpr int kAttnStageBytes = attn_stage_bytes(1);            // 2432
+constexpr int kAttnStages = 4;                                  // ring depth per warp, INT4 caches
+constexpr int kAttnStages8 = 3;                                 // INT8 caches (twice the bytes per tile)
+// Per-stage layout of a cache of BITS-bit codes: 16 K rows at pitch KP, 16 V
+// rows at pitch VROW (pitches padded so that the fragment reads are
+// conflict-free), then [16 tokens][NG] K scales and as many V scales (NG =
+// 128 / G scale groups per row).  KROW = bytes of codes per token in global
+// memory.
+template <int BITS>
+struct AttnRows {
+  static constexpr int KROW = 16 * BITS;                        // 64 or 128
+  static constexpr int KP = BITS == 8 ? KROW + 16 : KROW;
+  static constexpr int VROW = KROW + 16;
+  static constexpr int STV = kAttnTile * KP;
+  static constexpr int STS = STV + kAttnTile * VROW;
+};
+__host__ __device__ constexpr int attn_stage_bytes(int ng, int bits = 4) {
+  return (bits == 8 ? AttnRows<8>::STS : AttnRows<4>::STS) + 2 * kAttnTile * 4 * ng;
+}
 constexpr int kAttnCombPitch = kAttnDim + 4;                    // floats per head in the CTA merge
 constexpr int kAttnMaxSplits = 256;
 constexpr size_t kAttnStaticScratchBytes = size_t(16) << 20;  // scratch of the allocation-free entry
@@ -76,13 +88,15 @@ struct AttnArgs {
   float qmul;                // softmax_scale * log2(e) / sqrt(128)
   float inv_sqrt_dim;        // 1 / sqrt(128)
   int out_f32;
-  uint32_t vmask, vmagic;    // 0x000F000F and 0x43084308 (see int4x2_to_bf16x2)
+  uint32_t vmask, vmagic;    // INT4: 0x000F000F and 0x43084308 (see int4x2_to_bf16x2);
+                             // INT8: 0x007F007F and 0x43004300 (see int8x2_to_bf16x2)
+  uint32_t vsign;            // INT8: 0x00800080
 };
 
-template <int STAGES, int NG>
+template <int STAGES, int NG, int BITS>
 struct __align__(16) AttnSmem {
   union {
-    uint8_t stage[kAttnWarps][STAGES][attn_stage_bytes(NG)];
+    uint8_t stage[kAttnWarps][STAGES][attn_stage_bytes(NG, BITS)];
     float comb[kAttnWarps][kAttnHeads][kAttnCombPitch];
   } u;
   int8_t qd[4][kAttnHeads][kAttnDim];  // query digits [digit][head][dim]; digit 3 stays 0
@@ -137,6 +151,20 @@ __device__ __forceinline__ uint32_t int4x2_to_bf16x2(uint32_t x, uint32_t mask, 
   return r;
 }
 
+// Two INT8 codes (bytes at bits 0-7 and 16-23 of x) -> bf16x2 holding the
+// codes exactly.  With the low seven bits of a code c in the mantissa of
+// 128.0, the half reads 128 + (c mod 128); the code's sign bit, placed in the
+// lowest exponent bit of 128.0, gives 128 (c >= 0) or 256 (c < 0), and the
+// difference of the two is c.  Both inputs are one three-input logic
+// operation each (masks and patterns arrive as kernel arguments).
+__device__ __forceinline__ uint32_t int8x2_to_bf16x2(uint32_t x, uint32_t low7, uint32_t magic, uint32_t sign) {
+  uint32_t h, m, r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(low7), "r"(magic));  // (x & low7) | magic
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(m) : "r"(x), "r"(sign), "r"(magic));  // (x & sign) | magic
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(m));
+  return r;
+}
+
 // 2^x for the softmax weights (the ISA approximation; results below 2^-126,
 // i.e. weights below 2^-126 of the running maximum, flush to zero).
 __device__ __forceinline__ float exp2_ftz(float x) {
@@ -180,11 +208,15 @@ __device__ __forceinline__ void int4x8_to_s8x16(uint32_t w, uint32_t& even, uint
 // and the value codes are taken four dims per quarter so that every n8 tile
 // of the P.V product lies inside one group (the A operand p * vscale is cut
 // once per group).
-template <int STAGES, int NG>
+template <int STAGES, int NG, int BITS>
 __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const AttnArgs a) {
   static_assert(NG == 1 || NG == 2 || NG == 4, "groups of 128, 64 or 32 columns");
-  constexpr int SB = attn_stage_bytes(NG);
-  __shared__ AttnSmem<STAGES, NG> sm;
+  static_assert(BITS == 4 || BITS == 8, "INT4 or INT8 codes");
+  using RW = AttnRows<BITS>;
+  constexpr int KROW = RW::KROW, KP = RW::KP, VROW = RW::VROW, STV = RW::STV, STS = RW::STS;
+  constexpr int SB = attn_stage_bytes(NG, BITS);
+  extern __shared__ __align__(16) uint8_t attn_smem_raw[];
+  AttnSmem<STAGES, NG, BITS>& sm = *reinterpret_cast<AttnSmem<STAGES, NG, BITS>*>(attn_smem_raw);
   const int tid = threadIdx.x;
   const int w = tid >> 5;
   const int lane = tid & 31;
@@ -262,8 +294,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     *reinterpret_cast<uint32_t*>(&sm.qd[1][w][4 * lane]) = d1;
     *reinterpret_cast<uint32_t*>(&sm.qd[2][w][4 * lane]) = d2;
     *reinterpret_cast<uint32_t*>(&sm.qd[3][w][4 * lane]) = 0u;
-    // 2^(E' - 22) / 16: undo the fixed point and the 16 * code of the keys.
-    if (lane == 0) sm.qscale[w] = zero ? 0.f : __uint_as_float(uint32_t(E - 25) << 23);
+    // 2^(E' - 22): undo the fixed point (and / 16: the 16 * code of INT4 keys).
+    if (lane == 0) sm.qscale[w] = zero ? 0.f : __uint_as_float(uint32_t(BITS == 4 ? E - 25 : E - 21) << 23);
   }
   __syncthreads();
 
@@ -288,7 +320,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     }
   }
   const float qs = sm.qscale[hh];
-  const uint32_t vmask = a.vmask, vmagic = a.vmagic;
+  const uint32_t vmask = a.vmask, vmagic = a.vmagic, vsign = a.vsign;
   // Digit weights of the two rows this lane holds: rows g (digit g>>2) and
   // g+8 (digit (g>>2)+2; digit 3 is the zero row).
   const float wl = g < 4 ? 1.f : 256.f;
@@ -303,28 +335,30 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
   const int ntiles = (n_tok + kAttnTile - 1) / kAttnTile;
   const int nw = ntiles > w ? (ntiles - w + kAttnWarps - 1) / kAttnWarps : 0;
 
-  const uint8_t* kc = a.k_codes + row0 * kAttnKRow;
-  const uint8_t* vc = a.v_codes + row0 * kAttnKRow;
+  const uint8_t* kc = a.k_codes + row0 * KROW;
+  const uint8_t* vc = a.v_codes + row0 * KROW;
   const float* ksc = a.k_scales + row0 * NG;  // [batch, nkv, stride, NG]
   const float* vsc = a.v_scales + row0 * NG;
 
-  // Copy pattern of one tile (per array, 16 tokens x 4 chunks of 16 bytes):
-  // lane covers token lane/4 and 8 + lane/4, chunk lane%4; the scale copy
-  // takes one float per lane (K scales in lanes 0-15, V scales in 16-31).
-  const int ctok = lane >> 2, cpart = lane & 3;
+  // Copy pattern of one tile (per array, 16 tokens x CPR chunks of 16 bytes):
+  // lane covers chunk lane % CPR of tokens lane / CPR + TPP p (p < 16 / TPP);
+  // the scale copy takes one float per lane (K scales in lanes 0-15, V scales
+  // in 16-31).
+  constexpr int CPR = KROW / 16, TPP = 32 / CPR, NPASS = kAttnTile / TPP;
+  const int ctok = lane / CPR, cpart = lane % CPR;
   const uint32_t s_ring = static_cast<uint32_t>(__cvta_generic_to_shared(&sm.u.stage[w][0][0]));
-  const uint32_t d_k = ctok * kAttnKRow + cpart * 16;
-  const uint32_t d_v = kAttnStV + ctok * kAttnVRow + cpart * 16;
-  const uint32_t d_s = kAttnStS + 4 * lane;
+  const uint32_t d_k = ctok * KP + cpart * 16;
+  const uint32_t d_v = STV + ctok * VROW + cpart * 16;
+  const uint32_t d_s = STS + 4 * lane;
   const int64_t lane_tok = t_begin + int64_t(w) * kAttnTile + ctok;  // token of the first chunk, tile 0
-  const uint8_t* g_k = kc + lane_tok * kAttnKRow + cpart * 16;
-  const uint8_t* g_v = vc + lane_tok * kAttnKRow + cpart * 16;
+  const uint8_t* g_k = kc + lane_tok * KROW + cpart * 16;
+  const uint8_t* g_v = vc + lane_tok * KROW + cpart * 16;
   const float* g_s = (lane < 16 ? ksc : vsc) + t_begin + int64_t(w) * kAttnTile + (lane & 15);
   // NG > 1: scales [token][NG] per array; lane p < 4 NG copies K piece p,
   // lanes 4 NG .. 8 NG - 1 the V pieces (16 bytes = 4 / NG tokens each)
   const int sg_piece = lane % (4 * NG);
   const int sg_tok = sg_piece * 4 / NG;  // first token of this lane's piece in the tile
-  const uint32_t d_sg = kAttnStS + (lane < 4 * NG ? 0u : uint32_t(kAttnTile * 4 * NG)) + 16u * uint32_t(sg_piece);
+  const uint32_t d_sg = STS + (lane < 4 * NG ? 0u : uint32_t(kAttnTile * 4 * NG)) + 16u * uint32_t(sg_piece);
   const float* g_sg = (lane < 4 * NG ? ksc : vsc) + (t_begin + int64_t(w) * kAttnTile) * NG + 4 * sg_piece;
   constexpr int64_t kStepTok = int64_t(kAttnWarps) * kAttnTile;  // tokens between a warp's tiles
 
@@ -333,10 +367,11 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     const int64_t adv = int64_t(k) * kStepTok;
     const int r0 = (w + kAttnWarps * k) * kAttnTile;  // first token of the tile, from t_begin
     if (r0 + kAttnTile <= n_tok) {
-      cp_async16(st + d_k, g_k + adv * kAttnKRow);
-      cp_async16(st + d_k + 8 * kAttnKRow, g_k + (adv + 8) * kAttnKRow);
-      cp_async16(st + d_v, g_v + adv * kAttnKRow);
-      cp_async16(st + d_v + 8 * kAttnVRow, g_v + (adv + 8) * kAttnKRow);
+#pragma unroll
+      for (int p = 0; p < NPASS; ++p) {
+        cp_async16(st + d_k + TPP * p * KP, g_k + (adv + TPP * p) * KROW);
+        cp_async16(st + d_v + TPP * p * VROW, g_v + (adv + TPP * p) * KROW);
+      }
       if constexpr (NG == 1) {
         cp_async4(st + d_s, g_s + adv);
       } else if (lane < 8 * NG) {  // 4 NG pieces of 16 bytes of K scales, then as many of V
@@ -344,13 +379,14 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
       }
     } else {  // ragged last tile: rows past t_end are zero-filled, never read
       // (their source address is replaced by the first row of the head).
-      const bool v0 = r0 + ctok < n_tok, v1 = r0 + ctok + 8 < n_tok;
       const bool vs = r0 + (lane & 15) < n_tok;
       const float* s0 = lane < 16 ? ksc : vsc;
-      cp_async16_zfill(st + d_k, v0 ? g_k + adv * kAttnKRow : kc, v0);
-      cp_async16_zfill(st + d_k + 8 * kAttnKRow, v1 ? g_k + (adv + 8) * kAttnKRow : kc, v1);
-      cp_async16_zfill(st + d_v, v0 ? g_v + adv * kAttnKRow : vc, v0);
-      cp_async16_zfill(st + d_v + 8 * kAttnVRow, v1 ? g_v + (adv + 8) * kAttnKRow : vc, v1);
+#pragma unroll
+      for (int p = 0; p < NPASS; ++p) {
+        const bool vp = r0 + ctok + TPP * p < n_tok;
+        cp_async16_zfill(st + d_k + TPP * p * KP, vp ? g_k + (adv + TPP * p) * KROW : kc, vp);
+        cp_async16_zfill(st + d_v + TPP * p * VROW, vp ? g_v + (adv + TPP * p) * KROW : vc, vp);
+      }
       if constexpr (NG == 1) {
         cp_async4_zfill(st + d_s, vs ? g_s + adv : s0, vs);
       } else if (lane < 8 * NG) {  // the piece's tokens past t_end read nothing (zero fill)
@@ -390,18 +426,18 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     for (int q = 0; q < NG; ++q)
 #pragma unroll
       for (int i = 0; i < 4; ++i) c0[q][i] = c1[q][i] = 0;
-    {
+    if constexpr (BITS == 4) {
       uint32_t kw0[4], kw1[4];
       if constexpr (NG == 1) {
-        const uint4 k0 = *reinterpret_cast<const uint4*>(st + g * kAttnKRow + 16 * j);
-        const uint4 k1 = *reinterpret_cast<const uint4*>(st + (g + 8) * kAttnKRow + 16 * j);
+        const uint4 k0 = *reinterpret_cast<const uint4*>(st + g * KP + 16 * j);
+        const uint4 k1 = *reinterpret_cast<const uint4*>(st + (g + 8) * KP + 16 * j);
         kw0[0] = k0.x; kw0[1] = k0.y; kw0[2] = k0.z; kw0[3] = k0.w;
         kw1[0] = k1.x; kw1[1] = k1.y; kw1[2] = k1.z; kw1[3] = k1.w;
       } else {  // dims 32 s + 8 j .. + 7 = bytes 16 s + 4 j .. + 3 of a row
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          kw0[s] = *reinterpret_cast<const uint32_t*>(st + g * kAttnKRow + 16 * s + 4 * j);
-          kw1[s] = *reinterpret_cast<const uint32_t*>(st + (g + 8) * kAttnKRow + 16 * s + 4 * j);
+          kw0[s] = *reinterpret_cast<const uint32_t*>(st + g * KP + 16 * s + 4 * j);
+          kw1[s] = *reinterpret_cast<const uint32_t*>(st + (g + 8) * KP + 16 * s + 4 * j);
         }
       }
 #pragma unroll
@@ -412,12 +448,39 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
         int4x8_to_s8x16(kw1[s], e, od);
         mma_s8_16832(c1[s * NG / 4], qa[s], e, od);
       }
+    } else {
+      // the lane's 8 dims of k-step s are 8 consecutive bytes: even dims
+      // (a0, a1 of the query) and odd dims (a2, a3) by two byte permutes
+      uint2 kw0[4], kw1[4];
+      if constexpr (NG == 1) {  // dims 32 j + 8 s: bytes 32 j .. 32 j + 31
+        const uint4 k0a = *reinterpret_cast<const uint4*>(st + g * KP + 32 * j);
+        const uint4 k0b = *reinterpret_cast<const uint4*>(st + g * KP + 32 * j + 16);
+        const uint4 k1a = *reinterpret_cast<const uint4*>(st + (g + 8) * KP + 32 * j);
+        const uint4 k1b = *reinterpret_cast<const uint4*>(st + (g + 8) * KP + 32 * j + 16);
+        kw0[0] = make_uint2(k0a.x, k0a.y); kw0[1] = make_uint2(k0a.z, k0a.w);
+        kw0[2] = make_uint2(k0b.x, k0b.y); kw0[3] = make_uint2(k0b.z, k0b.w);
+        kw1[0] = make_uint2(k1a.x, k1a.y); kw1[1] = make_uint2(k1a.z, k1a.w);
+        kw1[2] = make_uint2(k1b.x, k1b.y); kw1[3] = make_uint2(k1b.z, k1b.w);
+      } else {  // dims 32 s + 8 j .. + 7
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          kw0[s] = *reinterpret_cast<const uint2*>(st + g * KP + 32 * s + 8 * j);
+          kw1[s] = *reinterpret_cast<const uint2*>(st + (g + 8) * KP + 32 * s + 8 * j);
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        mma_s8_16832(c0[s * NG / 4], qa[s], __byte_perm(kw0[s].x, kw0[s].y, 0x6420),
+                     __byte_perm(kw0[s].x, kw0[s].y, 0x7531));
+        mma_s8_16832(c1[s * NG / 4], qa[s], __byte_perm(kw1[s].x, kw1[s].y, 0x6420),
+                     __byte_perm(kw1[s].x, kw1[s].y, 0x7531));
+      }
     }
     // Scores.  Every lane holds digit partials of tokens 2j, 2j+1, 2j+8 and
     // 2j+9 for head g & 3; the lane pair (g, g ^ 4) shares that head, and the
     // low lane (g < 4) finishes tokens 2j, 2j+1 while the high lane finishes
     // 2j+8, 2j+9 (`own`), each adding the partner's partials.
-    const float* sc = reinterpret_cast<const float*>(st + kAttnStS);  // [16][NG] K, then [16][NG] V
+    const float* sc = reinterpret_cast<const float*>(st + STS);  // [16][NG] K, then [16][NG] V
     float sv0 = 0.f, sv1 = 0.f;
 #pragma unroll
     for (int q = 0; q < NG; ++q) {
@@ -485,14 +548,51 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
     }
 
     // --- PV: O[(head, part), dim] += P . V ---
-    if constexpr (NG == 1) {
+    if constexpr (BITS == 8 && NG == 1) {
+      // lane (g, j) feeds the value codes of dims 16g + i (n8 tile i) for
+      // tokens 2j, 2j+1 / 2j+8, 2j+9: byte i of each token's 16 bytes
+      const uint8_t* svp = st + STV + 16 * g;
+      const uint4 va = *reinterpret_cast<const uint4*>(svp + (2 * j) * VROW);
+      const uint4 vb = *reinterpret_cast<const uint4*>(svp + (2 * j + 1) * VROW);
+      const uint4 vcx = *reinterpret_cast<const uint4*>(svp + (2 * j + 8) * VROW);
+      const uint4 vd = *reinterpret_cast<const uint4*>(svp + (2 * j + 9) * VROW);
+      const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+      const uint32_t wc[4] = {vcx.x, vcx.y, vcx.z, vcx.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t sel = uint32_t((i & 3) | ((4 + (i & 3)) << 8));  // byte i%4 of each word to bytes 0, 2
+        mma_bf16_16816(o[i], pa[0], int8x2_to_bf16x2(__byte_perm(wa[i >> 2], wb[i >> 2], sel), vmask, vmagic, vsign),
+                       int8x2_to_bf16x2(__byte_perm(wc[i >> 2], wd[i >> 2], sel), vmask, vmagic, vsign));
+      }
+    } else if constexpr (BITS == 8) {
+      // n8 tile i = 4 qt + r: lane (g, j) feeds dim 32 qt + 8 (g >> 1) + 2 r +
+      // (g & 1), byte (g & 1) + 2 r of the 8 bytes at 32 qt + 8 (g >> 1)
+      const uint8_t* svp = st + STV + 8 * (g >> 1);
+      const uint32_t bsel = uint32_t(g & 1);
+#pragma unroll
+      for (int qt = 0; qt < 4; ++qt) {
+        const uint2 wa = *reinterpret_cast<const uint2*>(svp + (2 * j) * VROW + 32 * qt);
+        const uint2 wb = *reinterpret_cast<const uint2*>(svp + (2 * j + 1) * VROW + 32 * qt);
+        const uint2 wc = *reinterpret_cast<const uint2*>(svp + (2 * j + 8) * VROW + 32 * qt);
+        const uint2 wd = *reinterpret_cast<const uint2*>(svp + (2 * j + 9) * VROW + 32 * qt);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t b = bsel + 2 * (r & 1);  // byte within the word r >> 1
+          const uint32_t sel = b | ((4 + b) << 8);
+          const uint32_t xab = __byte_perm(r < 2 ? wa.x : wa.y, r < 2 ? wb.x : wb.y, sel);
+          const uint32_t xcd = __byte_perm(r < 2 ? wc.x : wc.y, r < 2 ? wd.x : wd.y, sel);
+          mma_bf16_16816(o[4 * qt + r], pa[qt * NG / 4], int8x2_to_bf16x2(xab, vmask, vmagic, vsign),
+                         int8x2_to_bf16x2(xcd, vmask, vmagic, vsign));
+        }
+      }
+    } else if constexpr (NG == 1) {
       // lane (g, j) feeds the value codes of dims 16g + i (n8 tile i) for
       // tokens 2j, 2j+1 / 2j+8, 2j+9
-      const uint8_t* svp = st + kAttnStV + 8 * g;
-      const uint2 va = *reinterpret_cast<const uint2*>(svp + (2 * j) * kAttnVRow);
-      const uint2 vb = *reinterpret_cast<const uint2*>(svp + (2 * j + 1) * kAttnVRow);
-      const uint2 vcx = *reinterpret_cast<const uint2*>(svp + (2 * j + 8) * kAttnVRow);
-      const uint2 vd = *reinterpret_cast<const uint2*>(svp + (2 * j + 9) * kAttnVRow);
+      const uint8_t* svp = st + STV + 8 * g;
+      const uint2 va = *reinterpret_cast<const uint2*>(svp + (2 * j) * VROW);
+      const uint2 vb = *reinterpret_cast<const uint2*>(svp + (2 * j + 1) * VROW);
+      const uint2 vcx = *reinterpret_cast<const uint2*>(svp + (2 * j + 8) * VROW);
+      const uint2 vd = *reinterpret_cast<const uint2*>(svp + (2 * j + 9) * VROW);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const uint32_t sel = (h & 1) ? 0x7632u : 0x5410u;
@@ -507,14 +607,14 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kv_decode_attn_kernel(const A
       // n8 tile i = 4 qt + r (quarter qt of the row, group qt * NG / 4): lane
       // (g, j) feeds dim 32 qt + 8 (g >> 1) + 2 r + (g & 1), i.e. nibble g & 1
       // of byte r of the word at byte 16 qt + 4 (g >> 1) of the token's row
-      const uint8_t* svp = st + kAttnStV + 4 * (g >> 1);
+      const uint8_t* svp = st + STV + 4 * (g >> 1);
       const int nsh = 4 * (g & 1);
 #pragma unroll
       for (int qt = 0; qt < 4; ++qt) {
-        const uint32_t wa = *reinterpret_cast<const uint32_t*>(svp + (2 * j) * kAttnVRow + 16 * qt);
-        const uint32_t wb = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 1) * kAttnVRow + 16 * qt);
-        const uint32_t wc = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 8) * kAttnVRow + 16 * qt);
-        const uint32_t wd = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 9) * kAttnVRow + 16 * qt);
+        const uint32_t wa = *reinterpret_cast<const uint32_t*>(svp + (2 * j) * VROW + 16 * qt);
+        const uint32_t wb = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 1) * VROW + 16 * qt);
+        const uint32_t wc = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 8) * VROW + 16 * qt);
+        const uint32_t wd = *reinterpret_cast<const uint32_t*>(svp + (2 * j + 9) * VROW + 16 * qt);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const uint32_t sel = uint32_t(r | (r << 4) | ((4 + r) << 8) | ((4 + r) << 12));  // byte r of each word

@@ -40,17 +40,34 @@
 
 namespace hadq {
 
-constexpr int kTcStages = 5;                       // 32 KB input stages
-constexpr int kTcAcc = 4;                          // TMEM accumulators of 128 columns
-constexpr int kTcEpiWG = 2;                        // epilogue warpgroups
-constexpr int kTcTileBlocks = 4;                   // 4096-point blocks per tile (N = 128)
+#ifndef HADQ_TC_EPI_WG
+#define HADQ_TC_EPI_WG 4
+#endif
+#ifndef HADQ_TC_BPP
+#define HADQ_TC_BPP 1
+#endif
+#ifndef HADQ_TC_TILE
+#define HADQ_TC_TILE 4
+#endif
+#ifndef HADQ_TC_STAGES
+#define HADQ_TC_STAGES (20 / HADQ_TC_TILE)
+#endif
+constexpr int kTcTileBlocks = HADQ_TC_TILE;        // 4096-point blocks per tile (N = 32 per block)
+constexpr int kTcStages = HADQ_TC_STAGES;          // input stages of one tile each
+constexpr int kTcAcc = 16 / kTcTileBlocks;         // TMEM accumulators (512 columns in all)
+constexpr int kTcEpiWG = HADQ_TC_EPI_WG;           // epilogue warpgroups
+constexpr int kTcBpp = HADQ_TC_BPP;                // blocks per epilogue pass (one barrier each)
+static_assert(kTcTileBlocks == 2 || kTcTileBlocks == 4, "tiles of 2 or 4 blocks");
+static_assert(kTcTileBlocks % kTcBpp == 0, "passes cover a tile");
+static_assert(kTcBpp == 1 || kTcBpp == 2 || kTcBpp == 4, "blocks per pass");
 constexpr int kTcStageBytes = kTcTileBlocks * 8192;
 constexpr int kTcABytes = 128 * 128 * 2;           // H_128 in bf16
 constexpr int kTcSignWarp0 = 4 * kTcEpiWG;         // warps 0 .. 4 kTcEpiWG - 1: epilogue
 constexpr int kTcProdWarp = kTcSignWarp0 + 4;      // then four sign warps, the producer
 constexpr int kTcMmaWarp = kTcProdWarp + 1;        // and the MMA warp (also allocates TMEM)
 constexpr int kTcThreads = (kTcMmaWarp + 1) * 32;
-constexpr uint32_t kTcTmemCols = kTcAcc * 128;
+constexpr int kTcAccCols = 32 * kTcTileBlocks;    // N of the MMA
+constexpr uint32_t kTcTmemCols = kTcAcc * kTcAccCols;
 constexpr unsigned long long kTcWaitNs = 1000000000ull;  // about one second per wait
 
 struct TcTail {
@@ -59,8 +76,8 @@ struct TcTail {
   uint64_t empty[kTcStages];   // MMAs done reading the stage
   uint64_t tfull[kTcAcc];      // accumulator written
   uint64_t tempty[kTcAcc];     // accumulator read by its warpgroup
-  alignas(16) uint32_t red[kTcEpiWG][2][2][4];  // [group][parity][block of the pair][warp]: max
-                                                // bits, read back as 16-byte vectors
+  alignas(16) uint32_t red[kTcEpiWG][2][kTcBpp][4];  // [group][parity][block of the pass][warp]:
+                                                     // max bits, read back as 16-byte vectors
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -101,11 +118,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
 }
 __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
   uint32_t ok;
+#ifdef HADQ_TC_WAIT_HINT_NS
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_addr(b)), "r"(parity), "n"(HADQ_TC_WAIT_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
       : "r"(smem_addr(b)), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 __device__ __forceinline__ unsigned long long global_ns() {
@@ -147,8 +172,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
          (uint64_t(swizzle) << 61);
 }
 // Instruction descriptor of kind::f16: D float32, A and B bf16, A K-major,
-// B MN-major, N = 128, M = 128.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// B MN-major, N = 32 x blocks per tile, M = 128.
+constexpr uint32_t kTcIdesc =
+    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t(kTcAccCols) >> 3) << 17) | ((128u >> 4) << 24);
 
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
   asm volatile(
@@ -187,6 +213,23 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&a)[32], float 
     a[j] = __uint_as_float(r[j]);
     b[j] = __uint_as_float(r[32 + j]);
   }
+}
+
+// 32 lanes x 32 columns (one block), waited for in the same statement.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&a)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) a[j] = __uint_as_float(r[j]);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -230,7 +273,18 @@ __device__ __forceinline__ float tc_h32_absmax(float (&v)[32]) {
   reg_stage<32, 2>(v);
   reg_stage<32, 4>(v);
   reg_stage<32, 8>(v);
+#ifdef HADQ_TC_MAX_AFTER
+  reg_stage<32, 16>(v);
+  float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    m0 = max3(m0, fabsf(v[i]), fabsf(v[i + 1]));
+    m1 = max3(m1, fabsf(v[i + 2]), fabsf(v[i + 3]));
+  }
+  return fmaxf(m0, m1);
+#else
   return reg_stage_absmax<32, 16>(v);
+#endif
 }
 
 template <int BITS, bool SIGNS>
@@ -323,7 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ad = smem_desc(abase + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2);
           const uint64_t bd = smem_desc(bbase + kk * 1024, 8192, 512, 4);
-          tc_mma(tmem + uint32_t(c * 128), ad, bd, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + uint32_t(c * kTcAccCols), ad, bd, kk > 0 ? 1u : 0u);
         }
         tc_commit(&tl->empty[s]);
         tc_commit(&tl->tfull[c]);
@@ -386,48 +440,53 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
       tc_fence_after();
       bool stop = false;
 #pragma unroll 1
-      for (int pr = 0; pr < 2; ++pr) {
-        float v0[32], v1[32];
+      for (int pr = 0; pr < kTcTileBlocks / kTcBpp; ++pr) {
+        float v[kTcBpp][32];
         if (ok) {
-          tmem_ld64(tmem + (uint32_t(32 * q) << 16) + uint32_t(c * 128 + 64 * pr), v0, v1);
+          const uint32_t ta = tmem + (uint32_t(32 * q) << 16) + uint32_t(c * kTcAccCols + 32 * kTcBpp * pr);
+          if constexpr (kTcBpp == 2) {
+            tmem_ld64(ta, v[0], v[1]);
+          } else {
+#pragma unroll
+            for (int b = 0; b < kTcBpp; ++b) tmem_ld32(ta + 32 * b, v[b]);
+          }
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0.0f;
+          for (int b = 0; b < kTcBpp; ++b)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[b][j] = 0.0f;
         }
-        if (pr == 1) {
+        if (pr == kTcTileBlocks / kTcBpp - 1) {  // the accumulator has been read
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tl->tempty[c]);
         }
-        const float m0 = tc_h32_absmax(v0), m1 = tc_h32_absmax(v1);
         // non-negative floats order as their bit patterns; a warp that gave up
         // votes ~0, which no |y| can reach
-        const uint32_t b0 = __reduce_max_sync(0xffffffffu, ok ? __float_as_uint(m0) : ~0u);
-        const uint32_t b1 = __reduce_max_sync(0xffffffffu, ok ? __float_as_uint(m1) : ~0u);
-        if (lane == 0) {
-          tl->red[g][par][0][q] = b0;
-          tl->red[g][par][1][q] = b1;
+#pragma unroll
+        for (int b = 0; b < kTcBpp; ++b) {
+          const float m = tc_h32_absmax(v[b]);
+          const uint32_t mb = __reduce_max_sync(0xffffffffu, ok ? __float_as_uint(m) : ~0u);
+          if (lane == 0) tl->red[g][par][b][q] = mb;
         }
         named_bar_sync(1 + g, 128);
-        const uint4 r0 = *reinterpret_cast<const uint4*>(tl->red[g][par][0]);  // after the barrier (memory clobber)
-        const uint4 r1 = *reinterpret_cast<const uint4*>(tl->red[g][par][1]);
+        uint32_t M[kTcBpp];
+#pragma unroll
+        for (int b = 0; b < kTcBpp; ++b) {
+          const uint4 r = *reinterpret_cast<const uint4*>(tl->red[g][par][b]);  // after the barrier
+          M[b] = max(max(r.x, r.y), max(r.z, r.w));
+          if (M[b] == ~0u) stop = true;
+        }
         par ^= 1u;
-        const uint32_t M0 = max(max(r0.x, r0.y), max(r0.z, r0.w));
-        const uint32_t M1 = max(max(r1.x, r1.y), max(r1.z, r1.w));
-        if (M0 == ~0u || M1 == ~0u) {
-          stop = true;
-          break;
-        }
-        const int64_t blk = t * kTcTileBlocks + 2 * pr;
-        if (blk < a.nblocks) {
-          const float m = __uint_as_float(M0);
-          if (h == 0) a.scales[blk] = m * a.scale_mul;
-          tc_store_codes<BITS>(v0, m, a.codes + blk * (4096 * BITS / 8) + h * CODE_BYTES);
-        }
-        if (blk + 1 < a.nblocks) {
-          const float m = __uint_as_float(M1);
-          if (h == 0) a.scales[blk + 1] = m * a.scale_mul;
-          tc_store_codes<BITS>(v1, m, a.codes + (blk + 1) * (4096 * BITS / 8) + h * CODE_BYTES);
+        if (stop) break;
+#pragma unroll
+        for (int b = 0; b < kTcBpp; ++b) {
+          const int64_t blk = t * kTcTileBlocks + kTcBpp * pr + b;
+          if (blk < a.nblocks) {
+            const float m = __uint_as_float(M[b]);
+            if (h == 0) a.scales[blk] = m * a.scale_mul;
+            tc_store_codes<BITS>(v[b], m, a.codes + blk * (4096 * BITS / 8) + h * CODE_BYTES);
+          }
         }
       }
       if (stop) {

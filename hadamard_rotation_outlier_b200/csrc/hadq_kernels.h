@@ -60,9 +60,11 @@ const void* generic_kernel_ptr(int direction, int bits);
 
 namespace hadq {
 
-// Decode attention over the rotated INT4 KV cache (head dim 128, ng = 1, 2 or
-// 4 scales per cached row: groups of 128, 64 or 32 columns), 128 threads per CTA.
-const void* kv_decode_attn_kernel_ptr(int ng);
+// Decode attention over the rotated INT4 or INT8 KV cache (head dim 128, ng =
+// 1, 2 or 4 scales per cached row: groups of 128, 64 or 32 columns), 128
+// threads per CTA, kv_decode_attn_smem(ng, bits) bytes of dynamic shared memory.
+const void* kv_decode_attn_kernel_ptr(int ng, int bits);
+size_t kv_decode_attn_smem(int ng, int bits);
 // Device address (current device) of the library's static attention scratch
 // of kAttnStaticScratchBytes, or NULL if the runtime cannot resolve it.
 void* attn_static_scratch();

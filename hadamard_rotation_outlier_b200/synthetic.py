@@ -359,6 +359,25 @@ def random_int4_cache(batch: int, n_kv_heads: int, stride: int, dim: int, seed: 
     return codes, scales
 
 
+def random_int8_cache(batch: int, n_kv_heads: int, stride: int, dim: int, seed: int,
+                      scale_range=(0.004, 0.012)):
+    """Seeded INT8 cache rows and positive float32 row scales.
+
+    Each code is the sum of four independent uniform draws from -31..31
+    (values -124..124, standard deviation about 36), stored as int8.  Returns
+    ``(codes int8 [batch, n_kv_heads, stride, dim], scales float32 [batch,
+    n_kv_heads, stride])``.
+    """
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0xCAC8, batch, n_kv_heads, stride, dim]))
+    shape = (batch, n_kv_heads, stride, dim)
+    codes = np.zeros(shape, np.int16)
+    for _ in range(4):
+        codes += rng.integers(-31, 32, size=shape, dtype=np.int16)
+    scales = rng.uniform(scale_range[0], scale_range[1],
+                         size=(batch, n_kv_heads, stride)).astype(np.float32)
+    return codes.astype(np.int8), scales
+
+
 def vertical_tokens(tokens: int, n: int, seed: int, skip_head: int = 0, skip_tail: int = 0) -> np.ndarray:
     """Seeded distinct token indices standing in for vertical-line tokens,
     drawn from [skip_head, tokens - skip_tail) and sorted."""

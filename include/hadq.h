@@ -311,10 +311,10 @@ hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales,
 
 /*
  * hadq_kv_decode_attention -- one decode step of attention over a KV cache
- * stored in the rotated basis as INT4 codes.
+ * stored in the rotated basis as INT4 or INT8 codes.
  *
  * The cache rows are what hadq_rotate_quantize writes for dim 128, block 128
- * (or -1), group 128 (or -1), 64 or 32, bits 4 and the same signs:
+ * (or -1), group 128 (or -1), 64 or 32, bits 4 or 8 and the same signs:
  * K_rot = (K * s) H and V_rot = (V * s) H, quantised per row or per group.  Because H is orthogonal,
  * (q H)(K H)^T = q K^T ("Hartmann rotation, lightweight QAT, streaming
  * attention", section 1), so the scores come from the rotated query against
@@ -329,9 +329,10 @@ hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales,
  * (kscale_t, vscale_t: the scale of each element's group.)
  *
  *   q            device, bfloat16 [batch, n_q_heads, dim], 8-byte aligned.
- *   k_codes,     device, uint8 [batch, n_kv_heads, token_stride, dim/2] packed
- *   v_codes      INT4 (element 2j in the low nibble of byte j), 16-byte
- *                aligned.  Only the first `tokens` rows of each head are read.
+ *   k_codes,     device [batch, n_kv_heads, token_stride, dim/2] bytes of packed
+ *   v_codes      INT4 (element 2j in the low nibble of byte j), or [..., dim]
+ *                int8 for bits 8; 16-byte aligned.  Only the first `tokens`
+ *                rows of each head are read.
  *   k_scales,    device, float32 [batch, n_kv_heads, token_stride, 128/group]:
  *   v_scales     the per-group scales of the codes (one per row for group 128),
  *                4-byte aligned; for group 64 or 32, 16-byte aligned with
@@ -343,7 +344,7 @@ hadq_status hadq_dequant_rotate_inv_keep(const void *codes, const float *scales,
  *   tokens       cached tokens attended over, 1 <= tokens <= token_stride,
  *                at most 2^30 (HADQ_ERR_UNSUPPORTED beyond).
  *   dim, block,  the cache's rotate+quantise parameters; the kernel supports
- *   bits, group  dim 128, block 128 or -1, bits 4, group 128 (or -1), 64 or 32
+ *   bits, group  dim 128, block 128 or -1, bits 4 or 8, group 128 (or -1), 64 or 32
  *                and returns HADQ_ERR_UNSUPPORTED for any other valid
  *                combination.
  *   signs        device int8 [dim] (4-byte aligned) or NULL, as for the cache.

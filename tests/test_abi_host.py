@@ -198,7 +198,7 @@ def _attn(lib, q=0x10000, kc=0x10000, ks=0x10000, vc=0x10000, vs=0x10000, batch=
     (dict(scale=float("inf")), B.HADQ_ERR_INVALID_ARG, "softmax_scale"),
     (dict(dtype=5), B.HADQ_ERR_INVALID_ARG, "out_dtype"),
     (dict(dim=64, block=64, group=64), B.HADQ_ERR_UNSUPPORTED, "dim 128"),
-    (dict(bits=8), B.HADQ_ERR_UNSUPPORTED, "bits 4"),
+    (dict(bits=5), B.HADQ_ERR_INVALID_ARG, "bits"),
     (dict(group=16), B.HADQ_ERR_UNSUPPORTED, "group 128, 64 or 32"),
     (dict(group=64, ks=0x10004), B.HADQ_ERR_MISALIGNED, "16-byte aligned"),
     (dict(group=64, stride=17, tokens=17), B.HADQ_ERR_MISALIGNED, "token_stride"),

@@ -35,37 +35,40 @@ def _q_tensor(bits):
     return _dev(bits.view(np.int16)).view(torch.bfloat16)
 
 
-def oracle_cache(batch, nkv, stride, seed, with_outliers=True, signs=None, group=128):
-    """K and V caches quantised by the oracle from seeded bf16 rows; scales
-    [batch, nkv, stride] for group 128, else [batch, nkv, stride, 128/group]."""
+def oracle_cache(batch, nkv, stride, seed, with_outliers=True, signs=None, group=128, bits=4):
+    """K and V caches quantised by the oracle from seeded bf16 rows; codes
+    [batch, nkv, stride, dim * bits / 8], scales [batch, nkv, stride] for
+    group 128, else [batch, nkv, stride, 128/group]."""
     rows = batch * nkv * stride
     cols = (3, 77, 101) if with_outliers else ()
     kx = S.random_bf16(rows, DIM, seed, outlier_cols=cols, outlier_scale=30.0)
     vx = S.random_bf16(rows, DIM, seed + 1)
-    k = O.rotate_quantize(kx, block=128, signs=signs, bits=4, group=group, method="fwht")
-    v = O.rotate_quantize(vx, block=128, signs=signs, bits=4, group=group, method="fwht")
+    k = O.rotate_quantize(kx, block=128, signs=signs, bits=bits, group=group, method="fwht")
+    v = O.rotate_quantize(vx, block=128, signs=signs, bits=bits, group=group, method="fwht")
     shape = (batch, nkv, stride)
     sshape = shape if group == 128 else shape + (DIM // group,)
-    return (k["codes"].reshape(shape + (DIM // 2,)), k["scales"].reshape(sshape),
-            v["codes"].reshape(shape + (DIM // 2,)), v["scales"].reshape(sshape))
+    per_row = DIM * bits // 8
+    return (k["codes"].reshape(shape + (per_row,)), k["scales"].reshape(sshape),
+            v["codes"].reshape(shape + (per_row,)), v["scales"].reshape(sshape))
 
 
-def run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, softmax_scale=None, workspace=None, group=128):
+def run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, softmax_scale=None, workspace=None, group=128,
+            bits=4):
     sg = None if signs is None else _dev(signs)
     out = B.hadq_kv_decode_attention(_q_tensor(qbits), _dev(kc), _dev(ks), _dev(vc), _dev(vs),
-                                     tokens=tokens, block=128, signs=sg, bits=4, group=group,
+                                     tokens=tokens, block=128, signs=sg, bits=bits, group=group,
                                      softmax_scale=softmax_scale, out_dtype=out_dtype,
                                      workspace=workspace)
     torch.cuda.synchronize()
     return out
 
 
-def oracle_attention(qbits, kc, ks, vc, vs, signs=None, softmax_scale=None, group=128):
+def oracle_attention(qbits, kc, ks, vc, vs, signs=None, softmax_scale=None, group=128, bits=4):
     """Oracle output and its allowance for the cache rows given."""
-    want = O.kv_decode_attention(qbits, kc, ks, vc, vs, DIM, 128, signs, 4, group, softmax_scale)
-    scores = O.kv_decode_scores(qbits, kc, ks, DIM, 128, signs, 4, group, softmax_scale)
+    want = O.kv_decode_attention(qbits, kc, ks, vc, vs, DIM, 128, signs, bits, group, softmax_scale)
+    scores = O.kv_decode_scores(qbits, kc, ks, DIM, 128, signs, bits, group, softmax_scale)
     nb, nkv, T = ks.shape[:3]
-    values = O.dequant_rotate_inv(vc.reshape(-1, DIM // 2), vs.reshape(-1), DIM, 128, signs, 4, group,
+    values = O.dequant_rotate_inv(vc.reshape(-1, DIM * bits // 8), vs.reshape(-1), DIM, 128, signs, bits, group,
                                   method="fwht").reshape(nb, nkv, T, DIM)
     return want, attention_allowance(want, scores, values, qbits.shape[1] // nkv)
 
@@ -256,3 +259,61 @@ def test_grouped_cache_rejections():
         B.hadq_kv_decode_attention(q, kc, ks8, kc, ks8, block=128, bits=4, group=16)
     assert e.value.status == B.HADQ_ERR_UNSUPPORTED
     assert B.hadq_launch_count() == n0
+
+
+INT8_CASES = [
+    # batch, n_q_heads, n_kv_heads, tokens, stride, signs, group
+    (1, 4, 1, 1, 1, False, 128),       # one cached token
+    (1, 4, 1, 16, 16, False, 128),     # one tile
+    (2, 8, 2, 37, 40, False, 128),     # ragged tail, stride > tokens
+    (1, 32, 8, 1000, 1000, True, 128), # GQA 4 with signs
+    (1, 16, 2, 513, 520, True, 128),   # two head groups per KV head
+    (1, 8, 1, 5000, 5000, False, 128), # many splits
+    (1, 8, 2, 300, 300, True, 64),     # groups of 64
+    (2, 8, 2, 37, 40, False, 32),      # groups of 32, ragged
+]
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("batch,nqh,nkv,tokens,stride,with_signs,group", INT8_CASES)
+def test_decode_attention_int8_cache(batch, nqh, nkv, tokens, stride, with_signs, group, out_dtype):
+    # caches quantised to INT8 (one scale per row, or per group of 64 or 32)
+    seed = 3000 + batch * 7 + nqh * 13 + tokens + group
+    signs = S.random_signs(DIM, seed) if with_signs else None
+    kc, ks, vc, vs = oracle_cache(batch, nkv, stride, seed, signs=signs, group=group, bits=8)
+    qbits = S.decode_query(batch, nqh, DIM, seed)
+    want = oracle_attention(qbits, kc[:, :, :tokens], ks[:, :, :tokens], vc[:, :, :tokens],
+                            vs[:, :, :tokens], signs, group=group, bits=8)
+    out = run_gpu(qbits, kc, ks, vc, vs, tokens, signs, out_dtype, group=group, bits=8)
+    compare(out, want, out_dtype, f"attention INT8 G={group} {batch}x{nqh}/{nkv} T={tokens}")
+
+
+def test_int8_cache_extreme_codes():
+    # every code at -128, -127 or +127 (the ends of the exact bf16 conversion)
+    rng = np.random.default_rng(17)
+    T = 200
+    kc = rng.choice(np.array([-128, -127, 127], np.int8), size=(1, 1, T, DIM))
+    vc = rng.choice(np.array([-128, -127, 127, 0, 1, -1], np.int8), size=(1, 1, T, DIM))
+    ks = rng.uniform(0.001, 0.01, size=(1, 1, T)).astype(np.float32)
+    vs = rng.uniform(0.001, 0.01, size=(1, 1, T)).astype(np.float32)
+    qbits = S.decode_query(1, 4, DIM, 17)
+    want = oracle_attention(qbits, kc, ks, vc, vs, bits=8)
+    out = run_gpu(qbits, kc, ks, vc, vs, T, None, torch.float32, bits=8)
+    compare(out, want, torch.float32, "INT8 extreme codes")
+
+
+def test_full_size_int8_decode_sampled_heads():
+    # the 131072-token decode shape with an INT8 cache, in the launch the
+    # benchmark times for it
+    dw = S.DECODE_WORKLOADS["d1_decode_q32_kv8_t131072_d128_int4"]
+    kc, ks = S.random_int8_cache(dw.batch, dw.n_kv_heads, dw.tokens, DIM, 81)
+    vc, vs = S.random_int8_cache(dw.batch, dw.n_kv_heads, dw.tokens, DIM, 82)
+    qbits = S.decode_query(dw.batch, dw.n_q_heads, DIM, 83)
+    out = run_gpu(qbits, kc, ks, vc, vs, dw.tokens, None, torch.bfloat16, bits=8)
+    g = dw.n_q_heads // dw.n_kv_heads
+    for kvh in (0, 3, 7):
+        sl = slice(kvh * g, (kvh + 1) * g)
+        want = oracle_attention(qbits[:, sl], kc[:, kvh:kvh + 1], ks[:, kvh:kvh + 1],
+                                vc[:, kvh:kvh + 1], vs[:, kvh:kvh + 1], bits=8)
+        compare(out[:, sl].contiguous(), want, torch.bfloat16, f"full size INT8, KV head {kvh}")
+    assert torch.isfinite(out.float()).all()

@@ -7,6 +7,8 @@ calls (nothing allocated per call): torch's allocator always, the device-wide
 free memory when no other process is on the device.
 """
 
+import gc
+
 import numpy as np
 import pytest
 import torch
@@ -63,6 +65,7 @@ def test_noalloc_matches_oracle_and_allocates_nothing(batch, nqh, nkv, tokens, w
     out = torch.empty((batch, nqh, DIM), dtype=torch.float32, device="cuda")
     B.hadq_kv_decode_attention_noalloc(*args, out=out, block=128, signs=sg, bits=4, group=128)
     torch.cuda.synchronize()
+    gc.collect()  # tensors of earlier tests freed now, not during the calls below
     free0, _ = torch.cuda.mem_get_info()
     alloc0 = torch.cuda.memory_allocated()
     n0 = B.hadq_launch_count()
@@ -70,7 +73,9 @@ def test_noalloc_matches_oracle_and_allocates_nothing(batch, nqh, nkv, tokens, w
         B.hadq_kv_decode_attention_noalloc(*args, out=out, block=128, signs=sg, bits=4, group=128)
     torch.cuda.synchronize()
     assert B.hadq_launch_count() == n0 + 3
-    assert torch.cuda.memory_allocated() == alloc0
+    # nothing allocated through torch (a collection of an earlier test's
+    # garbage could still lower the figure, never raise it)
+    assert torch.cuda.memory_allocated() <= alloc0
     if _alone_on_device():
         # a device allocation takes at least one 2 MiB page; other processes
         # on the device would move this figure, so it is read only when alone
