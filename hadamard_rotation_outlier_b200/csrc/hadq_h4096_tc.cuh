@@ -62,8 +62,9 @@ static_assert(kTcTileBlocks % kTcBpp == 0, "passes cover a tile");
 static_assert(kTcBpp == 1 || kTcBpp == 2 || kTcBpp == 4, "blocks per pass");
 constexpr int kTcStageBytes = kTcTileBlocks * 8192;
 constexpr int kTcABytes = 128 * 128 * 2;           // H_128 in bf16
+constexpr int kTcSignWarps = 4;
 constexpr int kTcSignWarp0 = 4 * kTcEpiWG;         // warps 0 .. 4 kTcEpiWG - 1: epilogue
-constexpr int kTcProdWarp = kTcSignWarp0 + 4;      // then four sign warps, the producer
+constexpr int kTcProdWarp = kTcSignWarp0 + kTcSignWarps;  // then the sign warps, the producer
 constexpr int kTcMmaWarp = kTcProdWarp + 1;        // and the MMA warp (also allocates TMEM)
 constexpr int kTcThreads = (kTcMmaWarp + 1) * 32;
 constexpr int kTcAccCols = 32 * kTcTileBlocks;    // N of the MMA
@@ -316,7 +317,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&tl->full[s], 1);
-      mbar_init(&tl->signd[s], 4);
+      mbar_init(&tl->signd[s], kTcSignWarps);
       mbar_init(&tl->empty[s], 1);
     }
     for (int c = 0; c < kTcAcc; ++c) {
