@@ -40,6 +40,8 @@
 
 namespace hadq {
 
+// Shape constants (the defaults are the measured best on the 16384 x 4096
+// workload; other values build for comparison).
 #ifndef HADQ_TC_EPI_WG
 #define HADQ_TC_EPI_WG 4
 #endif
@@ -62,7 +64,12 @@ static_assert(kTcTileBlocks % kTcBpp == 0, "passes cover a tile");
 static_assert(kTcBpp == 1 || kTcBpp == 2 || kTcBpp == 4, "blocks per pass");
 constexpr int kTcStageBytes = kTcTileBlocks * 8192;
 constexpr int kTcABytes = 128 * 128 * 2;           // H_128 in bf16
-constexpr int kTcSignWarps = 4;
+#ifndef HADQ_TC_SIGNW
+#define HADQ_TC_SIGNW 4
+#endif
+constexpr int kTcSignWarps = HADQ_TC_SIGNW;        // warps applying the signs
+constexpr int kTcSignPieces = 512 / (32 * kTcSignWarps);  // 16-byte pieces per thread and block image
+static_assert(kTcSignPieces * 32 * kTcSignWarps == 512, "sign pieces cover a block image");
 constexpr int kTcSignWarp0 = 4 * kTcEpiWG;         // warps 0 .. 4 kTcEpiWG - 1: epilogue
 constexpr int kTcProdWarp = kTcSignWarp0 + kTcSignWarps;  // then the sign warps, the producer
 constexpr int kTcMmaWarp = kTcProdWarp + 1;        // and the MMA warp (also allocates TMEM)
@@ -119,19 +126,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
 }
 __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
   uint32_t ok;
-#ifdef HADQ_TC_WAIT_HINT_NS
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_addr(b)), "r"(parity), "n"(HADQ_TC_WAIT_HINT_NS)
-      : "memory");
-#else
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
       : "r"(smem_addr(b)), "r"(parity)
       : "memory");
-#endif
   return ok != 0;
 }
 __device__ __forceinline__ unsigned long long global_ns() {
@@ -274,18 +273,7 @@ __device__ __forceinline__ float tc_h32_absmax(float (&v)[32]) {
   reg_stage<32, 2>(v);
   reg_stage<32, 4>(v);
   reg_stage<32, 8>(v);
-#ifdef HADQ_TC_MAX_AFTER
-  reg_stage<32, 16>(v);
-  float m0 = 0.0f, m1 = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    m0 = max3(m0, fabsf(v[i]), fabsf(v[i + 1]));
-    m1 = max3(m1, fabsf(v[i + 2]), fabsf(v[i + 3]));
-  }
-  return fmaxf(m0, m1);
-#else
   return reg_stage_absmax<32, 16>(v);
-#endif
 }
 
 template <int BITS, bool SIGNS>
@@ -391,14 +379,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
     }
   } else if (warp >= kTcSignWarp0) {
     if constexpr (SIGNS) {
-      // Thread st owns the 16-byte pieces st + 128 c (c = 0..3) of every 8 KB
+      // Thread st owns the 16-byte pieces st + 32 kTcSignWarps c of every 8 KB
       // block image.  Piece P holds h = P / 4 and the 8 values l = 8 ((P % 4)
       // XOR (h / 2) % 4) + e (the 64-byte swizzle).
       const int st = threadIdx.x - kTcSignWarp0 * 32;
-      uint4 mask[4];
+      constexpr int PS = 32 * kTcSignWarps;  // piece stride between a thread's pieces
+      uint4 mask[kTcSignPieces];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int P = st + 128 * c, h = P >> 2, l0 = 8 * ((P & 3) ^ ((h >> 1) & 3));
+      for (int c = 0; c < kTcSignPieces; ++c) {
+        const int P = st + PS * c, h = P >> 2, l0 = 8 * ((P & 3) ^ ((h >> 1) & 3));
         const int8_t* sg = a.signs + 32 * h + l0;
         mask[c] = make_uint4(pair_sign_mask(sg[0], sg[1]), pair_sign_mask(sg[2], sg[3]), pair_sign_mask(sg[4], sg[5]),
                              pair_sign_mask(sg[6], sg[7]));
@@ -415,13 +404,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
 #pragma unroll
         for (int r = 0; r < kTcTileBlocks; ++r)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 v = p[512 * r + 128 * c];
+          for (int c = 0; c < kTcSignPieces; ++c) {
+            uint4 v = p[512 * r + PS * c];
             v.x ^= mask[c].x;
             v.y ^= mask[c].y;
             v.z ^= mask[c].z;
             v.w ^= mask[c].w;
-            p[512 * r + 128 * c] = v;
+            p[512 * r + PS * c] = v;
           }
         fence_async_shared();  // the tensor cores read what this thread wrote
         __syncwarp();
