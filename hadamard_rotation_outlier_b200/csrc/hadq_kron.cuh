@@ -540,7 +540,9 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
       reg_fwht<16, 4>(v);
 #pragma unroll
       for (int kk = 0; kk < 16; ++kk) ((kk & 1) ? po : pe)[36 * (kk >> 1)] = v[kk];
-      __syncthreads();
+      // the 16 threads of row xi (t >> 4) are half of one warp and touch no
+      // other row, so the warp's own barrier orders the pass and the reads
+      __syncwarp();
       // the thread's 16 consecutive columns 16 u .. 16 u + 15: float4 i at
       // offset 4 (i ^ 2 (f & 1)) from the swizzled run start
       const float* base = ws + xi * pw + 36 * (u >> 1) + 16 * ((u & 1) ^ (f >> 1));
