@@ -34,7 +34,7 @@ KERNEL_SOURCES = {
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
     "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_mma.cuh", "hadq_kron.cuh", "k_kron.cu"],
     "h4096": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_h4096.cuh", "k_h4096.cu"],
-    "h4096tc": ["hadq_common.cuh", "hadq_h4096_tc.cuh", "k_h4096_tc.cu"],
+    "h4096tc": ["hadq_common.cuh", "hadq_tc.cuh", "hadq_h4096_tc.cuh", "k_h4096_tc.cu"],
 }
 
 TRAFFIC_FILE = "dram_traffic.txt"

@@ -81,12 +81,15 @@ def run_case(rows, dim, block, group, bits, with_signs, seed=1, dist="normal", o
 
 # (rows, dim, block, group, bits, signs, expected forward path)
 CASES = [
-    (300, 128, -1, -1, 8, False, "chunk_mma"),      # Q/K heads, INT8, per row
+    (300, 128, -1, -1, 8, False, "chunk_mma"),        # Q/K heads, INT8, per row
     (301, 128, 128, 128, 4, False, "chunk_mma"),    # KV rows, INT4, group 128
     (33, 384, 128, 128, 8, False, "chunk_mma"),     # three blocks per row, a short last slab
     (7, 11008, 128, 128, 4, False, "chunk_mma"),    # 86 blocks per row
     (1, 128, 128, 128, 4, False, "chunk_mma"),      # one block
     (65, 1024, 128, 128, 8, False, "chunk_mma"),
+    (1000, 11008, 128, 128, 4, True, "chunk_mma"),  # 86000 blocks: every warp takes several slabs
+    (640, 2560, 128, 128, 8, True, "chunk_mma"),    # INT8 with signs, 12800 blocks
+    (2049, 128, -1, -1, 4, False, "chunk_mma"),     # one block per row, a ragged last slab
     (37, 4096, 128, -1, 4, False, "chunk"),         # per-token scale over 32 blocks
     (9, 11008, 128, 128, 4, True, "chunk_mma"),     # 86 blocks, signs
     (45, 1152, 128, 128, 8, True, "chunk_mma"),     # signs, 9 blocks per row, a short last slab
