@@ -487,6 +487,8 @@ def kernel_name(wl) -> str:
         return KRON_KERNELS[B.hadq_kron_plan(0, wl.rows, wl.kron_a, wl.dim // wl.kron_a, wl.bits, wl.group)]
     if wl.asym:
         return "rq_chunk_asym_kernel"
+    if wl.keep:  # the kept-token calls run the chunk kernels' KEEP instances
+        return "rq_chunk_kernel"
     return KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)]
 
 
@@ -494,6 +496,8 @@ def dequant_kernel_name(wl) -> str:
     from hadamard_rotation_outlier_b200 import binding as B
     if wl.asym:
         return "dq_chunk_asym_kernel"
+    if wl.keep:
+        return "dq_chunk_kernel"
     path = B.hadq_plan(1, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)
     return {"chunk_mma": "dq_chunk_mma_kernel", "chunk": "dq_chunk_kernel", "blocked": "dq_blocked_kernel",
             "generic": "dq_generic_kernel"}.get(path, path)
