@@ -391,15 +391,18 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   const GenericArgs& a = k.g;
   extern __shared__ __align__(16) unsigned char tbuf[];
-  const int dim = a.dim, b = a.block, G = a.group, fa = k.a;
-  const int px = kron_tc_px(b), pw = kron_tc_pw(b);
+  // b = 256 (S256): the block and the shared-memory pitches are constants
+  const int dim = a.dim, b = S256 ? 256 : a.block, G = a.group, fa = k.a;
+  const int px = S256 ? kron_tc_px(256) : kron_tc_px(b), pw = S256 ? kron_tc_pw(256) : kron_tc_pw(b);
+  const int64_t nrows = a.rows;
+  const float scale_mul = a.scale_mul;
   unsigned char* xs = tbuf;
   float* ws = reinterpret_cast<float*>(tbuf + size_t(8) * KA * px);
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
   const int g = lane >> 2, t4 = lane & 3;
   const int e0 = 16 * t;
-  const int lb = kron_log2(b);
+  const int lb = S256 ? 8 : kron_log2(b);
   const int lanes_b = b >> 4, lanes_g = G >> 4;
   const int lg = kron_log2(G);
   const int gpr = dim >> lg, my_g = e0 >> lg;  // scale groups per row, this thread's group
@@ -460,13 +463,20 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
   const int half = (t >> 2) & 1;  // store order of the two 16-byte halves
 
   uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
-  if (int64_t(blockIdx.x) < a.rows) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + int64_t(blockIdx.x) * dim + e0);
+  // this thread's input, codes and scale for the current row, stepped by the
+  // grid's rows instead of recomputed from the row index
+  const int64_t xstep = int64_t(gridDim.x) * dim;
+  const uint16_t* xp = a.x + int64_t(blockIdx.x) * dim + e0;
+  uint8_t* cp = a.codes + (int64_t(blockIdx.x) * dim + e0) * BITS / 8;
+  float* sp = a.scales + int64_t(blockIdx.x) * gpr + my_g;
+  const int64_t cstep = xstep * BITS / 8, sstep = int64_t(gridDim.x) * gpr;
+  if (int64_t(blockIdx.x) < nrows) {
+    const uint4* src = reinterpret_cast<const uint4*>(xp);
     n0 = src[0];
     n1 = src[1];
   }
 
-  for (int64_t row = blockIdx.x; row < a.rows; row += gridDim.x) {
+  for (int64_t row = blockIdx.x; row < nrows; row += gridDim.x, xp += xstep, cp += cstep, sp += sstep) {
     const int64_t base = row * dim;
     {
       const uint4 s0 = make_uint4(n0.x ^ smask[0], n0.y ^ smask[1], n0.z ^ smask[2], n0.w ^ smask[3]);
@@ -475,15 +485,15 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
       dst[half] = half ? s1 : s0;
       dst[half ^ 1] = half ? s0 : s1;
     }
-    if (row + gridDim.x < a.rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(a.x + (row + gridDim.x) * dim + e0);
+    if (row + gridDim.x < nrows) {
+      const uint4* src = reinterpret_cast<const uint4*>(xp + xstep);
       n0 = src[0];
       n1 = src[1];
     }
     __syncthreads();
 
     // mixing: m-tile mt covers columns j = 16 mt .. 16 mt + 15
-    for (int mt = warp; mt < (b >> 4); mt += nwarps) {
+    for (int mt = warp; mt < (S256 ? 16 : (b >> 4)); mt += nwarps) {
       float d[KA][4];
 #pragma unroll
       for (int nt = 0; nt < KA; ++nt) d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0.0f;
@@ -578,7 +588,7 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
     for (int o = 1; o < lanes_g; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((t & (lanes_g - 1)) == 0) a.scales[row * gpr + my_g] = m * a.scale_mul;
+    if ((t & (lanes_g - 1)) == 0) *sp = m * scale_mul;
     if (a.rot) {
       float4* dst = reinterpret_cast<float4*>(a.rot + base + e0);
 #pragma unroll
@@ -599,11 +609,11 @@ __global__ void __maxnreg__((kron_tc_maxreg<KA, NS>())) rq_kron_tc_kernel(KronAr
       magic_code2(v[8 + 2 * i], v[9 + 2 * i], q.inv, cc1[2 * i], cc1[2 * i + 1]);
     }
     if constexpr (BITS == 8) {
-      *reinterpret_cast<uint4*>(a.codes + base + e0) =
+      *reinterpret_cast<uint4*>(cp) =
           make_uint4(pack_i8x4(cc0[0], cc0[1], cc0[2], cc0[3]), pack_i8x4(cc0[4], cc0[5], cc0[6], cc0[7]),
                      pack_i8x4(cc1[0], cc1[1], cc1[2], cc1[3]), pack_i8x4(cc1[4], cc1[5], cc1[6], cc1[7]));
     } else {
-      *reinterpret_cast<uint2*>(a.codes + (base + e0) / 2) = make_uint2(pack_i4x8(cc0), pack_i4x8(cc1));
+      *reinterpret_cast<uint2*>(cp) = make_uint2(pack_i4x8(cc0), pack_i4x8(cc1));
     }
   }
 }
