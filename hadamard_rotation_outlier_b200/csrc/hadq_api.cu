@@ -104,9 +104,11 @@ bool chunk_ok(int direction, const Shape& s) {
 
 hadq_path choose_path(int direction, const Shape& s, bool aligned16) {
   if (s.rows == 0) return HADQ_PATH_NONE;
-  if (aligned16 && direction == 0 && s.B == 128 && s.G == 128 && s.dim % 128 == 0)
+  // the tensor-core 128-point kernels index chunks with 32-bit integers
+  const bool mma_size_ok = s.rows * (s.dim / 128) < (int64_t(1) << 30);
+  if (aligned16 && direction == 0 && s.B == 128 && s.G == 128 && s.dim % 128 == 0 && mma_size_ok)
     return HADQ_PATH_CHUNK_MMA;
-  if (aligned16 && direction == 1 && s.B == 128 && s.G % 128 == 0 && s.dim % 128 == 0)
+  if (aligned16 && direction == 1 && s.B == 128 && s.G % 128 == 0 && s.dim % 128 == 0 && mma_size_ok)
     return HADQ_PATH_CHUNK_MMA;
   if (aligned16 && chunk_ok(direction, s)) return HADQ_PATH_CHUNK;
   if (aligned16 && direction == 0 && s.B == 4096 && s.dim % 4096 == 0 && s.G == 4096) {

@@ -117,12 +117,24 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkAr
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int g = lane >> 2, t4 = lane & 3;
   const uint2* s_sw = reinterpret_cast<const uint2*>(smem + chunk_mma_stage_bytes());
+  // Slab and chunk indices are 32-bit: the host takes this kernel only for
+  // fewer than 2^30 chunks (a 256 GiB input), so every index below, including
+  // the slab after next, stays under 2^31.  Byte offsets are widened.
+  const int wstride = int(gridDim.x) * kMmaWarps;
+  int slab = int(blockIdx.x) * kMmaWarps + wid;
+  const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
+  const int nslabs = int((a.nchunks + kMmaSlab - 1) / kMmaSlab);
+  uint8_t* st0 = smem + (2 * wid) * kMmaStageBytes;
+  uint8_t* st1 = st0 + kMmaStageBytes;
+  constexpr int SB = kMmaSlab * 256;  // input bytes per slab
+
+  // the first slab is in flight while the CTA builds its sign table
+  if (slab < nslabs) mma_slab_load<16>(xsrc + size_t(slab) * SB, slab_count(slab * kMmaSlab, a.nchunks, kMmaSlab), st0, lane);
+  cp_async_commit();
   if constexpr (SIGNS) {
     load_mma_sign_words(a.signs, a.cpr, reinterpret_cast<uint2*>(smem + chunk_mma_stage_bytes()));
     __syncthreads();
   }
-  const int64_t wstride = int64_t(gridDim.x) * kMmaWarps;
-  int64_t slab = int64_t(blockIdx.x) * kMmaWarps + wid;
   // column block of this warp's slab start, advanced from slab to slab
   int colc = SIGNS ? (int)((slab * kMmaSlab) % a.cpr) : 0;
   const int col_step = SIGNS ? (int)((wstride * kMmaSlab) % a.cpr) : 0;
@@ -144,26 +156,18 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkAr
   // half lane >> 4; tile row p adds 32 bytes
   const uint32_t lm_off = uint32_t(((lane & 7) + 8 * ((lane >> 3) & 1)) * kCPad + (lane >> 4) * 16);
 
-  const uint8_t* xsrc = reinterpret_cast<const uint8_t*>(a.x);
-  const int64_t nslabs = (a.nchunks + kMmaSlab - 1) / kMmaSlab;
-  uint8_t* st0 = smem + (2 * wid) * kMmaStageBytes;
-  uint8_t* st1 = st0 + kMmaStageBytes;
-  constexpr int SB = kMmaSlab * 256;  // input bytes per slab
-
-  if (slab < nslabs) mma_slab_load<16>(xsrc + slab * SB, slab_count(slab * kMmaSlab, a.nchunks, kMmaSlab), st0, lane);
-  cp_async_commit();
   for (int it = 0; slab < nslabs; ++it, slab += wstride) {
     uint8_t* cur = (it & 1) ? st1 : st0;
-    const int64_t c = slab * kMmaSlab;
+    const int c = slab * kMmaSlab;
     cp_async_wait<0>();
     __syncwarp();
     {
-      const int64_t nx = slab + wstride;
-      if (nx < nslabs) mma_slab_load<16>(xsrc + nx * SB, slab_count(nx * kMmaSlab, a.nchunks, kMmaSlab), (it & 1) ? st0 : st1, lane);
+      const int nx = slab + wstride;
+      if (nx < nslabs) mma_slab_load<16>(xsrc + size_t(nx) * SB, slab_count(nx * kMmaSlab, a.nchunks, kMmaSlab), (it & 1) ? st0 : st1, lane);
       cp_async_commit();
-      const int64_t n2 = nx + wstride;  // the slab after: into L2 now, staged next iteration
+      const int n2 = nx + wstride;  // the slab after: into L2 now, staged next iteration
       if (lane == 0 && n2 < nslabs)
-        prefetch_l2_bulk(xsrc + n2 * SB, uint32_t(slab_count(n2 * kMmaSlab, a.nchunks, kMmaSlab)) * 256u);
+        prefetch_l2_bulk(xsrc + size_t(n2) * SB, uint32_t(slab_count(n2 * kMmaSlab, a.nchunks, kMmaSlab)) * 256u);
     }
     const int nch = slab_count(c, a.nchunks, kMmaSlab);  // blocks beyond nch hold stale data: computed, never stored
     // sign words of this lane's blocks g + 8 r
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkAr
       if (t4 == 0 && live) a.scales[c + b] = m * a.scale_mul;
       if constexpr (ROT) {
         if (live) {
-          float* rr = a.rot + (c + b) * kCK + 4 * t4;
+          float* rr = a.rot + size_t(c + b) * kCK + 4 * t4;
 #pragma unroll
           for (int p = 0; p < 8; ++p)
             *reinterpret_cast<float4*>(rr + 16 * p) = make_float4(v[8 * p] * a.rsqrt_b, v[8 * p + 1] * a.rsqrt_b,
@@ -266,7 +270,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkAr
       }
     }
     __syncwarp();
-    mma_slab_store<CB / 16>(cur, nch, a.codes + c * CB, lane);
+    mma_slab_store<CB / 16>(cur, nch, a.codes + size_t(c) * CB, lane);
   }
   cp_async_wait<0>();
 }

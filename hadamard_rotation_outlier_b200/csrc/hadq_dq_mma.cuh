@@ -123,10 +123,6 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
   uint8_t* ostage = wbase + L::NS * 32 * L::CP;
   uint4* s_tab = reinterpret_cast<uint4*>(smem + (kCT / 32) * L::WARP_BYTES);
   const uint8_t* s_bytes = smem + (kCT / 32) * L::WARP_BYTES + kSignTabBytes;
-  if constexpr (SIGNS) {
-    load_sign_tables(a.signs, a.dim, s_tab, reinterpret_cast<uint32_t*>(smem + (kCT / 32) * L::WARP_BYTES + kSignTabBytes));
-    __syncthreads();
-  }
 
   // B fragments: H_16 entries between k-slot and column Q values (INT4:
   // high-nibble rows at 1/16), as f16 pairs {B[k][n], B[k + 1][n]} with
@@ -152,27 +148,35 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
   // group of 16, segment + (lane >> 4)
   const uint32_t lm_off = uint32_t(((lane & 7) + 8 * ((lane >> 3) & 1)) * L::CP + (lane >> 4) * 16);
 
-  const int64_t nslabs = (a.nchunks + 31) / 32;
-  const int64_t wstride = int64_t(gridDim.x) * (kCT / 32);
-  int64_t slab = int64_t(blockIdx.x) * (kCT / 32) + wid;
+  // Slab and chunk indices are 32-bit: the host takes this kernel only for
+  // fewer than 2^30 chunks, so every index below, including the slabs staged
+  // ahead, stays under 2^31.  Byte offsets are widened.
+  const int nslabs = int((a.nchunks + 31) / 32);
+  const int wstride = int(gridDim.x) * (kCT / 32);
+  int slab = int(blockIdx.x) * (kCT / 32) + wid;
   int colc = SIGNS ? (int)((slab * 32) % a.cpr) : 0;
   const int col_step = SIGNS ? (int)((wstride * 32) % a.cpr) : 0;
-  auto block_scale = [&](int64_t blk) {
+  auto block_scale = [&](int blk) {
     return blk < a.nchunks ? __ldg(a.scales_in + (a.gpc == 1 ? blk : blk / a.gpc)) : 0.0f;
   };
   // prologue: the first NS - 1 slabs of this warp in flight, the scales of the first
 #pragma unroll
   for (int k = 0; k < L::NS - 1; ++k) {
-    const int64_t sk = slab + k * wstride;
-    if (sk < nslabs) dq_mma_load<BITS>(a.codes_in + sk * 32 * L::CB, slab_count(sk * 32, a.nchunks, 32), wbase + k * 32 * L::CP, lane);
+    const int sk = slab + k * wstride;
+    if (sk < nslabs) dq_mma_load<BITS>(a.codes_in + size_t(sk) * (32 * L::CB), slab_count(sk * 32, a.nchunks, 32), wbase + k * 32 * L::CP, lane);
     cp_async_commit();
+  }
+  // the sign tables are built while those copies are in flight
+  if constexpr (SIGNS) {
+    load_sign_tables(a.signs, a.dim, s_tab, reinterpret_cast<uint32_t*>(smem + (kCT / 32) * L::WARP_BYTES + kSignTabBytes));
+    __syncthreads();
   }
   float sc_next[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) sc_next[i] = slab < nslabs ? block_scale(slab * 32 + g + 8 * i) : 0.0f;
   for (int it = 0; slab < nslabs; ++it, slab += wstride) {
     uint8_t* cur = wbase + (it % L::NS) * 32 * L::CP;
-    const int64_t c = slab * 32;
+    const int c = slab * 32;
     float sc[4];  // scales of this lane's blocks g + 8 i (i = 2 grp + r)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
@@ -180,15 +184,15 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
     __syncwarp();
     {
       // the stage read in the previous iteration takes the slab NS - 1 ahead
-      const int64_t nf = slab + (L::NS - 1) * wstride;
+      const int nf = slab + (L::NS - 1) * wstride;
       if (nf < nslabs)
-        dq_mma_load<BITS>(a.codes_in + nf * 32 * L::CB, slab_count(nf * 32, a.nchunks, 32),
+        dq_mma_load<BITS>(a.codes_in + size_t(nf) * (32 * L::CB), slab_count(nf * 32, a.nchunks, 32),
                           wbase + ((it + L::NS - 1) % L::NS) * 32 * L::CP, lane);
       cp_async_commit();
-      const int64_t n2 = nf + wstride;  // the slab after: into L2 now, staged next iteration
+      const int n2 = nf + wstride;  // the slab after: into L2 now, staged next iteration
       if (lane == 0 && n2 < nslabs)
-        prefetch_l2_bulk(a.codes_in + n2 * 32 * L::CB, uint32_t(slab_count(n2 * 32, a.nchunks, 32)) * L::CB);
-      const int64_t nx = slab + wstride;
+        prefetch_l2_bulk(a.codes_in + size_t(n2) * (32 * L::CB), uint32_t(slab_count(n2 * 32, a.nchunks, 32)) * L::CB);
+      const int nx = slab + wstride;
 #pragma unroll
       for (int i = 0; i < 4; ++i) sc_next[i] = nx < nslabs ? block_scale(nx * 32 + g + 8 * i) : 0.0f;
     }
@@ -307,7 +311,7 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
           }
           if constexpr (OUT_F32) {
             if (b < nch) {
-              float* dst = a.rot + (c + b) * kCK + j0;
+              float* dst = a.rot + size_t(c + b) * kCK + j0;
               const uint32_t mm[4] = {m4.x, m4.y, m4.z, m4.w};
               uint32_t o[8];
 #pragma unroll
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kCT, 3) dq_chunk_mma_kernel(ChunkArgs a) {
       fence_async_shared();  // the run stores are visible to the copy engine
       __syncwarp();
       if (lane == 0) {
-        bulk_store_s2g(reinterpret_cast<uint8_t*>(a.out_bf16) + c * 256, ostage, uint32_t(nch) * 256u);
+        bulk_store_s2g(reinterpret_cast<uint8_t*>(a.out_bf16) + size_t(c) * 256, ostage, uint32_t(nch) * 256u);
         bulk_commit();
       }
     }

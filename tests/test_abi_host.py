@@ -95,6 +95,9 @@ def test_plan_rejects(lib, args, msg):
     (1, 100, 1024, 64, 4, 128, False, True, "chunk"),             # dequant, 64-point blocks
     (1, 10, 1024, 256, 4, 64, False, True, "blocked"),            # 256-point dequant
     (0, 32768, 11008, 128, 4, 128, True, True, "chunk_mma"),      # 86 blocks of 128, signs
+    (0, 1 << 27, 1024, 128, 4, 128, False, True, "chunk"),        # 2^30 chunks: past 32-bit chunk indices
+    (0, (1 << 27) - 1, 1024, 128, 4, 128, False, True, "chunk_mma"),  # the largest count that stays
+    (1, 1 << 27, 1024, 128, 4, 128, False, True, "chunk"),        # the same limit for the dequantiser
     (0, 10, 1024, 256, 4, 64, True, True, "blocked"),             # 256-point blocks
     (0, 10, 96, 32, 8, -1, False, True, "blocked"),               # dim not a multiple of 128
     (0, 10, 32768, 128, 4, -1, False, True, "generic"),           # whole-row groups past 16384
