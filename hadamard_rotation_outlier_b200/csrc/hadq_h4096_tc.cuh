@@ -291,8 +291,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
       bool stop = false;
 #pragma unroll 1
       for (int pr = 0; pr < kTcTileBlocks / kTcBpp; ++pr) {
+        // A warp that gave up still reads its accumulator (allocated TMEM, so
+        // the read is safe); its values are never stored.
         float v[kTcBpp][32];
-        if (ok) {
+        {
           const uint32_t ta = tmem + (uint32_t(32 * q) << 16) + uint32_t(c * kTcAccCols + 32 * kTcBpp * pr);
           if constexpr (kTcBpp == 2) {
             tmem_ld64(ta, v[0], v[1]);
@@ -300,11 +302,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
 #pragma unroll
             for (int b = 0; b < kTcBpp; ++b) tmem_ld32(ta + 32 * b, v[b]);
           }
-        } else {
-#pragma unroll
-          for (int b = 0; b < kTcBpp; ++b)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[b][j] = 0.0f;
         }
         if (pr == kTcTileBlocks / kTcBpp - 1) {  // the accumulator has been read
           tc_fence_before();
