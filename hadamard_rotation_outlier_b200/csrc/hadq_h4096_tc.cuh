@@ -23,10 +23,10 @@
 //    (K-major, 128-byte swizzle, written once per CTA); B = the stage
 //    (MN-major, 64-byte swizzle, as the TMA left it).  Commits release the
 //    stage and hand the accumulator on;
-//  * epilogue (kTcEpiWG warpgroups, taking tiles in turn): tcgen05.ld of two
-//    blocks (64 columns) at a time, five butterfly stages, block maxima by
-//    warp reduction and one named barrier per pair of blocks, codes and
-//    scales to global memory.
+//  * epilogue (one warpgroup per block of a tile, so the four work on the
+//    same tile at once): tcgen05.ld of the block's 32 columns, five butterfly
+//    stages, the block maximum by warp reduction and one named barrier,
+//    codes and scales to global memory.
 // Every mbarrier wait gives up after about a second: the kernel then records
 // a fault (hadq_device_status reads it), every role leaves its loop, copies
 // still in flight are awaited (bounded), and the CTA frees its TMEM.
@@ -43,12 +43,6 @@ namespace hadq {
 
 // Shape constants (the defaults are the measured best on the 16384 x 4096
 // workload; other values build for comparison).
-#ifndef HADQ_TC_EPI_WG
-#define HADQ_TC_EPI_WG 4
-#endif
-#ifndef HADQ_TC_BPP
-#define HADQ_TC_BPP 1
-#endif
 #ifndef HADQ_TC_TILE
 #define HADQ_TC_TILE 4
 #endif
@@ -58,11 +52,8 @@ namespace hadq {
 constexpr int kTcTileBlocks = HADQ_TC_TILE;        // 4096-point blocks per tile (N = 32 per block)
 constexpr int kTcStages = HADQ_TC_STAGES;          // input stages of one tile each
 constexpr int kTcAcc = 16 / kTcTileBlocks;         // TMEM accumulators (512 columns in all)
-constexpr int kTcEpiWG = HADQ_TC_EPI_WG;           // epilogue warpgroups
-constexpr int kTcBpp = HADQ_TC_BPP;                // blocks per epilogue pass (one barrier each)
+constexpr int kTcEpiWG = kTcTileBlocks;            // epilogue warpgroups: one per block of a tile
 static_assert(kTcTileBlocks == 2 || kTcTileBlocks == 4, "tiles of 2 or 4 blocks");
-static_assert(kTcTileBlocks % kTcBpp == 0, "passes cover a tile");
-static_assert(kTcBpp == 1 || kTcBpp == 2 || kTcBpp == 4, "blocks per pass");
 constexpr int kTcStageBytes = kTcTileBlocks * 8192;
 constexpr int kTcABytes = 128 * 128 * 2;           // H_128 in bf16
 #ifndef HADQ_TC_SIGNW
@@ -86,8 +77,8 @@ struct TcTail {
   uint64_t empty[kTcStages];   // MMAs done reading the stage
   uint64_t tfull[kTcAcc];      // accumulator written
   uint64_t tempty[kTcAcc];     // accumulator read by its warpgroup
-  alignas(16) uint32_t red[kTcEpiWG][2][kTcBpp][4];  // [group][parity][block of the pass][warp]:
-                                                     // max bits, read back as 16-byte vectors
+  alignas(16) uint32_t red[kTcEpiWG][2][4];  // [group][parity][warp]: max bits, read back as
+                                             // 16-byte vectors
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -170,7 +161,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
     }
     for (int c = 0; c < kTcAcc; ++c) {
       mbar_init(&tl->tfull[c], 1);
-      mbar_init(&tl->tempty[c], 4);
+      mbar_init(&tl->tempty[c], 4 * kTcEpiWG);
     }
     tl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -278,67 +269,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) rq_h4096_tc_kernel(const __grid
       }
     }
   } else {
-    // Epilogue warpgroup g: warp q = warp % 4 reads TMEM lanes 32 q .. 32 q + 31.
+    // Epilogue warpgroup g takes block g of every tile; its warp q = warp % 4
+    // reads TMEM lanes 32 q .. 32 q + 31.
     const int g = warp >> 2, q = warp & 3, h = 32 * q + lane;
     constexpr int CODE_BYTES = BITS == 8 ? 32 : 16;
     uint32_t par = 0;
     int it = 0;
     for (int64_t t = first; t < a.ntiles; t += step, ++it) {
-      if (it % kTcEpiWG != g) continue;
       const int c = it % kTcAcc;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tl->tfull[c], (it / kTcAcc) & 1, abort));
       tc_fence_after();
-      bool stop = false;
-#pragma unroll 1
-      for (int pr = 0; pr < kTcTileBlocks / kTcBpp; ++pr) {
-        // A warp that gave up still reads its accumulator (allocated TMEM, so
-        // the read is safe); its values are never stored.
-        float v[kTcBpp][32];
-        {
-          const uint32_t ta = tmem + (uint32_t(32 * q) << 16) + uint32_t(c * kTcAccCols + 32 * kTcBpp * pr);
-          if constexpr (kTcBpp == 2) {
-            tmem_ld64(ta, v[0], v[1]);
-          } else {
-#pragma unroll
-            for (int b = 0; b < kTcBpp; ++b) tmem_ld32(ta + 32 * b, v[b]);
-          }
-        }
-        if (pr == kTcTileBlocks / kTcBpp - 1) {  // the accumulator has been read
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tl->tempty[c]);
-        }
-        // non-negative floats order as their bit patterns; a warp that gave up
-        // votes ~0, which no |y| can reach
-#pragma unroll
-        for (int b = 0; b < kTcBpp; ++b) {
-          const float m = tc_h32_absmax(v[b]);
-          const uint32_t mb = __reduce_max_sync(0xffffffffu, ok ? __float_as_uint(m) : ~0u);
-          if (lane == 0) tl->red[g][par][b][q] = mb;
-        }
-        named_bar_sync(1 + g, 128);
-        uint32_t M[kTcBpp];
-#pragma unroll
-        for (int b = 0; b < kTcBpp; ++b) {
-          const uint4 r = *reinterpret_cast<const uint4*>(tl->red[g][par][b]);  // after the barrier
-          M[b] = max(max(r.x, r.y), max(r.z, r.w));
-          if (M[b] == ~0u) stop = true;
-        }
-        par ^= 1u;
-        if (stop) break;
-#pragma unroll
-        for (int b = 0; b < kTcBpp; ++b) {
-          const int64_t blk = t * kTcTileBlocks + kTcBpp * pr + b;
-          if (blk < a.nblocks) {
-            const float m = __uint_as_float(M[b]);
-            if (h == 0) a.scales[blk] = m * a.scale_mul;
-            tc_store_codes<BITS>(v[b], m, a.codes + blk * (4096 * BITS / 8) + h * CODE_BYTES);
-          }
-        }
-      }
-      if (stop) {
+      // A warp that gave up still reads its accumulator (allocated TMEM, so
+      // the read is safe); its values are never stored.
+      float v[32];
+      tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(c * kTcAccCols + 32 * g), v);
+      tc_fence_before();  // this warp's part of the accumulator has been read
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->tempty[c]);
+      // non-negative floats order as their bit patterns; a warp that gave up
+      // votes ~0, which no |y| can reach
+      const float m = tc_h32_absmax(v);
+      const uint32_t mb = __reduce_max_sync(0xffffffffu, ok ? __float_as_uint(m) : ~0u);
+      if (lane == 0) tl->red[g][par][q] = mb;
+      named_bar_sync(1 + g, 128);
+      const uint4 r = *reinterpret_cast<const uint4*>(tl->red[g][par]);  // after the barrier
+      const uint32_t M = max(max(r.x, r.y), max(r.z, r.w));
+      par ^= 1u;
+      if (M == ~0u) {
         if (h == 0) tc_give_up(&tl->abort, a.fault);
         break;
+      }
+      const int64_t blk = t * kTcTileBlocks + g;
+      if (blk < a.nblocks) {
+        const float mf = __uint_as_float(M);
+        if (h == 0) a.scales[blk] = mf * a.scale_mul;
+        tc_store_codes<BITS>(v, mf, a.codes + blk * (4096 * BITS / 8) + h * CODE_BYTES);
       }
     }
   }
