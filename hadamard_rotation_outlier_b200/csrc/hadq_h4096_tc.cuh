@@ -76,7 +76,7 @@ struct TcTail {
   uint64_t signd[kTcStages];   // signs applied (signed calls)
   uint64_t empty[kTcStages];   // MMAs done reading the stage
   uint64_t tfull[kTcAcc];      // accumulator written
-  uint64_t tempty[kTcAcc];     // accumulator read by its warpgroup
+  uint64_t tempty[kTcAcc];     // accumulator read by every epilogue warp
   alignas(16) uint32_t red[kTcEpiWG][2][4];  // [group][parity][warp]: max bits, read back as
                                              // 16-byte vectors
   uint32_t tmem_base;
