@@ -109,8 +109,11 @@ __host__ __device__ inline size_t chunk_mma_smem_bytes(int dim, bool signs) {
 
 // ROT: also write the rotated float32 values (a.rot); a separate instance so
 // that the codes-only kernel carries no registers for them.
+// Four CTAs per SM (112 registers): with the five-CTA cap (95 registers) the
+// compiler recomputed masks and addresses in every slab, 50 more
+// instructions per slab, and the kernel ran 2-5 % slower.
 template <int BITS, bool SIGNS, bool ROT>
-__global__ void __launch_bounds__(kMmaWarps * 32, 5) rq_chunk_mma_kernel(ChunkArgs a) {
+__global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkArgs a) {
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per block
   extern __shared__ __align__(16) uint8_t smem[];
