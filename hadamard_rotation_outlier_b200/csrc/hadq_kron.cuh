@@ -377,12 +377,13 @@ __device__ __forceinline__ void bf16_split3(float f, uint32_t (&t)[3]) {
 // S256 (b = 256): bits 4-7 of the column index run as a strided pass over W
 // (16 columns u + 16 k per thread, 4 register stages, written back) before the
 // consecutive pass, instead of four lane-shuffle stages.
-// Register caps: 64 (a 320-thread CTA three times per SM) wherever the B
-// fragments allow it, 96 (twice) for the three-term split of a <= 24, 128 for
-// a <= 32 with the split.
+// Register caps: 64 (a 320-thread CTA three times per SM) for a <= 16, 96
+// (twice) for 16 < a <= 24 and for the three-term split of a <= 24, 128 for
+// a <= 32 with the split.  For the +-1 factor of a = 20, 96 registers and
+// two CTAs ran 2.5 % faster than 64 registers and three.
 template <int KA, int NS>
 constexpr int kron_tc_maxreg() {
-  return NS == 3 ? (KA <= 2 ? 64 : KA == 3 ? 96 : 128) : (KA <= 3 ? 64 : 96);
+  return NS == 3 ? (KA <= 2 ? 64 : KA == 3 ? 96 : 128) : (KA <= 2 ? 64 : 96);
 }
 
 template <int BITS, int KA, int NS, bool S256>
