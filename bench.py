@@ -487,8 +487,9 @@ def kernel_name(wl) -> str:
         return KRON_KERNELS[B.hadq_kron_plan(0, wl.rows, wl.kron_a, wl.dim // wl.kron_a, wl.bits, wl.group)]
     if wl.asym:
         return "rq_chunk_asym_kernel"
-    if wl.keep:  # the kept-token calls run the chunk kernels' KEEP instances
-        return "rq_chunk_kernel"
+    if wl.keep:  # the kept-token calls run KEEP instances: the tensor-core quantiser for 128-point
+        # blocks with a scale per block, else the chunk kernel
+        return "rq_chunk_mma_kernel" if wl.block == 128 and wl.group == 128 else "rq_chunk_kernel"
     return KERNEL_NAMES[B.hadq_plan(0, wl.rows, wl.dim, wl.block, wl.bits, wl.group, wl.with_signs, True)]
 
 

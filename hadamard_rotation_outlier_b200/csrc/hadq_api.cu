@@ -296,7 +296,10 @@ hadq_status launch_chunk(int direction, const Shape& s, hadq::ChunkArgs a, bool 
   return launch_chunk_args(direction, s, ka, false, f32, stream);
 }
 
-hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+// `ka` carries the kept-token table when `keep`; the plain kernels read only
+// its ChunkArgs base.
+hadq_status launch_chunk_mma_args(const Shape& s, hadq::ChunkKeepArgs ka, bool keep, cudaStream_t stream) {
+  hadq::ChunkArgs& a = ka;
   a.cpr = s.dim / hadq::kCK;
   a.nchunks = s.rows * a.cpr;
   a.slab_chunks = hadq::kMmaSlab;
@@ -304,7 +307,8 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
   a.dim = s.dim;
   a.log_g = 7;
   a.gpc = 1;
-  const void* fn = hadq::chunk_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr);
+  const void* fn = keep ? hadq::keep_chunk_mma_kernel_ptr(s.bits, s.has_signs)
+                        : hadq::chunk_mma_kernel_ptr(s.bits, s.has_signs, a.rot != nullptr);
   const size_t smem = hadq::chunk_mma_smem_bytes(s.dim, s.has_signs);
   const int threads = hadq::kMmaWarps * 32;
   int res = 1;
@@ -315,7 +319,7 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
   const int64_t slabs = (a.nchunks + hadq::kMmaSlab - 1) / hadq::kMmaSlab;
   const int64_t want = (slabs + hadq::kMmaWarps - 1) / hadq::kMmaWarps;  // one slab per warp
   const unsigned grid = (unsigned)(want < cap ? want : cap);
-  void* args[] = {&a};
+  void* args[] = {&ka};
   e = cudaLaunchKernel(fn, dim3(grid), dim3(threads), args, smem, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -323,6 +327,12 @@ hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t str
     return fail(HADQ_ERR_CUDA, "128-block tensor-core kernel launch failed: %s", cudaGetErrorString(e));
   }
   return after_launch("128-block tensor-core kernel");
+}
+
+hadq_status launch_chunk_mma(const Shape& s, hadq::ChunkArgs a, cudaStream_t stream) {
+  hadq::ChunkKeepArgs ka{};
+  static_cast<hadq::ChunkArgs&>(ka) = a;
+  return launch_chunk_mma_args(s, ka, false, stream);
 }
 
 hadq_status launch_dq_chunk_mma(const Shape& s, hadq::ChunkArgs a, bool f32, cudaStream_t stream) {
@@ -847,6 +857,11 @@ static hadq_status keep_check(const Shape& s, int64_t heads, int64_t tokens, con
   return HADQ_OK;
 }
 
+// Kept-token quantise calls that the 128-point tensor-core kernel takes.
+static bool keep_mma_ok(const Shape& s) {
+  return s.B == 128 && s.G == 128 && s.dim % 128 == 0 && s.rows * (s.dim / 128) < (int64_t(1) << 30);
+}
+
 hadq_status hadq_rotate_quantize_keep(const void* x, int64_t heads, int64_t tokens, int32_t dim, int32_t block,
                                       const int8_t* signs, int32_t bits, int32_t group, const int32_t* keep_slot,
                                       int32_t n_keep, void* codes, float* scales, void* kept,
@@ -877,6 +892,9 @@ hadq_status hadq_rotate_quantize_keep(const void* x, int64_t heads, int64_t toke
   a.kept = static_cast<uint16_t*>(kept);
   a.keep_tokens = tokens;
   a.n_keep = n_keep;
+  // 128-point blocks with one scale per block take the tensor-core quantiser
+  // (32-bit chunk indices), the rest the chunk kernels
+  if (keep_mma_ok(s)) return launch_chunk_mma_args(s, a, true, reinterpret_cast<cudaStream_t>(stream));
   return launch_chunk_args(0, s, a, true, false, reinterpret_cast<cudaStream_t>(stream));
 }
 

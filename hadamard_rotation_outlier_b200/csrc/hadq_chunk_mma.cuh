@@ -109,11 +109,15 @@ __host__ __device__ inline size_t chunk_mma_smem_bytes(int dim, bool signs) {
 
 // ROT: also write the rotated float32 values (a.rot); a separate instance so
 // that the codes-only kernel carries no registers for them.
+// KEEP: kept-token rows (the keep table of ChunkKeepArgs) leave as bf16 copies
+// in a.kept, with codes and scale 0; each lane looks up the keep-table entries
+// of its two blocks one slab ahead.
 // Four CTAs per SM (112 registers): with the five-CTA cap (95 registers) the
 // compiler recomputed masks and addresses in every slab, 50 more
 // instructions per slab, and the kernel ran 2-5 % slower.
-template <int BITS, bool SIGNS, bool ROT>
-__global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkArgs a) {
+template <int BITS, bool SIGNS, bool ROT, bool KEEP = false>
+__global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkArgsT<KEEP> a) {
+  static_assert(!(ROT && KEEP), "kept-token calls write no rotated values");
   constexpr float QMAX = (float)((1 << (BITS - 1)) - 1);
   constexpr int CB = BITS == 8 ? 128 : 64;  // code bytes per block
   extern __shared__ __align__(16) uint8_t smem[];
@@ -134,6 +138,14 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
   // the first slab is in flight while the CTA builds its sign table
   if (slab < nslabs) mma_slab_load<16>(xsrc + size_t(slab) * SB, slab_count(slab * kMmaSlab, a.nchunks, kMmaSlab), st0, lane);
   cp_async_commit();
+  int ks_next[2] = {-1, -1};  // KEEP: keep-table entries of blocks g, g + 8 of the next slab
+  if constexpr (KEEP) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int ch = slab * kMmaSlab + g + 8 * r;
+      if (slab < nslabs && ch < a.nchunks) ks_next[r] = kept_slot_of(a, ch);
+    }
+  }
   if constexpr (SIGNS) {
     load_mma_sign_words(a.signs, a.cpr, reinterpret_cast<uint2*>(smem + chunk_mma_stage_bytes()));
     __syncthreads();
@@ -162,12 +174,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
   for (int it = 0; slab < nslabs; ++it, slab += wstride) {
     uint8_t* cur = (it & 1) ? st1 : st0;
     const int c = slab * kMmaSlab;
+    const int ks[2] = {ks_next[0], ks_next[1]};
     cp_async_wait<0>();
     __syncwarp();
     {
       const int nx = slab + wstride;
       if (nx < nslabs) mma_slab_load<16>(xsrc + size_t(nx) * SB, slab_count(nx * kMmaSlab, a.nchunks, kMmaSlab), (it & 1) ? st0 : st1, lane);
       cp_async_commit();
+      if constexpr (KEEP) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int ch = nx * kMmaSlab + g + 8 * r;
+          ks_next[r] = (nx < nslabs && ch < a.nchunks) ? kept_slot_of(a, ch) : -1;
+        }
+      }
       const int n2 = nx + wstride;  // the slab after: into L2 now, staged next iteration
       if (lane == 0 && n2 < nslabs)
         prefetch_l2_bulk(xsrc + size_t(n2) * SB, uint32_t(slab_count(n2 * kMmaSlab, a.nchunks, kMmaSlab)) * 256u);
@@ -212,6 +232,23 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
     reg_stage<64, 8>(u);
     reg_stage<64, 16>(u);
     reg_stage<64, 32>(u);
+    // KEEP: a kept block's staged bf16 input goes out unchanged, 64 bytes per
+    // lane of its four, before its slot takes the codes
+    bool kept[2] = {false, false};
+    if constexpr (KEEP) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int b = g + 8 * r;
+        const int64_t kofs = b < nch ? kept_offset(a, c + b, ks[r]) : -1;
+        if (kofs >= 0) {
+          kept[r] = true;
+          const uint4* src = reinterpret_cast<const uint4*>(cur + b * kCPad + 64 * t4);
+          uint4* dst = reinterpret_cast<uint4*>(a.kept + kofs + 32 * t4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = src[i];
+        }
+      }
+    }
     __syncwarp();  // every lane has loaded its fragments: the slots take the codes
 
     // 3. per block: maximum, scale, codes
@@ -229,6 +266,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
       float m = fmaxf(m0, m1);
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if constexpr (KEEP)
+        if (kept[r]) m = 0.0f;  // scale 0
       const int b = g + 8 * r;
       const bool live = b < nch;
       if (t4 == 0 && live) a.scales[c + b] = m * a.scale_mul;
@@ -255,7 +294,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
           uint32_t c0, c1, c2, c3;
           magic_code2(v[8 * p], v[8 * p + 1], q.inv, c0, c1);
           magic_code2(v[8 * p + 2], v[8 * p + 3], q.inv, c2, c3);
-          *reinterpret_cast<uint32_t*>(slot + 16 * p + 4 * t4) = pack_i8x4(c0, c1, c2, c3);  // outputs 16 p + 4 t4 .. + 3
+          const uint32_t wd = (KEEP && kept[r]) ? 0u : pack_i8x4(c0, c1, c2, c3);
+          *reinterpret_cast<uint32_t*>(slot + 16 * p + 4 * t4) = wd;  // outputs 16 p + 4 t4 .. + 3
         }
       } else {
         // rows p and p + 1 in one word: its low half holds outputs 16 p + 4 t4 .. + 3, the high half those of p + 1
@@ -266,7 +306,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
           magic_code2(v[8 * p + 2], v[8 * p + 3], q.inv, cc[2], cc[3]);
           magic_code2(v[8 * p + 8], v[8 * p + 9], q.inv, cc[4], cc[5]);
           magic_code2(v[8 * p + 10], v[8 * p + 11], q.inv, cc[6], cc[7]);
-          const uint32_t wd = pack_i4x8(cc);
+          const uint32_t wd = (KEEP && kept[r]) ? 0u : pack_i4x8(cc);
           *reinterpret_cast<uint16_t*>(slot + 8 * p + 2 * t4) = (uint16_t)(wd & 0xffffu);
           *reinterpret_cast<uint16_t*>(slot + 8 * p + 8 + 2 * t4) = (uint16_t)(wd >> 16);
         }

@@ -22,6 +22,8 @@ inline const void* dq_chunk_kernel_ptr(int bits, int B, bool signs, bool scale_f
 // Kept-token variants (groups of >= 128 columns, warp teams).
 const void* keep_chunk_kernel_ptr(int bits, int B, bool signs);
 const void* keep_dq_chunk_kernel_ptr(int bits, int B, bool signs, bool f32);
+// Kept-token variant of the 128-point tensor-core quantiser (B = G = 128).
+const void* keep_chunk_mma_kernel_ptr(int bits, bool signs);
 // Kronecker rotation F (x) H_b (direction 0 forward, 1 inverse), 256 threads.
 const void* kron_kernel_ptr(int direction, int bits);
 // Forward register variant (b and G in 16..512, dim / 16 threads per CTA).

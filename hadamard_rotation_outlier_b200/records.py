@@ -30,7 +30,8 @@ KERNEL_SOURCES = {
               "k_chunk_dq4.cu", "k_chunk_dq8.cu", "k_chunk_mma.cu", "k_full4096.cu", "k_generic.cu",
               "hadq_dq_mma.cuh", "k_dq_mma.cu"],
     "attn": ["hadq_common.cuh", "hadq_attn.cuh", "k_attn.cu"],
-    "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "k_keep_rq.cu", "k_keep_dq.cu"],
+    "keep": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_chunk_mma.cuh", "k_keep_rq.cu",
+             "k_keep_dq.cu"],
     "asym": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_asym.cuh", "k_asym.cu"],
     "kron": ["hadq_common.cuh", "hadq_generic.cuh", "hadq_mma.cuh", "hadq_kron.cuh", "k_kron.cu"],
     "h4096": ["hadq_common.cuh", "hadq_chunk.cuh", "hadq_mma.cuh", "hadq_h4096.cuh", "k_h4096.cu"],

@@ -31,6 +31,12 @@ CASES = [
     (4, 77, 128, 32, 128, 4, True, (0, 0, ())),          # nothing kept
     (2, 40, 128, 128, -1, 8, False, (40, 0, ())),        # everything kept
     (2, 33, 512, 16, 256, 4, False, (3, 3, (17,))),
+    # block = group = 128: the tensor-core quantiser's kept-token instances
+    (2, 300, 128, 128, 128, 4, True, (4, 16, (50, 51, 200))),
+    (3, 97, 256, 128, 128, 8, False, (1, 8, (3,))),    # two blocks per row, ragged last slab
+    (2, 40, 128, 128, 128, 4, True, (40, 0, ())),       # everything kept
+    (5, 61, 384, 128, 128, 4, False, (0, 0, ())),       # nothing kept, three blocks per row
+    (1, 1, 128, 128, 128, 8, True, (1, 0, ())),         # one token, kept
 ]
 
 
