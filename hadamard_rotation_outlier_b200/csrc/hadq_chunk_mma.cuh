@@ -138,12 +138,22 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
   // the first slab is in flight while the CTA builds its sign table
   if (slab < nslabs) mma_slab_load<16>(xsrc + size_t(slab) * SB, slab_count(slab * kMmaSlab, a.nchunks, kMmaSlab), st0, lane);
   cp_async_commit();
-  int ks_next[2] = {-1, -1};  // KEEP: keep-table entries of blocks g, g + 8 of the next slab
+  // KEEP: keep-table entries of blocks g, g + 8 of the slab staged next.  The
+  // token (row mod tokens) and the block's place in its row are carried from
+  // slab to slab with adds, so that no division runs in the loop.
+  int ks_next[2] = {-1, -1};
+  int k_tok[2] = {0, 0}, k_col[2] = {0, 0};
+  int k_dr = 0, k_dt = 0;  // advance per slab step: blocks within a row, tokens
   if constexpr (KEEP) {
+    const uint32_t cpr = uint32_t(a.cpr), toks = uint32_t(a.keep_tokens), step = uint32_t(wstride) * kMmaSlab;
+    k_dr = int(step % cpr);
+    k_dt = int((step / cpr) % toks);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int ch = slab * kMmaSlab + g + 8 * r;
-      if (slab < nslabs && ch < a.nchunks) ks_next[r] = kept_slot_of(a, ch);
+      const uint32_t ch = uint32_t(slab * kMmaSlab + g + 8 * r);
+      k_col[r] = int(ch % cpr);
+      k_tok[r] = int((ch / cpr) % toks);
+      if (slab < nslabs && int(ch) < a.nchunks) ks_next[r] = __ldg(a.keep_slot + k_tok[r]);
     }
   }
   if constexpr (SIGNS) {
@@ -184,8 +194,13 @@ __global__ void __launch_bounds__(kMmaWarps * 32, 4) rq_chunk_mma_kernel(ChunkAr
       if constexpr (KEEP) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
+          k_col[r] += k_dr;
+          const int carry = k_col[r] >= a.cpr;
+          if (carry) k_col[r] -= a.cpr;
+          k_tok[r] += k_dt + carry;
+          if (k_tok[r] >= a.keep_tokens) k_tok[r] -= int(a.keep_tokens);
           const int ch = nx * kMmaSlab + g + 8 * r;
-          ks_next[r] = (nx < nslabs && ch < a.nchunks) ? kept_slot_of(a, ch) : -1;
+          ks_next[r] = (nx < nslabs && ch < a.nchunks) ? __ldg(a.keep_slot + k_tok[r]) : -1;
         }
       }
       const int n2 = nx + wstride;  // the slab after: into L2 now, staged next iteration
