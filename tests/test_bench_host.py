@@ -4,6 +4,7 @@ the committed DRAM-traffic lookup."""
 
 import json
 import os
+import re
 import sys
 
 import pytest
@@ -50,6 +51,28 @@ def test_every_workload_has_a_kernel_family_with_sources():
         assert R.workload_family(wl) in R.KERNEL_SOURCES
     for dw in S.DECODE_WORKLOADS.values():
         assert R.workload_family(dw) == "attn"
+
+
+def test_kernel_families_cover_every_included_header():
+    # a record stays valid only while its kernels' sources are unchanged, so a
+    # family must list every header its translation units include (directly
+    # or through other headers); the declarations header holds no device code
+    csrc = os.path.join(bench.ROOT, "hadamard_rotation_outlier_b200", "csrc")
+
+    def included(name, seen):
+        with open(os.path.join(csrc, name)) as f:
+            for h in re.findall(r'#include "([^"]+)"', f.read()):
+                if os.path.exists(os.path.join(csrc, h)) and h not in seen:
+                    seen.add(h)
+                    included(h, seen)
+        return seen
+
+    for fam, files in R.KERNEL_SOURCES.items():
+        need = set()
+        for f in files:
+            if f.endswith(".cu"):
+                need |= included(f, set())
+        assert not need - set(files) - {"hadq_kernels.h"}, (fam, sorted(need - set(files)))
 
 
 def test_records_follow_the_source_hash(tmp_path, monkeypatch):
